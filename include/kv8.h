@@ -1,0 +1,173 @@
+/*
+ * kv8.h -- C ABI of libkv8: paged INT8 KV-cache decode attention for B200
+ * (sm_100a).
+ *
+ * The method [KV-Cache 全栈优化系统, 主要特性 "低比特线性与 KV-cache 压缩"]:
+ * keys and values are quantised dynamically per token to INT8, kept
+ * compressed in the cache, and restored on demand inside attention.  The
+ * cache is paged [KV Cache 优化全景解析——从基础原理到工程实践, §4.2
+ * PagedAttention]: each sequence's logical 16-token blocks map through a
+ * block table to physically scattered blocks, and several sequences may list
+ * the same physical block (shared prefixes).  Query heads are grouped onto KV
+ * heads [same page, §3.3 GQA].  Decode attention is
+ * softmax(q K^T / sqrt(d)) V [same page, §2.1] with FP32 accumulation
+ * [大模型推理加速：KV Cache与vLLM技术解析, §4.1 混合精度计算].
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument except the stream is a DEVICE pointer owned by
+ *     the caller.  The library allocates nothing and keeps no state between
+ *     calls.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; a KV8_OK return means the
+ *     work was launched, not that it finished.
+ *   - Argument checks are made on the host before anything is launched; a
+ *     failed check launches nothing and returns KV8_ERR_INVALID_ARG,
+ *     KV8_ERR_UNSUPPORTED or KV8_ERR_WORKSPACE.  KV8_ERR_CUDA reports a launch
+ *     error (cudaGetLastError).  Nothing aborts, exits or traps.
+ *   - Device-resident indices (slot_mapping, block_tables, context_lens) are
+ *     trusted: they must lie in range (the caller's contract).
+ *   - Supported shapes: head_dim == 128, block_size == 16,
+ *     num_q_heads / num_kv_heads in {1, 2, 4, 8}; other values return
+ *     KV8_ERR_UNSUPPORTED.  Device pointers must be 16-byte aligned.
+ *
+ * Memory layout (row-major, innermost last)
+ *   k_cache, v_cache  int8    [num_blocks][num_kv_heads][block_size][head_dim]
+ *   k_scales,v_scales float32 [num_blocks][num_kv_heads][block_size]
+ *   One (block, kv_head) "page" is block_size*head_dim = 2048 contiguous code
+ *   bytes plus 64 contiguous scale bytes.  Token t of sequence b lives in
+ *   physical block block_tables[b][t / block_size] at offset t % block_size.
+ */
+#ifndef KV8_H
+#define KV8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define KV8_OK 0
+#define KV8_ERR_INVALID_ARG 1 /* null pointer, bad shape, misaligned buffer */
+#define KV8_ERR_UNSUPPORTED 2 /* valid but not built: head_dim, block, group */
+#define KV8_ERR_WORKSPACE 3   /* workspace missing or smaller than required */
+#define KV8_ERR_CUDA 4        /* a CUDA launch or attribute call failed */
+
+/* Output element types for kv8_paged_decode_attention / kv8_split_reduce. */
+#define KV8_OUT_BF16 0
+#define KV8_OUT_F32 1
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kv8_status_string(int32_t status);
+
+/*
+ * kv8_quantize_append -- quantise new K/V rows and store them in the cache.
+ *
+ * Defined by [KV-Cache 全栈优化系统, 主要特性]: per-token dynamic INT8
+ * quantisation, with the quantisation group one KV head's head_dim values
+ * [大模型推理加速, §4.1: quant group size 128].  For every token i and KV head
+ * h, separately for K and for V:
+ *     a = max_j |x_j|                      (exact, fp32)
+ *     s = a / 127 in IEEE fp32 (round to nearest even); s = 0 when a == 0
+ *     c_j = clamp(rint(x_j / s), -127, 127), x_j / s an IEEE fp32 division,
+ *           rint ties to even; c_j = 0 when s == 0
+ * Codes go to block slot_mapping[i] / block_size at offset
+ * slot_mapping[i] % block_size [KV Cache 优化全景解析, §4.2: the block table
+ * maps logical to physical blocks]; the scale goes beside them.
+ *
+ *   k_new, v_new   bf16 [n_tokens][num_kv_heads][head_dim], read only
+ *   slot_mapping   int64 [n_tokens]; slot < 0 means padding: token skipped
+ *   k_cache, v_cache, k_scales, v_scales   written at the mapped slots only
+ * The caller must not point two tokens at one slot in a call, nor point a
+ * slot at a block other sequences share (copy it first).
+ * n_tokens == 0 launches nothing and returns KV8_OK.
+ */
+int32_t kv8_quantize_append(const void *k_new, const void *v_new,
+                            const int64_t *slot_mapping, int64_t n_tokens,
+                            int32_t num_kv_heads, int32_t head_dim,
+                            int32_t block_size, int64_t num_blocks,
+                            int8_t *k_cache, int8_t *v_cache, float *k_scales,
+                            float *v_scales, void *stream);
+
+/*
+ * kv8_decode_workspace_bytes -- bytes of workspace a split launch needs.
+ *
+ * Workspace holds, per (sequence, query head, context chunk), the chunk's
+ * running max and sum (2 fp32) and its unnormalised output (head_dim fp32).
+ * Returns 0 when chunk_tokens == 0 or every context fits one chunk.
+ */
+size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                  int32_t head_dim, int32_t max_context_len,
+                                  int32_t chunk_tokens);
+
+/*
+ * kv8_paged_decode_attention -- one decode step of GQA attention over the
+ * paged INT8 cache, for one new query token per sequence.
+ *
+ * For sequence b and query head h (KV head h / (num_q_heads/num_kv_heads),
+ * [KV Cache 优化全景解析, §3.3]) over the n = context_lens[b] cached tokens
+ * t (the token appended this step included, [大模型推理加速, §2.1: append the
+ * new K/V, then attend over the whole cache]):
+ *     k_hat_t = kc_t * ks_t,  v_hat_t = vc_t * vs_t      (dequantise)
+ *     score_t = softmax_scale * <q, k_hat_t>
+ *     out     = sum_t softmax(score)_t * v_hat_t
+ * [KV Cache 优化全景解析, §2.1], accumulated in fp32 with an online softmax.
+ * n == 0 gives an all-zero output row.
+ *
+ *   q              bf16 [batch][num_q_heads][head_dim]
+ *   block_tables   int32 [batch][max_blocks_per_seq]; entries past
+ *                  ceil(n / block_size) are never read
+ *   context_lens   int32 [batch]; every value <= max_context_len
+ *   max_context_len  host-side bound on context_lens (sizes the grid);
+ *                  must be <= max_blocks_per_seq * block_size
+ *   softmax_scale  <= 0 selects 1/sqrt(head_dim)
+ *   chunk_tokens   0: one pass per (sequence, KV head), no workspace.
+ *                  > 0 (a multiple of block_size): the context is split into
+ *                  chunks of that many tokens processed in parallel; a
+ *                  sequence that fits one chunk writes `out` directly, the
+ *                  others write partials to `workspace` and this call then
+ *                  enqueues kv8_split_reduce on the same stream.
+ *   workspace      device buffer of >= kv8_decode_workspace_bytes(...) bytes
+ *                  (may be NULL when that is 0); contents are scratch
+ *   out            [batch][num_q_heads][head_dim] of bf16 (out_dtype ==
+ *                  KV8_OUT_BF16, round to nearest even) or fp32 (KV8_OUT_F32)
+ * The caches are only read; blocks may be shared between sequences.
+ */
+int32_t kv8_paged_decode_attention(
+    const void *q, const int8_t *k_cache, const int8_t *v_cache,
+    const float *k_scales, const float *v_scales, const int32_t *block_tables,
+    const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void *workspace,
+    size_t workspace_bytes, void *out, int32_t out_dtype, void *stream);
+
+/*
+ * kv8_split_reduce -- merge the per-chunk partials of a split decode launch.
+ *
+ * For each (b, h) whose context spans C = ceil(n / chunk_tokens) > 1 chunks,
+ * with chunk partials (m_c, l_c, o_c) written in base-2 exponent form
+ * (o_c = sum_t 2^(s_t - m_c) v_hat_t, l_c = sum_t 2^(s_t - m_c),
+ * s_t = score_t * log2(e)):
+ *     M = max_c m_c,  L = sum_c l_c 2^(m_c - M),
+ *     out = sum_c o_c 2^(m_c - M) / L
+ * i.e. the log-sum-exp merge of the chunk softmaxes.  Rows with C <= 1 are
+ * left untouched (the split launch wrote them).  kv8_paged_decode_attention
+ * calls this itself; it is exported for pipelining and for tests.
+ *
+ *   workspace      as written by a split launch with the same batch,
+ *                  num_q_heads, head_dim, max_context_len and chunk_tokens
+ *   context_lens   int32 [batch], the same values the split launch read
+ */
+int32_t kv8_split_reduce(const void *workspace, size_t workspace_bytes,
+                         const int32_t *context_lens, int32_t batch,
+                         int32_t num_q_heads, int32_t head_dim,
+                         int32_t max_context_len, int32_t chunk_tokens,
+                         void *out, int32_t out_dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KV8_H */

@@ -1,0 +1,142 @@
+"""CPU oracle for paged INT8 KV decode attention (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import this package.  The product path (the CUDA
+library under ``paged_int8_kv_b200``) never loads it, and the two share no
+code: this module wraps ``kv8_oracle.c`` (plain C, single threaded) with
+ctypes and adds nothing but argument marshalling.
+
+What each function computes, and the passage it follows, is stated in
+``kv8_oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kv8_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libkv8_oracle.so")
+
+ORACLE_OK = 0
+ORACLE_BAD_ARG = 1
+ORACLE_NONFINITE = 2
+ORACLE_NOMEM = 3
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile kv8_oracle.c into libkv8_oracle.so with gcc (no fast-math)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + ".tmp"
+    cmd = ["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math",
+           "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    P = ctypes.c_void_p
+    i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+    lib.oracle_quantize_append.restype = ctypes.c_int
+    lib.oracle_quantize_append.argtypes = [P, P, i64, i32, i32, i32, i64, P, P]
+    lib.oracle_decode_attention.restype = ctypes.c_int
+    lib.oracle_decode_attention.argtypes = [
+        P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, f64, P, i64, P]
+    lib.oracle_kv_cache_bytes.restype = f64
+    lib.oracle_kv_cache_bytes.argtypes = [i64] * 7
+    lib.oracle_kv8_scale_bytes.restype = f64
+    lib.oracle_kv8_scale_bytes.argtypes = [i64] * 4
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _check(rc: int, what: str):
+    if rc != ORACLE_OK:
+        raise ValueError(f"{what}: oracle status {rc}")
+
+
+def quantize_append(x_bf16: np.ndarray, slot_mapping: np.ndarray,
+                    cache: np.ndarray, scales: np.ndarray) -> None:
+    """Quantise x (uint16 bf16 bits, [n_tokens, H_kv, D]) into cache/scales in place.
+
+    cache: int8 [num_blocks, H_kv, block_size, D]; scales: float32
+    [num_blocks, H_kv, block_size].  Both must be C-contiguous.
+    """
+    lib = _load()
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    assert cache.dtype == np.int8 and cache.flags.c_contiguous
+    assert scales.dtype == np.float32 and scales.flags.c_contiguous
+    nb, hkv, bs, d = cache.shape
+    assert x.shape[1:] == (hkv, d) and sm.shape == (x.shape[0],)
+    assert scales.shape == (nb, hkv, bs)
+    rc = lib.oracle_quantize_append(_ptr(x), _ptr(sm), x.shape[0], hkv, d, bs,
+                                    nb, _ptr(cache), _ptr(scales))
+    _check(rc, "oracle_quantize_append")
+
+
+def decode_attention(q_bf16: np.ndarray, k_cache: np.ndarray,
+                     v_cache: np.ndarray, k_scales: np.ndarray,
+                     v_scales: np.ndarray, block_tables: np.ndarray,
+                     context_lens: np.ndarray, softmax_scale: float = 0.0,
+                     pairs=None) -> np.ndarray:
+    """fp64 decode attention over the dequantised paged cache.
+
+    q_bf16: uint16 [B, H_q, D].  Returns float64 [B, H_q, D], or
+    [len(pairs), D] when ``pairs`` (a list of (b, h)) is given.
+    """
+    lib = _load()
+    q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    for a in (k_cache, v_cache):
+        assert a.dtype == np.int8 and a.flags.c_contiguous
+    for a in (k_scales, v_scales):
+        assert a.dtype == np.float32 and a.flags.c_contiguous
+    B, hq, d = q.shape
+    nb, hkv, bs, d2 = k_cache.shape
+    assert d2 == d and v_cache.shape == k_cache.shape
+    assert bt.shape[0] == B and cl.shape == (B,)
+    if pairs is None:
+        out = np.zeros((B, hq, d), dtype=np.float64)
+        pp, npairs = None, 0
+    else:
+        pa = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+        npairs = pa.shape[0]
+        out = np.zeros((npairs, d), dtype=np.float64)
+        pp = _ptr(pa)
+    rc = lib.oracle_decode_attention(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales),
+        _ptr(bt), _ptr(cl), B, hq, hkv, d, bs, bt.shape[1], nb,
+        float(softmax_scale), pp, npairs, _ptr(out))
+    _check(rc, "oracle_decode_attention")
+    return out
+
+
+def kv_cache_bytes(layers: int, batch: int, seq_len: int, kv_heads: int,
+                   head_dim: int, bytes_num: int, bytes_den: int = 1) -> float:
+    """2*L*B*T*H_kv*d_h*bytes, bytes = bytes_num/bytes_den."""
+    return _load().oracle_kv_cache_bytes(layers, batch, seq_len, kv_heads,
+                                         head_dim, bytes_num, bytes_den)
+
+
+def kv8_scale_bytes(layers: int, batch: int, seq_len: int, kv_heads: int) -> float:
+    """Bytes of fp32 scales the INT8 cache adds (one per token, head, K/V)."""
+    return _load().oracle_kv8_scale_bytes(layers, batch, seq_len, kv_heads)

@@ -1,0 +1,257 @@
+/*
+ * kv8_oracle.c -- plain, slow, single-threaded CPU oracle for paged INT8 KV
+ * decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the smoke check and the bench's CPU-baseline
+ * leg use it.  It shares no code, header, table or helper with the CUDA
+ * library; it is written from the definitions on the source pages:
+ *
+ *   [KV-Cache 全栈优化系统, 主要特性 "低比特线性与 KV-cache 压缩"]
+ *       K/V are quantised dynamically per token to INT8, stored compressed and
+ *       restored on demand inside attention.
+ *   [大模型推理加速：KV Cache与vLLM技术解析, §4.1 混合精度计算]
+ *       quant group size 128 (one head_dim); attention accumulates in FP32.
+ *   [KV Cache 优化全景解析——从基础原理到工程实践, §2.1 formula
+ *    Attention(Q,K,V) = softmax(QK^T / sqrt(d_k)) V]
+ *   [same page, §3.3 GQA]   h query heads split into G groups sharing one K/V.
+ *   [same page, §4.2 PagedAttention]   logical blocks -> physical blocks via a
+ *       block table; several sequences may map to the same physical block.
+ *   [same page, §2.3 KV Cache 内存计算公式]
+ *       memory = 2 * L * B * T * H_kv * d_h * bytes_per_element.
+ *
+ * Readings where the pages are silent (all listed in the design notes):
+ *   - one scale per (token, KV head), s = fl32(max|x| / 127), stored as fp32;
+ *   - code = clamp(rint(fl32(x / s)), -127, 127), IEEE single division and
+ *     ties-to-even rounding; s = 0 and all codes 0 for an all-zero vector;
+ *   - attention is computed in fp64 over the dequantised cache
+ *     k_hat = code * scale (exact in double), softmax scale 1/sqrt(d);
+ *   - GQA grouping is contiguous: KV head = query head / (H_q / H_kv);
+ *   - a context of length 0 gives an all-zero output row.
+ *
+ * Layouts (the same ones the library documents, restated here on purpose):
+ *   x (bf16 bits)  [n_tokens][H_kv][D]
+ *   cache (int8)   [num_blocks][H_kv][block_size][D]
+ *   scales (fp32)  [num_blocks][H_kv][block_size]
+ *   q (bf16 bits)  [B][H_q][D]
+ *   block_tables   int32 [B][max_blocks_per_seq]
+ *   out (fp64)     [B][H_q][D]
+ *
+ * Build: gcc -O2 -std=c99 -ffp-contract=off -fPIC -shared (no fast-math).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_NONFINITE 2
+#define ORACLE_NOMEM 3
+
+/* bf16 is the top half of an IEEE binary32. */
+static float bf16_bits_to_float(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/*
+ * Quantise one tensor (K or V) of new tokens and write it into the paged
+ * cache through slot_mapping (slot = physical_block * block_size + offset;
+ * a negative slot means "padding, skip this token").
+ * Returns ORACLE_OK, ORACLE_BAD_ARG (slot out of range) or ORACLE_NONFINITE.
+ */
+int oracle_quantize_append(const uint16_t *x, const int64_t *slot_mapping,
+                           int64_t n_tokens, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t block_size,
+                           int64_t num_blocks, int8_t *cache, float *scales)
+{
+    if (n_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < n_tokens; ++i) {
+        int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        int64_t blk = slot / block_size;
+        int64_t off = slot % block_size;
+        if (blk >= num_blocks)
+            return ORACLE_BAD_ARG;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            const uint16_t *row = x + (i * num_kv_heads + h) * (int64_t)head_dim;
+            /* step 1-2: amax over the head's d values, exact in fp32 */
+            float a = 0.0f;
+            for (int32_t j = 0; j < head_dim; ++j) {
+                float v = bf16_bits_to_float(row[j]);
+                if (!isfinite(v))
+                    return ORACLE_NONFINITE;
+                float m = fabsf(v);
+                if (m > a)
+                    a = m;
+            }
+            /* step 3-4: the scale, one IEEE single division */
+            float s = (a == 0.0f) ? 0.0f : a / 127.0f;
+            int64_t base = (blk * num_kv_heads + h) * (int64_t)block_size + off;
+            int8_t *dst = cache + base * head_dim;
+            /* step 5-6: code = clamp(rint(x / s)) */
+            for (int32_t j = 0; j < head_dim; ++j) {
+                int code = 0;
+                if (s != 0.0f) {
+                    float y = bf16_bits_to_float(row[j]) / s;
+                    float r = nearbyintf(y); /* default mode: ties to even */
+                    if (r > 127.0f)
+                        r = 127.0f;
+                    if (r < -127.0f)
+                        r = -127.0f;
+                    code = (int)r;
+                }
+                dst[j] = (int8_t)code;
+            }
+            /* step 7: the scale beside the codes */
+            scales[base] = s;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Exact decode attention for one (sequence b, query head h), fp64.
+ * out_row receives head_dim doubles.
+ */
+static int attend_one(const uint16_t *q, const int8_t *k_cache,
+                      const int8_t *v_cache, const float *k_scales,
+                      const float *v_scales, const int32_t *block_tables,
+                      const int32_t *context_lens, int32_t num_q_heads,
+                      int32_t num_kv_heads, int32_t head_dim,
+                      int32_t block_size, int32_t max_blocks_per_seq,
+                      int64_t num_blocks, double softmax_scale, int32_t b,
+                      int32_t h, double *out_row)
+{
+    int32_t group = num_q_heads / num_kv_heads;
+    int32_t kvh = h / group;
+    int32_t n = context_lens[b];
+    for (int32_t j = 0; j < head_dim; ++j)
+        out_row[j] = 0.0;
+    if (n == 0)
+        return ORACLE_OK;
+    if (n < 0 || n > max_blocks_per_seq * block_size)
+        return ORACLE_BAD_ARG;
+
+    const uint16_t *qrow = q + ((int64_t)b * num_q_heads + h) * head_dim;
+    double *score = (double *)malloc(sizeof(double) * (size_t)n);
+    if (!score)
+        return ORACLE_NOMEM;
+
+    /* scores: softmax_scale * sum_j q_j * (kc * ks) */
+    double smax = -INFINITY;
+    for (int32_t t = 0; t < n; ++t) {
+        int64_t phys = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
+        int64_t off = t % block_size;
+        if (phys < 0 || phys >= num_blocks) {
+            free(score);
+            return ORACLE_BAD_ARG;
+        }
+        int64_t base = (phys * num_kv_heads + kvh) * (int64_t)block_size + off;
+        double ks = (double)k_scales[base];
+        const int8_t *kc = k_cache + base * head_dim;
+        double dot = 0.0;
+        for (int32_t j = 0; j < head_dim; ++j)
+            dot += (double)bf16_bits_to_float(qrow[j]) * ((double)kc[j] * ks);
+        score[t] = softmax_scale * dot;
+        if (score[t] > smax)
+            smax = score[t];
+    }
+    /* softmax weights and the weighted sum of dequantised V rows */
+    double denom = 0.0;
+    for (int32_t t = 0; t < n; ++t) {
+        score[t] = exp(score[t] - smax);
+        denom += score[t];
+    }
+    for (int32_t t = 0; t < n; ++t) {
+        int64_t phys = block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
+        int64_t off = t % block_size;
+        int64_t base = (phys * num_kv_heads + kvh) * (int64_t)block_size + off;
+        double vs = (double)v_scales[base];
+        const int8_t *vc = v_cache + base * head_dim;
+        double w = score[t] / denom;
+        for (int32_t j = 0; j < head_dim; ++j)
+            out_row[j] += w * ((double)vc[j] * vs);
+    }
+    free(score);
+    for (int32_t j = 0; j < head_dim; ++j)
+        if (!isfinite(out_row[j]))
+            return ORACLE_NONFINITE;
+    return ORACLE_OK;
+}
+
+/*
+ * Decode attention for a list of (b, h) pairs (pairs = 2*n_pairs int32, NULL
+ * meaning every pair in row-major order).  out holds n_pairs * head_dim
+ * doubles (B * H_q * head_dim when pairs == NULL).
+ * softmax_scale <= 0 selects 1/sqrt(head_dim).
+ */
+int oracle_decode_attention(const uint16_t *q, const int8_t *k_cache,
+                            const int8_t *v_cache, const float *k_scales,
+                            const float *v_scales, const int32_t *block_tables,
+                            const int32_t *context_lens, int32_t batch,
+                            int32_t num_q_heads, int32_t num_kv_heads,
+                            int32_t head_dim, int32_t block_size,
+                            int32_t max_blocks_per_seq, int64_t num_blocks,
+                            double softmax_scale, const int32_t *pairs,
+                            int64_t n_pairs, double *out)
+{
+    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_q_heads % num_kv_heads != 0)
+        return ORACLE_BAD_ARG;
+    if (softmax_scale <= 0.0)
+        softmax_scale = 1.0 / sqrt((double)head_dim);
+    int64_t count = pairs ? n_pairs : (int64_t)batch * num_q_heads;
+    for (int64_t p = 0; p < count; ++p) {
+        int32_t b, h;
+        if (pairs) {
+            b = pairs[2 * p];
+            h = pairs[2 * p + 1];
+        } else {
+            b = (int32_t)(p / num_q_heads);
+            h = (int32_t)(p % num_q_heads);
+        }
+        if (b < 0 || b >= batch || h < 0 || h >= num_q_heads)
+            return ORACLE_BAD_ARG;
+        int rc = attend_one(q, k_cache, v_cache, k_scales, v_scales,
+                            block_tables, context_lens, num_q_heads,
+                            num_kv_heads, head_dim, block_size,
+                            max_blocks_per_seq, num_blocks, softmax_scale, b, h,
+                            out + p * head_dim);
+        if (rc != ORACLE_OK)
+            return rc;
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * KV-cache size closed form [KV Cache 优化全景解析, §2.3]:
+ *   2 * L * B * T * H_kv * d_h * bytes_per_element,
+ * with bytes_per_element = elem_bytes_num / elem_bytes_den (INT4 = 1/2).
+ * Returned as a double (exact for every value below 2^53).
+ */
+double oracle_kv_cache_bytes(int64_t layers, int64_t batch, int64_t seq_len,
+                             int64_t kv_heads, int64_t head_dim,
+                             int64_t elem_bytes_num, int64_t elem_bytes_den)
+{
+    double elems = 2.0 * (double)layers * (double)batch * (double)seq_len *
+                   (double)kv_heads * (double)head_dim;
+    return elems * (double)elem_bytes_num / (double)elem_bytes_den;
+}
+
+/*
+ * Extra bytes the INT8 format spends on its fp32 scales: one per
+ * (K or V, layer, sequence, token, KV head).  Not part of the page formula.
+ */
+double oracle_kv8_scale_bytes(int64_t layers, int64_t batch, int64_t seq_len,
+                              int64_t kv_heads)
+{
+    return 2.0 * (double)layers * (double)batch * (double)seq_len *
+           (double)kv_heads * 4.0;
+}
