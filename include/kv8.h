@@ -43,6 +43,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define KV8_API __attribute__((visibility("default")))
+#else
+#define KV8_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -59,7 +65,7 @@ extern "C" {
 #define KV8_OUT_F32 1
 
 /* Human-readable name of a status code (static string, never NULL). */
-const char *kv8_status_string(int32_t status);
+KV8_API const char *kv8_status_string(int32_t status);
 
 /*
  * kv8_quantize_append -- quantise new K/V rows and store them in the cache.
@@ -83,7 +89,7 @@ const char *kv8_status_string(int32_t status);
  * slot at a block other sequences share (copy it first).
  * n_tokens == 0 launches nothing and returns KV8_OK.
  */
-int32_t kv8_quantize_append(const void *k_new, const void *v_new,
+KV8_API int32_t kv8_quantize_append(const void *k_new, const void *v_new,
                             const int64_t *slot_mapping, int64_t n_tokens,
                             int32_t num_kv_heads, int32_t head_dim,
                             int32_t block_size, int64_t num_blocks,
@@ -97,7 +103,7 @@ int32_t kv8_quantize_append(const void *k_new, const void *v_new,
  * running max and sum (2 fp32) and its unnormalised output (head_dim fp32).
  * Returns 0 when chunk_tokens == 0 or every context fits one chunk.
  */
-size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
+KV8_API size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
                                   int32_t head_dim, int32_t max_context_len,
                                   int32_t chunk_tokens);
 
@@ -134,7 +140,7 @@ size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
  *                  KV8_OUT_BF16, round to nearest even) or fp32 (KV8_OUT_F32)
  * The caches are only read; blocks may be shared between sequences.
  */
-int32_t kv8_paged_decode_attention(
+KV8_API int32_t kv8_paged_decode_attention(
     const void *q, const int8_t *k_cache, const int8_t *v_cache,
     const float *k_scales, const float *v_scales, const int32_t *block_tables,
     const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
@@ -160,11 +166,32 @@ int32_t kv8_paged_decode_attention(
  *                  num_q_heads, head_dim, max_context_len and chunk_tokens
  *   context_lens   int32 [batch], the same values the split launch read
  */
-int32_t kv8_split_reduce(const void *workspace, size_t workspace_bytes,
+KV8_API int32_t kv8_split_reduce(const void *workspace, size_t workspace_bytes,
                          const int32_t *context_lens, int32_t batch,
                          int32_t num_q_heads, int32_t head_dim,
                          int32_t max_context_len, int32_t chunk_tokens,
                          void *out, int32_t out_dtype, void *stream);
+
+/*
+ * kv8_set_decode_kernel -- choose how kv8_paged_decode_attention computes a
+ * page (process-wide, for tuning and for comparing the two forms):
+ *   0  automatic (default),
+ *   1  CUDA-core form: codes converted to fp32 in registers, fp32 FMA,
+ *   2  tensor-core form: codes converted exactly to fp16, q.k and p.v on
+ *      mma tiles with fp32 accumulation.
+ * Both compute the same function; results differ only by rounding order.
+ * Returns KV8_ERR_INVALID_ARG for any other value.  Not thread-safe with
+ * respect to concurrent decode calls.
+ */
+KV8_API int32_t kv8_set_decode_kernel(int32_t kind);
+
+/*
+ * kv8_read_device_status -- synchronise the current device, then read the
+ * library's sticky device status word (0 = clean; bit 0 = a kernel gave up
+ * waiting for one of its own shared-memory copies and skipped that work
+ * instead of hanging).  clear != 0 resets the word to 0 afterwards.
+ */
+KV8_API int32_t kv8_read_device_status(uint32_t *status, int32_t clear);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,33 @@
+"""paged_int8_kv_b200 -- paged INT8 KV-cache decode attention for B200.
+
+The computation lives in ``libkv8.so`` (CUDA for sm_100a, C ABI declared in
+``include/kv8.h``).  This package only loads that library and marshals
+arguments; see ``_binding`` for the functions, which carry the C names.
+
+    from paged_int8_kv_b200 import kv8_quantize_append, kv8_paged_decode_attention
+
+The library is loaded on first use of any of these names (so that
+``paged_int8_kv_b200.build`` can run before it exists); if it is missing or
+cannot be loaded, that first use raises ImportError.  There is no fallback.
+"""
+import importlib
+
+_BINDING_NAMES = {
+    "EXPORTED", "KV8_ERR_CUDA", "KV8_ERR_INVALID_ARG", "KV8_ERR_UNSUPPORTED",
+    "KV8_ERR_WORKSPACE", "KV8_OK", "KV8_OUT_BF16", "KV8_OUT_F32", "LIB_PATH",
+    "Kv8Error", "default_softmax_scale", "kv8_decode_workspace_bytes",
+    "kv8_paged_decode_attention", "kv8_quantize_append",
+    "kv8_read_device_status", "kv8_set_decode_kernel", "kv8_split_reduce",
+    "kv8_status_string",
+}
+_RUNTIME_NAMES = {"PagedKV8Cache", "fill_from_host"}
+
+__all__ = sorted(_BINDING_NAMES | _RUNTIME_NAMES)
+
+
+def __getattr__(name):
+    if name in _BINDING_NAMES:
+        return getattr(importlib.import_module("._binding", __name__), name)
+    if name in _RUNTIME_NAMES:
+        return getattr(importlib.import_module(".runtime", __name__), name)
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")

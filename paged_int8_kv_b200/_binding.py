@@ -1,0 +1,161 @@
+"""ctypes binding of libkv8 (include/kv8.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and does
+nothing but turn torch tensors into pointers and sizes, pass the current CUDA
+stream, and raise ``Kv8Error`` on a non-zero status.  All computation runs in
+the CUDA kernels of ``libkv8.so``; there is no Python or CPU fallback, and a
+missing or unloadable library raises at import of this module.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkv8.so")
+
+KV8_OK = 0
+KV8_ERR_INVALID_ARG = 1
+KV8_ERR_UNSUPPORTED = 2
+KV8_ERR_WORKSPACE = 3
+KV8_ERR_CUDA = 4
+KV8_OUT_BF16 = 0
+KV8_OUT_F32 = 1
+
+EXPORTED = (
+    "kv8_status_string",
+    "kv8_quantize_append",
+    "kv8_decode_workspace_bytes",
+    "kv8_paged_decode_attention",
+    "kv8_split_reduce",
+    "kv8_set_decode_kernel",
+    "kv8_read_device_status",
+)
+
+
+class Kv8Error(RuntimeError):
+    def __init__(self, func: str, status: int, name: str):
+        super().__init__(f"{func} failed: {name} ({status})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libkv8.so not found at {LIB_PATH}; build it with "
+            "`python -m paged_int8_kv_b200.build` (there is no fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    sz = ctypes.c_size_t
+    lib.kv8_status_string.restype = ctypes.c_char_p
+    lib.kv8_status_string.argtypes = [i32]
+    lib.kv8_quantize_append.restype = i32
+    lib.kv8_quantize_append.argtypes = [P, P, P, i64, i32, i32, i32, i64, P, P, P, P, P]
+    lib.kv8_decode_workspace_bytes.restype = sz
+    lib.kv8_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    lib.kv8_paged_decode_attention.restype = i32
+    lib.kv8_paged_decode_attention.argtypes = [
+        P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
+        P, sz, P, i32, P]
+    lib.kv8_split_reduce.restype = i32
+    lib.kv8_split_reduce.argtypes = [P, sz, P, i32, i32, i32, i32, i32, P, i32, P]
+    lib.kv8_set_decode_kernel.restype = i32
+    lib.kv8_set_decode_kernel.argtypes = [i32]
+    lib.kv8_read_device_status.restype = i32
+    lib.kv8_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
+    return lib
+
+
+lib = _load()
+
+
+def _check(func: str, status: int) -> None:
+    if status != KV8_OK:
+        raise Kv8Error(func, status, lib.kv8_status_string(status).decode())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _p(t) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def kv8_status_string(status: int) -> str:
+    return lib.kv8_status_string(status).decode()
+
+
+def kv8_quantize_append(k_new: torch.Tensor, v_new: torch.Tensor,
+                        slot_mapping: torch.Tensor, k_cache: torch.Tensor,
+                        v_cache: torch.Tensor, k_scales: torch.Tensor,
+                        v_scales: torch.Tensor, stream=None) -> None:
+    """k_new/v_new bf16 [n, H_kv, D]; slot_mapping int64 [n]; caches int8
+    [NB, H_kv, 16, D]; scales fp32 [NB, H_kv, 16] (all on the GPU)."""
+    nb, hkv, bs, d = k_cache.shape
+    _check("kv8_quantize_append", lib.kv8_quantize_append(
+        _p(k_new), _p(v_new), _p(slot_mapping), slot_mapping.shape[0], hkv, d,
+        bs, nb, _p(k_cache), _p(v_cache), _p(k_scales), _p(v_scales),
+        _stream(stream)))
+
+
+def kv8_decode_workspace_bytes(batch: int, num_q_heads: int, head_dim: int,
+                               max_context_len: int, chunk_tokens: int) -> int:
+    return int(lib.kv8_decode_workspace_bytes(batch, num_q_heads, head_dim,
+                                              max_context_len, chunk_tokens))
+
+
+def kv8_paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor,
+                               v_cache: torch.Tensor, k_scales: torch.Tensor,
+                               v_scales: torch.Tensor,
+                               block_tables: torch.Tensor,
+                               context_lens: torch.Tensor, out: torch.Tensor,
+                               max_context_len: int, chunk_tokens: int = 512,
+                               workspace: torch.Tensor | None = None,
+                               softmax_scale: float = 0.0,
+                               stream=None) -> torch.Tensor:
+    """q bf16 [B, H_q, D]; out bf16 or fp32 [B, H_q, D] (written in place)."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    out_dtype = KV8_OUT_F32 if out.dtype == torch.float32 else KV8_OUT_BF16
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("kv8_paged_decode_attention", lib.kv8_paged_decode_attention(
+        _p(q), _p(k_cache), _p(v_cache), _p(k_scales), _p(v_scales),
+        _p(block_tables), _p(context_lens), B, hq, hkv, d, bs,
+        block_tables.shape[1], nb, int(max_context_len), float(softmax_scale),
+        int(chunk_tokens), _p(workspace), ws_bytes, _p(out), out_dtype,
+        _stream(stream)))
+    return out
+
+
+def kv8_split_reduce(workspace: torch.Tensor, context_lens: torch.Tensor,
+                     out: torch.Tensor, max_context_len: int,
+                     chunk_tokens: int, stream=None) -> torch.Tensor:
+    B, hq, d = out.shape
+    out_dtype = KV8_OUT_F32 if out.dtype == torch.float32 else KV8_OUT_BF16
+    _check("kv8_split_reduce", lib.kv8_split_reduce(
+        _p(workspace), workspace.numel() * workspace.element_size(),
+        _p(context_lens), B, hq, d, int(max_context_len), int(chunk_tokens),
+        _p(out), out_dtype, _stream(stream)))
+    return out
+
+
+def kv8_set_decode_kernel(kind: int) -> None:
+    _check("kv8_set_decode_kernel", lib.kv8_set_decode_kernel(int(kind)))
+
+
+def kv8_read_device_status(clear: bool = True) -> int:
+    v = ctypes.c_uint32(0)
+    _check("kv8_read_device_status", lib.kv8_read_device_status(ctypes.byref(v), int(clear)))
+    return int(v.value)
+
+
+def default_softmax_scale(head_dim: int = 128) -> float:
+    return 1.0 / math.sqrt(head_dim)

@@ -1,0 +1,262 @@
+// kv8_api.cu -- the extern "C" entry points of libkv8 (declared, with their
+// contracts, in include/kv8.h): host-side argument checks, tensor-map
+// encoding for the TMA page copies, and kernel launches.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "../../include/kv8.h"
+#include "kv8_internal.h"
+
+namespace {
+
+using kv8::kBlockSize;
+using kv8::kHeadDim;
+
+bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+bool aligned4(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 3u) == 0;
+}
+
+bool group_supported(int32_t g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
+                                cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Tensor map over a code cache viewed as [num_blocks*H_kv pages][16 rows]
+// [128 bytes]: one box is one page, written to shared memory with the
+// 128-byte swizzle (16-byte chunk j of row r lands at chunk j ^ (r & 7)).
+bool encode_page_map(CUtensorMap* map, const int8_t* cache, int64_t pages) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim),
+                        static_cast<cuuint64_t>(kBlockSize),
+                        static_cast<cuuint64_t>(pages)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim),
+                           static_cast<cuuint64_t>(kHeadDim * kBlockSize)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kHeadDim),
+                       static_cast<cuuint32_t>(kBlockSize), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                  const_cast<int8_t*>(cache), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Effective split: chunk tokens and chunk count for a launch.
+void split_shape(int32_t max_context_len, int32_t chunk_tokens,
+                 int32_t* chunk_eff, int32_t* max_chunks) {
+  if (chunk_tokens <= 0) {
+    int32_t c = ((max_context_len + kBlockSize - 1) / kBlockSize) * kBlockSize;
+    *chunk_eff = c < kBlockSize ? kBlockSize : c;
+    *max_chunks = 1;
+  } else {
+    *chunk_eff = chunk_tokens;
+    int32_t mc = (max_context_len + chunk_tokens - 1) / chunk_tokens;
+    *max_chunks = mc < 1 ? 1 : mc;
+  }
+}
+
+int32_t g_decode_kernel = 0;  // 0 auto, 1 CUDA-core FMA, 2 tensor-core mma
+
+}  // namespace
+
+extern "C" {
+
+const char* kv8_status_string(int32_t status) {
+  switch (status) {
+    case KV8_OK: return "KV8_OK";
+    case KV8_ERR_INVALID_ARG: return "KV8_ERR_INVALID_ARG";
+    case KV8_ERR_UNSUPPORTED: return "KV8_ERR_UNSUPPORTED";
+    case KV8_ERR_WORKSPACE: return "KV8_ERR_WORKSPACE";
+    case KV8_ERR_CUDA: return "KV8_ERR_CUDA";
+    default: return "KV8_ERR_UNKNOWN";
+  }
+}
+
+int32_t kv8_quantize_append(const void* k_new, const void* v_new,
+                            const int64_t* slot_mapping, int64_t n_tokens,
+                            int32_t num_kv_heads, int32_t head_dim,
+                            int32_t block_size, int64_t num_blocks,
+                            int8_t* k_cache, int8_t* v_cache, float* k_scales,
+                            float* v_scales, void* stream) {
+  if (n_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0)
+    return KV8_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || block_size != kBlockSize)
+    return KV8_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return KV8_OK;
+  if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache || !k_scales ||
+      !v_scales)
+    return KV8_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned4(k_scales) || !aligned4(v_scales) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return KV8_ERR_INVALID_ARG;
+  if (n_tokens > (int64_t(1) << 40) / num_kv_heads) return KV8_ERR_UNSUPPORTED;
+  int rc = kv8::launch_quantize_append(
+      k_new, v_new, slot_mapping, n_tokens, num_kv_heads, k_cache, v_cache,
+      k_scales, v_scales, static_cast<cudaStream_t>(stream));
+  return rc == 0 ? KV8_OK : KV8_ERR_CUDA;
+}
+
+size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                  int32_t head_dim, int32_t max_context_len,
+                                  int32_t chunk_tokens) {
+  if (batch <= 0 || num_q_heads <= 0 || head_dim != kHeadDim ||
+      max_context_len <= 0 || chunk_tokens <= 0)
+    return 0;
+  int32_t chunk_eff, max_chunks;
+  split_shape(max_context_len, chunk_tokens, &chunk_eff, &max_chunks);
+  if (max_chunks <= 1) return 0;
+  return kv8::workspace_total_bytes(batch, num_q_heads, max_chunks);
+}
+
+int32_t kv8_paged_decode_attention(
+    const void* q, const int8_t* k_cache, const int8_t* v_cache,
+    const float* k_scales, const float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void* workspace,
+    size_t workspace_bytes, void* out, int32_t out_dtype, void* stream) {
+  // ---- shape checks
+  if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+      max_context_len < 0 || chunk_tokens < 0)
+    return KV8_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return KV8_ERR_INVALID_ARG;
+  if (out_dtype != KV8_OUT_BF16 && out_dtype != KV8_OUT_F32)
+    return KV8_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || block_size != kBlockSize)
+    return KV8_ERR_UNSUPPORTED;
+  if (!group_supported(num_q_heads / num_kv_heads)) return KV8_ERR_UNSUPPORTED;
+  if (chunk_tokens % block_size != 0) return KV8_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_context_len) >
+      static_cast<int64_t>(max_blocks_per_seq) * block_size)
+    return KV8_ERR_INVALID_ARG;
+  if (batch > 65535 || num_kv_heads > 65535) return KV8_ERR_UNSUPPORTED;
+  if (num_blocks > INT32_MAX / num_kv_heads) return KV8_ERR_UNSUPPORTED;
+  if (batch == 0) return KV8_OK;
+  // ---- pointer checks
+  if (!q || !k_cache || !v_cache || !k_scales || !v_scales || !block_tables ||
+      !context_lens || !out)
+    return KV8_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(k_scales) || !aligned16(v_scales) || !aligned4(block_tables) ||
+      !aligned4(context_lens) || !aligned16(out))
+    return KV8_ERR_INVALID_ARG;
+
+  int32_t chunk_eff, max_chunks;
+  split_shape(max_context_len, chunk_tokens, &chunk_eff, &max_chunks);
+  float* ws_ml = nullptr;
+  float* ws_o = nullptr;
+  if (max_chunks > 1) {
+    const size_t need = kv8::workspace_total_bytes(batch, num_q_heads, max_chunks);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace))
+      return KV8_ERR_WORKSPACE;
+    ws_ml = static_cast<float*>(workspace);
+    ws_o = reinterpret_cast<float*>(
+        static_cast<uint8_t*>(workspace) +
+        kv8::workspace_ml_bytes(batch, num_q_heads, max_chunks));
+  }
+
+  CUtensorMap tmk, tmv;
+  const int64_t pages = num_blocks * num_kv_heads;
+  if (!encode_page_map(&tmk, k_cache, pages) ||
+      !encode_page_map(&tmv, v_cache, pages))
+    return KV8_ERR_CUDA;
+
+  if (!(softmax_scale > 0.0f))
+    softmax_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)));
+  kv8::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.ws_ml = ws_ml;
+  p.ws_o = ws_o;
+  p.out = out;
+  p.batch = batch;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.chunk_tokens = chunk_eff;
+  p.max_chunks = max_chunks;
+  p.out_f32 = out_dtype == KV8_OUT_F32 ? 1 : 0;
+  p.q_scale = static_cast<float>(static_cast<double>(softmax_scale) *
+                                 1.4426950408889634074);  // log2(e)
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = kv8::launch_decode(p, tmk, tmv, g_decode_kernel, st);
+  if (rc == -2) return KV8_ERR_UNSUPPORTED;
+  if (rc != 0) return KV8_ERR_CUDA;
+  if (max_chunks > 1) {
+    rc = kv8::launch_split_reduce(ws_ml, ws_o, context_lens, batch, num_q_heads,
+                                  chunk_eff, max_chunks, out, p.out_f32, st);
+    if (rc != 0) return KV8_ERR_CUDA;
+  }
+  return KV8_OK;
+}
+
+int32_t kv8_split_reduce(const void* workspace, size_t workspace_bytes,
+                         const int32_t* context_lens, int32_t batch,
+                         int32_t num_q_heads, int32_t head_dim,
+                         int32_t max_context_len, int32_t chunk_tokens,
+                         void* out, int32_t out_dtype, void* stream) {
+  if (batch < 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+      chunk_tokens <= 0)
+    return KV8_ERR_INVALID_ARG;
+  if (out_dtype != KV8_OUT_BF16 && out_dtype != KV8_OUT_F32)
+    return KV8_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim) return KV8_ERR_UNSUPPORTED;
+  if (chunk_tokens % kBlockSize != 0) return KV8_ERR_INVALID_ARG;
+  if (batch == 0) return KV8_OK;
+  if (!context_lens || !out || !aligned16(out) || !aligned4(context_lens))
+    return KV8_ERR_INVALID_ARG;
+  int32_t chunk_eff, max_chunks;
+  split_shape(max_context_len, chunk_tokens, &chunk_eff, &max_chunks);
+  if (max_chunks <= 1) return KV8_OK;  // nothing was split
+  const size_t need = kv8::workspace_total_bytes(batch, num_q_heads, max_chunks);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return KV8_ERR_WORKSPACE;
+  const float* ws_ml = static_cast<const float*>(workspace);
+  const float* ws_o = reinterpret_cast<const float*>(
+      static_cast<const uint8_t*>(workspace) +
+      kv8::workspace_ml_bytes(batch, num_q_heads, max_chunks));
+  int rc = kv8::launch_split_reduce(
+      ws_ml, ws_o, context_lens, batch, num_q_heads, chunk_eff, max_chunks, out,
+      out_dtype == KV8_OUT_F32 ? 1 : 0, static_cast<cudaStream_t>(stream));
+  return rc == 0 ? KV8_OK : KV8_ERR_CUDA;
+}
+
+int32_t kv8_set_decode_kernel(int32_t kind) {
+  if (kind < 0 || kind > 2) return KV8_ERR_INVALID_ARG;
+  g_decode_kernel = kind;
+  return KV8_OK;
+}
+
+int32_t kv8_read_device_status(uint32_t* status, int32_t clear) {
+  if (!status) return KV8_ERR_INVALID_ARG;
+  return kv8::read_device_status(status, clear) == 0 ? KV8_OK : KV8_ERR_CUDA;
+}
+
+}  // extern "C"

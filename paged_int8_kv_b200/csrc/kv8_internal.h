@@ -1,0 +1,65 @@
+// kv8_internal.h -- launchers shared between the kv8 translation units.
+// Not part of the public ABI (include/kv8.h is).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kv8 {
+
+constexpr int kHeadDim = 128;
+constexpr int kBlockSize = 16;
+constexpr int kPageBytes = kHeadDim * kBlockSize;  // 2048 code bytes
+
+// Everything a decode launch needs besides the two tensor maps.
+struct DecodeParams {
+  const __nv_bfloat16* q;       // [B][Hq][128]
+  const float* k_scales;        // [NB][Hkv][16]
+  const float* v_scales;
+  const int32_t* block_tables;  // [B][MBS]
+  const int32_t* context_lens;  // [B]
+  float* ws_ml;                 // [B][Hq][max_chunks][2] (m, l), base-2
+  float* ws_o;                  // [B][Hq][max_chunks][128]
+  void* out;                    // [B][Hq][128] bf16 or f32
+  int32_t batch;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t max_blocks_per_seq;
+  int32_t chunk_tokens;  // > 0, multiple of 16
+  int32_t max_chunks;    // ceil(max_context_len / chunk_tokens)
+  int32_t out_f32;       // 1 = fp32 output, 0 = bf16
+  float q_scale;         // softmax_scale * log2(e)
+};
+
+// Workspace carve-up shared by the decode and reduce launchers.
+size_t workspace_ml_bytes(int32_t batch, int32_t num_q_heads,
+                          int32_t max_chunks);
+size_t workspace_total_bytes(int32_t batch, int32_t num_q_heads,
+                             int32_t max_chunks);
+
+int launch_quantize_append(const void* k_new, const void* v_new,
+                           const int64_t* slot_mapping, int64_t n_tokens,
+                           int32_t num_kv_heads, int8_t* k_cache,
+                           int8_t* v_cache, float* k_scales, float* v_scales,
+                           cudaStream_t stream);
+
+// Returns 0 on success, -1 on a CUDA error, -2 if the group size has no
+// compiled kernel.
+int launch_decode(const DecodeParams& p, const CUtensorMap& tmk,
+                  const CUtensorMap& tmv, int32_t variant,
+                  cudaStream_t stream);
+
+int launch_split_reduce(const float* ws_ml, const float* ws_o,
+                        const int32_t* context_lens, int32_t batch,
+                        int32_t num_q_heads, int32_t chunk_tokens,
+                        int32_t max_chunks, void* out, int32_t out_f32,
+                        cudaStream_t stream);
+
+// Reads (and optionally clears) the sticky device status word after a
+// device-wide synchronize.  Returns 0, or -1 on a CUDA error.
+int read_device_status(uint32_t* value, int clear);
+
+}  // namespace kv8

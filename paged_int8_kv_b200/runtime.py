@@ -1,0 +1,93 @@
+"""Device-memory owner for one layer's paged INT8 KV cache.
+
+``PagedKV8Cache`` allocates the four cache tensors (codes and scales for K
+and V, layout as in include/kv8.h) and a reusable split-K workspace with
+PyTorch, and forwards to the C entry points.  It is plumbing only: every
+number it produces comes from the CUDA kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _binding as B
+
+
+class PagedKV8Cache:
+    def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int = 128,
+                 block_size: int = 16, device: str | torch.device = "cuda",
+                 poison: bool = True):
+        self.num_blocks = int(num_blocks)
+        self.num_kv_heads = int(num_kv_heads)
+        self.head_dim = int(head_dim)
+        self.block_size = int(block_size)
+        self.device = torch.device(device)
+        shape = (self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim)
+        sshape = shape[:3]
+        self.k_cache = torch.empty(shape, dtype=torch.int8, device=self.device)
+        self.v_cache = torch.empty(shape, dtype=torch.int8, device=self.device)
+        self.k_scales = torch.empty(sshape, dtype=torch.float32, device=self.device)
+        self.v_scales = torch.empty(sshape, dtype=torch.float32, device=self.device)
+        if poison:
+            self.poison()
+        self._ws = None
+
+    def poison(self) -> None:
+        """Unwritten slots read as code 127 with a NaN scale."""
+        self.k_cache.fill_(127)
+        self.v_cache.fill_(127)
+        self.k_scales.fill_(float("nan"))
+        self.v_scales.fill_(float("nan"))
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size()
+                   for t in (self.k_cache, self.v_cache, self.k_scales, self.v_scales))
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor,
+               slot_mapping: torch.Tensor, stream=None) -> None:
+        B.kv8_quantize_append(k_new, v_new, slot_mapping, self.k_cache,
+                              self.v_cache, self.k_scales, self.v_scales,
+                              stream=stream)
+
+    def workspace(self, batch: int, num_q_heads: int, max_context_len: int,
+                  chunk_tokens: int) -> torch.Tensor | None:
+        need = B.kv8_decode_workspace_bytes(batch, num_q_heads, self.head_dim,
+                                            max_context_len, chunk_tokens)
+        if need == 0:
+            return None
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def decode(self, q: torch.Tensor, block_tables: torch.Tensor,
+               context_lens: torch.Tensor, max_context_len: int,
+               chunk_tokens: int = 512, out: torch.Tensor | None = None,
+               out_dtype: torch.dtype = torch.bfloat16,
+               softmax_scale: float = 0.0, stream=None) -> torch.Tensor:
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        ws = self.workspace(q.shape[0], q.shape[1], max_context_len, chunk_tokens)
+        return B.kv8_paged_decode_attention(
+            q, self.k_cache, self.v_cache, self.k_scales, self.v_scales,
+            block_tables, context_lens, out, max_context_len,
+            chunk_tokens=chunk_tokens, workspace=ws,
+            softmax_scale=softmax_scale, stream=stream)
+
+
+def fill_from_host(cache: PagedKV8Cache, segments, stream=None) -> int:
+    """Copy host (k, v, slot_mapping) segments to the GPU and append them.
+
+    ``segments`` yields numpy arrays: k and v as bf16 bit patterns (uint16)
+    [n, H_kv, D] and slot_mapping int64 [n].  Returns the number of tokens
+    appended.  Each segment is staged through pinned memory.
+    """
+    total = 0
+    for k, v, slots in segments:
+        n = int(slots.shape[0])
+        if n == 0:
+            continue
+        kt = torch.from_numpy(k).view(torch.bfloat16).pin_memory().to(cache.device, non_blocking=True)
+        vt = torch.from_numpy(v).view(torch.bfloat16).pin_memory().to(cache.device, non_blocking=True)
+        st = torch.from_numpy(slots).pin_memory().to(cache.device, non_blocking=True)
+        cache.append(kt, vt, st, stream=stream)
+        total += n
+    return total

@@ -1,0 +1,98 @@
+"""The C-ABI library loads without a GPU, exports every entry point the
+header declares, and rejects bad arguments on the host (no kernel runs)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_int8_kv_b200 import build
+    build.build()
+    return ctypes.CDLL(build.LIB)
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(kv8_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "kv8_paged_decode_attention" in names and len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_names_match_header():
+    import paged_int8_kv_b200 as pk
+    assert sorted(pk.EXPORTED) == _declared()
+    for n in pk.EXPORTED:
+        assert callable(getattr(pk, n))
+
+
+def test_status_strings():
+    import paged_int8_kv_b200 as pk
+    assert pk.kv8_status_string(0) == "KV8_OK"
+    assert pk.kv8_status_string(3) == "KV8_ERR_WORKSPACE"
+    assert pk.kv8_status_string(99) == "KV8_ERR_UNKNOWN"
+
+
+def test_workspace_bytes_closed_form():
+    import paged_int8_kv_b200 as pk
+    # batch 64, 32 q heads, 32K context, chunks of 512 -> 64 chunks
+    ws = pk.kv8_decode_workspace_bytes(64, 32, 128, 32768, 512)
+    ml = 64 * 32 * 64 * 2 * 4
+    assert ws == ((ml + 255) // 256) * 256 + 64 * 32 * 64 * 128 * 4
+    assert pk.kv8_decode_workspace_bytes(64, 32, 128, 512, 512) == 0
+    assert pk.kv8_decode_workspace_bytes(64, 32, 128, 32768, 0) == 0
+    assert pk.kv8_decode_workspace_bytes(64, 32, 64, 32768, 512) == 0
+
+
+def _decode(lib, **kw):
+    a = dict(q=16, kc=16, vc=16, ks=16, vs=16, bt=16, cl=16, batch=1, hq=8,
+             hkv=2, d=128, bs=16, mbs=4, nb=8, maxlen=64, scale=0.0, chunk=0,
+             ws=0, wsb=0, out=16, odt=0, stream=0)
+    a.update(kw)
+    f = lib.kv8_paged_decode_attention
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    f.restype = i32
+    f.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32,
+                  ctypes.c_float, i32, P, ctypes.c_size_t, P, i32, P]
+    return f(a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["bt"], a["cl"],
+             a["batch"], a["hq"], a["hkv"], a["d"], a["bs"], a["mbs"], a["nb"],
+             a["maxlen"], a["scale"], a["chunk"], a["ws"], a["wsb"], a["out"],
+             a["odt"], a["stream"])
+
+
+def test_host_validation_rejects_before_launch(lib):
+    # Every call below fails its host checks, so no pointer is dereferenced.
+    assert _decode(lib, d=64) == 2                 # head_dim unsupported
+    assert _decode(lib, bs=32) == 2                # block size unsupported
+    assert _decode(lib, hq=12, hkv=4) == 2         # group of 3 not built
+    assert _decode(lib, hq=8, hkv=3) == 1          # not a multiple
+    assert _decode(lib, maxlen=65) == 1            # > mbs * block_size
+    assert _decode(lib, chunk=24) == 1             # not a block multiple
+    assert _decode(lib, odt=7) == 1                # bad output dtype
+    assert _decode(lib, q=0) == 1                  # null pointer
+    assert _decode(lib, kc=8) == 1                 # misaligned cache
+    assert _decode(lib, chunk=16, maxlen=64) == 3  # split needs a workspace
+    assert _decode(lib, batch=0) == 0              # nothing to do
+    f = lib.kv8_quantize_append
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    f.restype = i32
+    f.argtypes = [P, P, P, i64, i32, i32, i32, i64, P, P, P, P, P]
+    assert f(16, 16, 16, 4, 2, 64, 16, 8, 16, 16, 16, 16, 0) == 2
+    assert f(16, 16, 16, -1, 2, 128, 16, 8, 16, 16, 16, 16, 0) == 1
+    assert f(16, 16, 16, 0, 2, 128, 16, 8, 16, 16, 16, 16, 0) == 0
+    assert f(0, 16, 16, 4, 2, 128, 16, 8, 16, 16, 16, 16, 0) == 1
+    assert lib.kv8_set_decode_kernel(5) == 1
