@@ -193,6 +193,44 @@ KV8_API int32_t kv8_set_decode_kernel(int32_t kind);
  */
 KV8_API int32_t kv8_read_device_status(uint32_t *status, int32_t clear);
 
+/*
+ * kv8_paged_decode_attention_noalloc -- kv8_paged_decode_attention for
+ * callers that cannot allocate device memory.
+ *
+ * The source pages have no counterpart for this entry point; it exists for
+ * callers that cannot hand the split-K decode a workspace: code running
+ * inside a framework that owns every byte of device memory (a serving engine
+ * that reserves almost the whole GPU for its KV pool up front, a plugin whose
+ * host offers no workspace), or latency-critical code that must not call
+ * cudaMalloc because it can synchronise the device.
+ *
+ * Arguments and results are those of kv8_paged_decode_attention without
+ * `workspace` / `workspace_bytes`: the caller still passes every input and
+ * the output.  The chunk partials go to a fixed scratch array inside the
+ * library, KV8_NOALLOC_WORKSPACE_BYTES long, which every GPU that loads the
+ * library holds until the process exits.  Nothing is allocated or freed.
+ *   - Limit: a launch whose split needs more than
+ *     KV8_NOALLOC_WORKSPACE_BYTES (kv8_decode_workspace_bytes(...) of the
+ *     same arguments) returns KV8_ERR_WORKSPACE and launches nothing; use a
+ *     larger chunk_tokens (fewer chunks) or the allocating entry point.
+ *   - The first call on each device looks up the array's device address on
+ *     that device (cudaGetSymbolAddress); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents;
+ *     nothing in it has to start at zero.  Calls whose kernels overlap on the
+ *     GPU (e.g. on unordered streams) race on it: order them.
+ */
+#define KV8_NOALLOC_WORKSPACE_BYTES (16u << 20) /* 16 MiB per device */
+
+KV8_API int32_t kv8_paged_decode_attention_noalloc(
+    const void *q, const int8_t *k_cache, const int8_t *v_cache,
+    const float *k_scales, const float *v_scales, const int32_t *block_tables,
+    const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void *out, int32_t out_dtype,
+    void *stream);
+
 #ifdef __cplusplus
 }
 #endif

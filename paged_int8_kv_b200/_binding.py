@@ -33,6 +33,7 @@ EXPORTED = (
     "kv8_split_reduce",
     "kv8_set_decode_kernel",
     "kv8_read_device_status",
+    "kv8_paged_decode_attention_noalloc",
 )
 
 
@@ -64,6 +65,10 @@ def _load() -> ctypes.CDLL:
     lib.kv8_split_reduce.argtypes = [P, sz, P, i32, i32, i32, i32, i32, P, i32, P]
     lib.kv8_set_decode_kernel.restype = i32
     lib.kv8_set_decode_kernel.argtypes = [i32]
+    lib.kv8_paged_decode_attention_noalloc.restype = i32
+    lib.kv8_paged_decode_attention_noalloc.argtypes = [
+        P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
+        P, i32, P]
     lib.kv8_read_device_status.restype = i32
     lib.kv8_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
     return lib
@@ -132,6 +137,31 @@ def kv8_paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor,
         block_tables.shape[1], nb, int(max_context_len), float(softmax_scale),
         int(chunk_tokens), _p(workspace), ws_bytes, _p(out), out_dtype,
         _stream(stream)))
+    return out
+
+
+def kv8_paged_decode_attention_noalloc(q: torch.Tensor, k_cache: torch.Tensor,
+                                       v_cache: torch.Tensor,
+                                       k_scales: torch.Tensor,
+                                       v_scales: torch.Tensor,
+                                       block_tables: torch.Tensor,
+                                       context_lens: torch.Tensor,
+                                       out: torch.Tensor, max_context_len: int,
+                                       chunk_tokens: int = 512,
+                                       softmax_scale: float = 0.0,
+                                       stream=None) -> torch.Tensor:
+    """Like kv8_paged_decode_attention, for callers that cannot allocate:
+    the split partials use the library's fixed per-device scratch array."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    out_dtype = KV8_OUT_F32 if out.dtype == torch.float32 else KV8_OUT_BF16
+    _check("kv8_paged_decode_attention_noalloc",
+           lib.kv8_paged_decode_attention_noalloc(
+               _p(q), _p(k_cache), _p(v_cache), _p(k_scales), _p(v_scales),
+               _p(block_tables), _p(context_lens), B, hq, hkv, d, bs,
+               block_tables.shape[1], nb, int(max_context_len),
+               float(softmax_scale), int(chunk_tokens), _p(out), out_dtype,
+               _stream(stream)))
     return out
 
 
