@@ -289,8 +289,16 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     sampler = ClockSampler(uuid)
     barrier()
     torch.cuda.synchronize()
+    # clocks: the sampler starts under the same load (untimed steps for about
+    # a second) so that its samples cover the timed region and the load
+    # leading into it
     sampler.start()
-    time.sleep(0.3)
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < 1.0:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize()
+    barrier()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
