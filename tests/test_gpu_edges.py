@@ -42,17 +42,61 @@ def _ref(oracle_mod, w):
                                        w.context_lens)
 
 
+@pytest.mark.parametrize("kind", [1, 2], ids=["cudacore", "tensorcore"])
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (8, 2), (16, 2), (4, 1)])
 @pytest.mark.parametrize("chunk", [0, 16, 512])
-def test_ragged_groups_chunks(pk, oracle_mod, hq, hkv, chunk):
+def test_ragged_groups_chunks(pk, oracle_mod, hq, hkv, chunk, kind):
     w = W.make_workload("ragged", 2000 + hq * 10 + hkv, RAGGED, hq, hkv,
                         extra_blocks=7, outliers=(3, 10.0), chunk_tokens=chunk)
     ref = _ref(oracle_mod, w)
     cache, q, bt, cl = U.device_inputs(w)
-    for dt, bf in ((torch.float32, False), (torch.bfloat16, True)):
-        gpu = U.gpu_decode(cache, q, bt, cl, w, chunk_tokens=chunk, out_dtype=dt)
-        U.assert_close(gpu, ref, bf16=bf)
-        assert np.all(gpu[0] == 0.0)  # empty context -> zeros
+    pk.kv8_set_decode_kernel(kind)
+    try:
+        for dt, bf in ((torch.float32, False), (torch.bfloat16, True)):
+            gpu = U.gpu_decode(cache, q, bt, cl, w, chunk_tokens=chunk,
+                               out_dtype=dt)
+            U.assert_close(gpu, ref, bf16=bf)
+            if not bf:
+                assert np.abs(gpu - ref).max() < 1e-4
+            assert np.all(gpu[0] == 0.0)  # empty context -> zeros
+    finally:
+        pk.kv8_set_decode_kernel(0)
+
+
+@pytest.mark.parametrize("scale", [2.0 ** -40, 1.0, 2.0 ** 20])
+def test_tensorcore_extreme_magnitudes(pk, oracle_mod, scale):
+    # q and V far from unit scale exercise the power-of-two normalisation of
+    # q and of the fp16 probabilities in the tensor-core form
+    w = W.make_workload("mag", 2100, [700, 64, 1], 16, 4, extra_blocks=2)
+    q = W.bf16_bits_to_f32(w.q()) * np.float32(scale)
+    w._q = W.f32_to_bf16_bits(q)
+    base = w.private_kv
+
+    def scaled(b, _base=base):
+        k, v = _base(b)
+        vf = W.bf16_bits_to_f32(v) * np.float32(1.0 / scale if scale > 1 else scale)
+        return k, W.f32_to_bf16_bits(vf)
+    w.private_kv = scaled
+    ref = _ref(oracle_mod, w)
+    cache, qd, bt, cl = U.device_inputs(w)
+    for kind in (1, 2):
+        pk.kv8_set_decode_kernel(kind)
+        gpu = U.gpu_decode(cache, qd, bt, cl, w, chunk_tokens=256)
+        denom = max(np.abs(ref).max(), 1e-30)
+        assert np.abs(gpu - ref).max() / denom < 1e-4, kind
+    pk.kv8_set_decode_kernel(0)
+
+
+def test_tensorcore_matches_cudacore(pk):
+    w = W.make_workload("kinds", 2200, [5000, 3000, 17], 64, 8, extra_blocks=1,
+                        outliers=(4, 8.0))
+    cache, q, bt, cl = U.device_inputs(w)
+    outs = []
+    for kind in (1, 2):
+        pk.kv8_set_decode_kernel(kind)
+        outs.append(U.gpu_decode(cache, q, bt, cl, w, chunk_tokens=512))
+    pk.kv8_set_decode_kernel(0)
+    assert np.abs(outs[0] - outs[1]).max() < 1e-4
 
 
 def test_block_permutation_bit_identical(pk):
