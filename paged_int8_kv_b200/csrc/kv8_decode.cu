@@ -271,12 +271,16 @@ struct SimtMath {
 
 // Tensor-core form (mma.sync m16n8k16, fp16 operands, fp32 accumulation).
 // Per 16-token page a warp computes
-//   S[16 x 16]   = q'[16 x 128] . K_code^T     rows = query heads (>= G: 0)
+//   S^T[16 x 8]   = K_code[16 x 128] . q'^T[128 x 8]    rows = the 16 tokens
 //   O^T[128 x 8] += V_code^T[128 x 16] . P''^T[16 x 8]   cols = query heads
-// i.e. 2 n-tiles x 8 k-steps for the scores and 8 m-tiles x (hi, lo) for
-// the output.  Thread (r = lane/4, c = lane%4) holds, after the q.k mma,
-// the scores of head r for tokens {2c, 2c+1, 8+2c, 9+2c}: exactly its B
-// fragment of P''^T for the p.v mma, so no data moves between lanes.
+// i.e. 8 k-steps for the scores and 8 m-tiles x (hi, lo) for the output;
+// columns >= G carry zero q and are never stored.  Thread (r = lane/4,
+// c = lane%4) owns, in both products, heads 2c and 2c+1: it holds their
+// scores for tokens r and 8+r, keeps their running max, and holds their
+// O^T columns, so the softmax bookkeeping never leaves the thread except
+// on a (rare) change of the reference max.  P'' moves from the S^T layout
+// to the B-operand layout of the p.v mma with two 8x8 movmatrix transposes
+// per fp16 half.
 // Exactness of the operands:
 //   * codes -> fp16 exactly: the byte c+128 is placed under the fp16
 //     exponent of 1024, giving 1152 + c exactly, then 1152 is subtracted;
@@ -302,6 +306,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0,
       "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 8x8 transpose of 16-bit elements held in the mma fragment layout.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
@@ -360,16 +371,17 @@ __device__ __forceinline__ uint32_t word_of(const uint4& a, int i) {
 
 template <int G>
 struct MmaMath {
-  int lane, r, c;
-  uint32_t qa[8], qb[8];
-  float qfac;      // 2^e * softmax_scale * log2(e), head r
-  float ot[8][4];  // O^T fragments: heads 2c, 2c+1 at two dims per m-tile
-  float m_run, l_run;
-  int e_run;       // P'' carries 2^-e_run
-  float vlim;      // 2^(e_run + kVSlack)
-  float fs;        // 2^-e_run
   static constexpr float kSlack = 8.0f;  // log2 units
   static constexpr int kVSlack = 4;
+  int lane, r, c;
+  uint2 qk[8];      // B fragments of q'^T (head r): k-step s
+  float qf0, qf1;   // score factors of heads 2c, 2c+1
+  float ot[8][4];   // O^T fragments: heads 2c, 2c+1 at two dims per m-tile
+  float m0, m1;     // reference max of heads 2c, 2c+1 (base 2)
+  float l0, l1;     // this thread's partial sums of heads 2c, 2c+1
+  int e_run;        // P'' carries 2^-e_run (warp-uniform)
+  float vlim;       // 2^(e_run + kVSlack)
+  float fs;         // 2^-e_run
 
   __device__ __forceinline__ void init(const __nv_bfloat16* qg, float q_scale,
                                        int lane_) {
@@ -404,16 +416,19 @@ struct MmaMath {
     const float f1 = pow2i(sh / 2), f2 = pow2i(sh - sh / 2);
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
-      qa[s] = pack_h2(qv[4 * s + 0] * f1 * f2, qv[4 * s + 2] * f1 * f2);
-      qb[s] = pack_h2(qv[4 * s + 1] * f1 * f2, qv[4 * s + 3] * f1 * f2);
+      qk[s].x = pack_h2(qv[4 * s + 0] * f1 * f2, qv[4 * s + 2] * f1 * f2);
+      qk[s].y = pack_h2(qv[4 * s + 1] * f1 * f2, qv[4 * s + 3] * f1 * f2);
     }
-    qfac = q_scale * pow2i(-(sh / 2)) * pow2i(-(sh - sh / 2));
+    const float qf = q_scale * pow2i(-(sh / 2)) * pow2i(-(sh - sh / 2));
+    // this thread's score columns are heads 2c and 2c+1 (quads 2c, 2c+1)
+    qf0 = __shfl_sync(kFull, qf, 8 * c);
+    qf1 = __shfl_sync(kFull, qf, 8 * c + 4);
     reset();
   }
 
   __device__ __forceinline__ void reset() {
-    m_run = -INFINITY;
-    l_run = 0.0f;
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.0f;
     e_run = -126;
     vlim = 0.0f;
     fs = 1.0f;
@@ -426,8 +441,7 @@ struct MmaMath {
   __device__ __forceinline__ void page(const uint8_t* tk, const uint8_t* tv,
                                        const float* ks, const float* vs,
                                        int nv) {
-    // ---- S = q' K^T: n-tile 0 = tokens 0..7 (this thread: token r),
-    //                  n-tile 1 = tokens 8..15 (token 8 + r)
+    // ---- S^T = K q'^T: rows r (token r) and r+8 (token 8+r)
     const uint8_t* ra = tk + r * 128;
     const uint8_t* rb = tk + (8 + r) * 128;
     const int sw = r & 7;  // (8 + r) & 7 == r & 7
@@ -435,93 +449,94 @@ struct MmaMath {
     const uint4 ka1 = *reinterpret_cast<const uint4*>(ra + (((2 * c + 1) ^ sw) << 4));
     const uint4 kb0 = *reinterpret_cast<const uint4*>(rb + (((2 * c) ^ sw) << 4));
     const uint4 kb1 = *reinterpret_cast<const uint4*>(rb + (((2 * c + 1) ^ sw) << 4));
-    float s0[4] = {0.f, 0.f, 0.f, 0.f};
-    float s1[4] = {0.f, 0.f, 0.f, 0.f};
+    float st[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
-      uint32_t e0, o0, e1, o1;
-      k_word_to_h2(word_of(s < 4 ? ka0 : ka1, s & 3), e0, o0);
-      k_word_to_h2(word_of(s < 4 ? kb0 : kb1, s & 3), e1, o1);
-      mma16816(s0, qa[s], 0u, qb[s], 0u, e0, o0);
-      mma16816(s1, qa[s], 0u, qb[s], 0u, e1, o1);
+      uint32_t ea, oa, eb, ob;
+      k_word_to_h2(word_of(s < 4 ? ka0 : ka1, s & 3), ea, oa);
+      k_word_to_h2(word_of(s < 4 ? kb0 : kb1, s & 3), eb, ob);
+      mma16816(st, ea, eb, oa, ob, qk[s].x, qk[s].y);
     }
-    // this thread's tokens: 2c, 2c+1 (s0[0..1]) and 8+2c, 9+2c (s1[0..1])
-    const int t0 = 2 * c, t2 = 8 + 2 * c;
-    const float2 ksa = *reinterpret_cast<const float2*>(ks + t0);
-    const float2 ksb = *reinterpret_cast<const float2*>(ks + t2);
-    const float2 vsa = *reinterpret_cast<const float2*>(vs + t0);
-    const float2 vsb = *reinterpret_cast<const float2*>(vs + t2);
-    const bool v0 = t0 < nv, v1 = t0 + 1 < nv, v2 = t2 < nv, v3 = t2 + 1 < nv;
+    // st: [0] token r head 2c, [1] token r head 2c+1,
+    //     [2] token 8+r head 2c, [3] token 8+r head 2c+1
+    const bool va = r < nv, vb = 8 + r < nv;
+    const float ksa = ks[r], ksb = ks[8 + r];
+    const float vsa = va ? vs[r] : 0.0f, vsb = vb ? vs[8 + r] : 0.0f;
     float sc[4];
-    sc[0] = v0 ? s0[0] * qfac * ksa.x : -INFINITY;
-    sc[1] = v1 ? s0[1] * qfac * ksa.y : -INFINITY;
-    sc[2] = v2 ? s1[0] * qfac * ksb.x : -INFINITY;
-    sc[3] = v3 ? s1[1] * qfac * ksb.y : -INFINITY;
-    float vsv[4];
-    vsv[0] = v0 ? vsa.x : 0.0f;
-    vsv[1] = v1 ? vsa.y : 0.0f;
-    vsv[2] = v2 ? vsb.x : 0.0f;
-    vsv[3] = v3 ? vsb.y : 0.0f;
+    sc[0] = va ? st[0] * qf0 * ksa : -INFINITY;
+    sc[1] = va ? st[1] * qf1 * ksa : -INFINITY;
+    sc[2] = vb ? st[2] * qf0 * ksb : -INFINITY;
+    sc[3] = vb ? st[3] * qf1 * ksb : -INFINITY;
 
-    // Lazy rescaling: the reference max m_run (per head) and the exponent
-    // e_run (per warp) move only when a score exceeds m_run + kSlack or a
-    // V scale exceeds 2^(e_run + kVSlack); otherwise probabilities up to
-    // 2^kSlack are accumulated against the stale reference, which keeps
-    // every P'' below 2^(kSlack + kVSlack) (inside the fp16 range).
-    const float lmax = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-    const float lvmax = fmaxf(fmaxf(vsv[0], vsv[1]), fmaxf(vsv[2], vsv[3]));
-    const bool move = lmax > m_run + kSlack || lvmax > vlim;
+    // Lazy rescaling: the reference maxima (per head) and the exponent
+    // e_run (per warp) move only when a score exceeds its reference by
+    // more than kSlack or a V scale exceeds 2^(e_run + kVSlack); otherwise
+    // probabilities up to 2^kSlack are accumulated against the stale
+    // reference, which keeps every P'' below 2^(kSlack + kVSlack).
+    const float lm0 = fmaxf(sc[0], sc[2]);
+    const float lm1 = fmaxf(sc[1], sc[3]);
+    const float lv = fmaxf(vsa, vsb);
+    const bool move = lm0 > m0 + kSlack || lm1 > m1 + kSlack || lv > vlim;
     if (__any_sync(kFull, move)) {
-      float mx = fmaxf(lmax, __shfl_xor_sync(kFull, lmax, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-      float vmax = fmaxf(lvmax, __shfl_xor_sync(kFull, lvmax, 1));
-      vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, 2));
-      const float m_new = fmaxf(m_run, mx);
-      // every lane holds the same 16 tokens' scales: e_new is warp-uniform
-      const int e_new = vmax > vlim ? exp_frexp(vmax) : e_run;
-      const float a_l = (m_new == m_run) ? 1.0f : ex2(m_run - m_new);
-      const float a_o = a_l * pow2i(max(e_run - e_new, -126));
-      l_run *= a_l;
-      m_run = m_new;
+      float x0 = lm0, x1 = lm1, vx = lv;
+#pragma unroll
+      for (int m = 4; m < 32; m <<= 1) {
+        x0 = fmaxf(x0, __shfl_xor_sync(kFull, x0, m));
+        x1 = fmaxf(x1, __shfl_xor_sync(kFull, x1, m));
+        vx = fmaxf(vx, __shfl_xor_sync(kFull, vx, m));
+      }
+      const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+      // every lane sees the same 16 tokens' scales: e_new is warp-uniform
+      const int e_new = vx > vlim ? exp_frexp(vx) : e_run;
+      const float ef = pow2i(max(e_run - e_new, -126));
+      const float a0 = (n0 == m0) ? 1.0f : ex2(m0 - n0);
+      const float a1 = (n1 == m1) ? 1.0f : ex2(m1 - n1);
+      l0 *= a0;
+      l1 *= a1;
+      m0 = n0;
+      m1 = n1;
       e_run = e_new;
       vlim = pow2i(min(e_new + kVSlack, 127));
       fs = pow2i(-e_new);
-      const float ae = __shfl_sync(kFull, a_o, 8 * c);      // head 2c
-      const float ao = __shfl_sync(kFull, a_o, 8 * c + 4);  // head 2c+1
+      const float b0 = a0 * ef, b1 = a1 * ef;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        ot[i][0] *= ae;
-        ot[i][1] *= ao;
-        ot[i][2] *= ae;
-        ot[i][3] *= ao;
+        ot[i][0] *= b0;
+        ot[i][1] *= b1;
+        ot[i][2] *= b0;
+        ot[i][3] *= b1;
       }
     }
-    const float m_use = m_run == -INFINITY ? 0.0f : m_run;
-    float pr[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) pr[i] = ex2(sc[i] - m_use);
-    l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
-    float pp[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) pp[i] = pr[i] * (vsv[i] * fs);
-    const uint32_t h0 = pack_h2(pp[0], pp[1]);
-    const uint32_t h2 = pack_h2(pp[2], pp[3]);
-    const float2 f0 = unpack_h2(h0);
-    const float2 f2 = unpack_h2(h2);
-    const uint32_t l0 = pack_h2(pp[0] - f0.x, pp[1] - f0.y);
-    const uint32_t l2 = pack_h2(pp[2] - f2.x, pp[3] - f2.y);
+    const float u0 = m0 == -INFINITY ? 0.0f : m0;
+    const float u1 = m1 == -INFINITY ? 0.0f : m1;
+    const float p0 = ex2(sc[0] - u0), p1 = ex2(sc[1] - u1);
+    const float p2 = ex2(sc[2] - u0), p3 = ex2(sc[3] - u1);
+    l0 += p0 + p2;
+    l1 += p1 + p3;
+    const float wa = vsa * fs, wb = vsb * fs;
+    const float q0 = p0 * wa, q1 = p1 * wa, q2 = p2 * wb, q3 = p3 * wb;
+    // fp16 hi/lo in the S^T layout (rows = tokens, cols = heads) ...
+    const uint32_t ha = pack_h2(q0, q1), hb = pack_h2(q2, q3);
+    const float2 fa = unpack_h2(ha), fb = unpack_h2(hb);
+    const uint32_t la = pack_h2(q0 - fa.x, q1 - fa.y);
+    const uint32_t lb = pack_h2(q2 - fb.x, q3 - fb.y);
+    // ... transposed to B fragments of P''^T: head r, tokens {2c, 2c+1}
+    // (tokens 0..7 matrix) and {8+2c, 9+2c} (tokens 8..15 matrix)
+    const uint32_t h0 = movmatrix_t(ha), h2 = movmatrix_t(hb);
+    const uint32_t g0 = movmatrix_t(la), g2 = movmatrix_t(lb);
 
     // ---- O^T += V^T P''^T: tokens 2c, 2c+1, 8+2c, 9+2c, 16-byte chunk r
+    const int t0 = 2 * c, t2 = 8 + 2 * c;
     const int cr0 = (r ^ (2 * c)) << 4;      // tokens 2c and 8+2c
     const int cr1 = (r ^ (2 * c + 1)) << 4;  // tokens 2c+1 and 9+2c
-    const uint4 va = *reinterpret_cast<const uint4*>(tv + t0 * 128 + cr0);
-    const uint4 vb = *reinterpret_cast<const uint4*>(tv + (t0 + 1) * 128 + cr1);
-    const uint4 vc = *reinterpret_cast<const uint4*>(tv + t2 * 128 + cr0);
-    const uint4 vd = *reinterpret_cast<const uint4*>(tv + (t2 + 1) * 128 + cr1);
+    const uint4 vA = *reinterpret_cast<const uint4*>(tv + t0 * 128 + cr0);
+    const uint4 vB = *reinterpret_cast<const uint4*>(tv + (t0 + 1) * 128 + cr1);
+    const uint4 vC = *reinterpret_cast<const uint4*>(tv + t2 * 128 + cr0);
+    const uint4 vD = *reinterpret_cast<const uint4*>(tv + (t2 + 1) * 128 + cr1);
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      const uint32_t A = word_of(va, w), B = word_of(vb, w);
-      const uint32_t C = word_of(vc, w), D = word_of(vd, w);
+      const uint32_t A = word_of(vA, w), B = word_of(vB, w);
+      const uint32_t C = word_of(vC, w), D = word_of(vD, w);
       const uint32_t X = prmt(A, B, 0x5140u) ^ 0x80808080u;  // bytes 0,1
       const uint32_t Y = prmt(A, B, 0x7362u) ^ 0x80808080u;  // bytes 2,3
       const uint32_t Z = prmt(C, D, 0x5140u) ^ 0x80808080u;
@@ -531,22 +546,25 @@ struct MmaMath {
         const uint32_t a0 = v_pair(X, 0x4140u), a1 = v_pair(X, 0x4342u);
         const uint32_t a2 = v_pair(Z, 0x4140u), a3 = v_pair(Z, 0x4342u);
         mma16816(ot[2 * w], a0, a1, a2, a3, h0, h2);
-        mma16816(ot[2 * w], a0, a1, a2, a3, l0, l2);
+        mma16816(ot[2 * w], a0, a1, a2, a3, g0, g2);
       }
       // m-tile 2w+1: rows r / r+8 = byte 2 / byte 3
       {
         const uint32_t a0 = v_pair(Y, 0x4140u), a1 = v_pair(Y, 0x4342u);
         const uint32_t a2 = v_pair(U, 0x4140u), a3 = v_pair(U, 0x4342u);
         mma16816(ot[2 * w + 1], a0, a1, a2, a3, h0, h2);
-        mma16816(ot[2 * w + 1], a0, a1, a2, a3, l0, l2);
+        mma16816(ot[2 * w + 1], a0, a1, a2, a3, g0, g2);
       }
     }
   }
 
   __device__ __forceinline__ void record(float* rec) {
-    float l = l_run;
-    l += __shfl_xor_sync(kFull, l, 1);
-    l += __shfl_xor_sync(kFull, l, 2);
+    float s0 = l0, s1 = l1;
+#pragma unroll
+    for (int m = 4; m < 32; m <<= 1) {
+      s0 += __shfl_xor_sync(kFull, s0, m);
+      s1 += __shfl_xor_sync(kFull, s1, m);
+    }
     const float f = pow2i(e_run);
     const int h0 = 2 * c, h1 = 2 * c + 1;
 #pragma unroll
@@ -563,9 +581,15 @@ struct MmaMath {
         rec[h1 * kD + dB] = ot[i][3] * f;
       }
     }
-    if (r < G && c == 0) {
-      rec[G * kD + r] = m_run;
-      rec[G * kD + G + r] = l;
+    if (r == 0) {
+      if (h0 < G) {
+        rec[G * kD + h0] = m0;
+        rec[G * kD + G + h0] = s0;
+      }
+      if (h1 < G) {
+        rec[G * kD + h1] = m1;
+        rec[G * kD + G + h1] = s1;
+      }
     }
   }
 };
