@@ -3,8 +3,9 @@
 
 A step is one pass of the whole hot path over one decode batch:
 kv8_quantize_append of the batch's new K/V tokens, then
-kv8_paged_decode_attention (split-K kernel + split reduce) over every
-sequence's paged INT8 cache.  The default workload is the Llama-3.1-8B layer
+kv8_paged_decode_attention (one split-K kernel whose last chunk per
+sequence and KV head merges the partials) over every sequence's paged INT8
+cache.  The default workload is the Llama-3.1-8B layer
 shape at batch 64 with 32768-token contexts (4.43 GB of codes and scales,
 larger than L2, read once per step).
 
@@ -259,7 +260,10 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     ab = algorithmic_bytes(w)
     if ab["total"] <= 4 * 126e6:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    launches_per_step = 2 + (1 if (ws is not None) else 0)
+    # per step: the quantize-append kernel and the decode kernel (a split
+    # launch also enqueues a small memset of its merge tickets)
+    launches_per_step = 2
+    memsets_per_step = 1 if ws is not None else 0
 
     def step():
         cache.append(k_new, v_new, slots)
@@ -402,13 +406,15 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
                      "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                                     if peak_kind == "measured" else "fallback 6650 GB/s",
-                     "kernel": "kv8_paged_decode_attention (split kernel + split reduce)",
+                     "kernel": "decode_kernel (split-K pages + fused chunk merge), "
+                               "timed as the kv8_paged_decode_attention call",
                      "algorithmic_bytes": ab["total"],
                      "traffic": recorded_traffic(w.name)},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
+        "memsets": memsets_per_step * args.steps,
         "clocks": clocks,
         "device_status": status,
         "cpu_baseline": cpu,

@@ -100,7 +100,8 @@ KV8_API int32_t kv8_quantize_append(const void *k_new, const void *v_new,
  * kv8_decode_workspace_bytes -- bytes of workspace a split launch needs.
  *
  * Workspace holds, per (sequence, query head, context chunk), the chunk's
- * running max and sum (2 fp32) and its unnormalised output (head_dim fp32).
+ * running max and sum (2 fp32) and its unnormalised output (head_dim fp32),
+ * plus one 32-bit merge ticket per (sequence, query head).
  * Returns 0 when chunk_tokens == 0 or every context fits one chunk.
  */
 KV8_API size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
@@ -132,8 +133,11 @@ KV8_API size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
  *                  > 0 (a multiple of block_size): the context is split into
  *                  chunks of that many tokens processed in parallel; a
  *                  sequence that fits one chunk writes `out` directly, the
- *                  others write partials to `workspace` and this call then
- *                  enqueues kv8_split_reduce on the same stream.
+ *                  others write per-chunk partials to `workspace`, and the
+ *                  last chunk of each (sequence, KV head) to finish merges
+ *                  them into `out` in the same kernel (the merge that
+ *                  kv8_split_reduce performs).  The call enqueues a memset
+ *                  of the merge tickets and one kernel.
  *   workspace      device buffer of >= kv8_decode_workspace_bytes(...) bytes
  *                  (may be NULL when that is 0); contents are scratch
  *   out            [batch][num_q_heads][head_dim] of bf16 (out_dtype ==
@@ -160,7 +164,9 @@ KV8_API int32_t kv8_paged_decode_attention(
  *     out = sum_c o_c 2^(m_c - M) / L
  * i.e. the log-sum-exp merge of the chunk softmaxes.  Rows with C <= 1 are
  * left untouched (the split launch wrote them).  kv8_paged_decode_attention
- * calls this itself; it is exported for pipelining and for tests.
+ * performs this merge inside its own kernel; this entry point re-runs it
+ * from the partials a split launch left in the workspace (for pipelining
+ * and for tests), with the same arithmetic in the same order.
  *
  *   workspace      as written by a split launch with the same batch,
  *                  num_q_heads, head_dim, max_context_len and chunk_tokens

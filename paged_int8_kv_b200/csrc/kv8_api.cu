@@ -168,14 +168,17 @@ int32_t kv8_paged_decode_attention(
   split_shape(max_context_len, chunk_tokens, &chunk_eff, &max_chunks);
   float* ws_ml = nullptr;
   float* ws_o = nullptr;
+  uint32_t* ws_ctr = nullptr;
   if (max_chunks > 1) {
     const size_t need = kv8::workspace_total_bytes(batch, num_q_heads, max_chunks);
     if (!workspace || workspace_bytes < need || !aligned16(workspace))
       return KV8_ERR_WORKSPACE;
-    ws_ml = static_cast<float*>(workspace);
-    ws_o = reinterpret_cast<float*>(
-        static_cast<uint8_t*>(workspace) +
-        kv8::workspace_ml_bytes(batch, num_q_heads, max_chunks));
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    const size_t ml_bytes = kv8::workspace_ml_bytes(batch, num_q_heads, max_chunks);
+    const size_t o_bytes = kv8::workspace_o_bytes(batch, num_q_heads, max_chunks);
+    ws_ml = reinterpret_cast<float*>(base);
+    ws_o = reinterpret_cast<float*>(base + ml_bytes);
+    ws_ctr = reinterpret_cast<uint32_t*>(base + ml_bytes + o_bytes);
   }
 
   CUtensorMap tmk, tmv;
@@ -194,6 +197,7 @@ int32_t kv8_paged_decode_attention(
   p.context_lens = context_lens;
   p.ws_ml = ws_ml;
   p.ws_o = ws_o;
+  p.ws_ctr = ws_ctr;
   p.out = out;
   p.batch = batch;
   p.num_q_heads = num_q_heads;
@@ -206,14 +210,13 @@ int32_t kv8_paged_decode_attention(
                                  1.4426950408889634074);  // log2(e)
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (ws_ctr &&
+      cudaMemsetAsync(ws_ctr, 0, kv8::workspace_ctr_bytes(batch, num_q_heads),
+                      st) != cudaSuccess)
+    return KV8_ERR_CUDA;
   int rc = kv8::launch_decode(p, tmk, tmv, g_decode_kernel, st);
   if (rc == -2) return KV8_ERR_UNSUPPORTED;
   if (rc != 0) return KV8_ERR_CUDA;
-  if (max_chunks > 1) {
-    rc = kv8::launch_split_reduce(ws_ml, ws_o, context_lens, batch, num_q_heads,
-                                  chunk_eff, max_chunks, out, p.out_f32, st);
-    if (rc != 0) return KV8_ERR_CUDA;
-  }
   return KV8_OK;
 }
 

@@ -97,6 +97,97 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, float v,
     static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
 }
 
+// Hardware base-2 exponential (MUFU), relative error ~2^-22; -inf -> 0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^e for e in [-126, 127], built from the exponent bits.
+__device__ __forceinline__ float pow2i(int e) {
+  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+}
+
+// For x > 0 normal: the e with x = f * 2^e, f in [0.5, 1); x <= 2^-126 -> -125.
+__device__ __forceinline__ int exp_frexp(float x) {
+  const int be = static_cast<int>((__float_as_uint(x) >> 23) & 0xFF);
+  return be == 0 ? -125 : be - 126;
+}
+
+// Log-sum-exp merge of one query head's C chunk partials into its output
+// row: chunk c holds m_c (base-2 max), l_c (sum of 2^(s - m_c)) and o_c[d]
+// (sum of 2^(s - m_c) v_hat[d]);
+//   M = max_c m_c,  L = sum_c l_c 2^(m_c - M),
+//   out[d] = sum_c o_c[d] 2^(m_c - M) / L.
+// Called by every thread of a CTA of NW warps (it synchronises the CTA);
+// `red` is NW*128 + 2 floats of shared memory.  Warp 0 finds M and L; then
+// warp w sums chunks w, w + NW, ... for 4 dims per lane with float4 loads,
+// and warp 0 adds the NW partial sums.  The fused merge of a split decode
+// and the standalone reduce kernel both use it with the same NW, so they
+// produce identical results.
+template <int NW>
+__device__ __forceinline__ void merge_head(const float* ml, const float* o,
+                                           int nchunks, void* out,
+                                           int64_t out_row, int out_f32,
+                                           float* red) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    float mx = -INFINITY;
+    for (int c = lane; c < nchunks; c += 32) mx = fmaxf(mx, __ldcg(&ml[2 * c]));
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1)
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+    float ls = 0.0f;
+    for (int c = lane; c < nchunks; c += 32) {
+      const float mc = __ldcg(&ml[2 * c]);
+      ls += (mc == -INFINITY) ? 0.0f : __ldcg(&ml[2 * c + 1]) * ex2(mc - mx);
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) ls += __shfl_xor_sync(kFull, ls, m);
+    if (lane == 0) {
+      red[NW * kD] = mx;
+      red[NW * kD + 1] = ls;
+    }
+  }
+  __syncthreads();
+  const float M = red[NW * kD];
+  const float L = red[NW * kD + 1];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int c = warp; c < nchunks; c += NW) {
+    const float mc = __ldcg(&ml[2 * c]);
+    const float w = (mc == -INFINITY) ? 0.0f : ex2(mc - M);
+    const float4 v =
+        __ldcg(reinterpret_cast<const float4*>(o + static_cast<int64_t>(c) * kD) + lane);
+    acc.x += w * v.x;
+    acc.y += w * v.y;
+    acc.z += w * v.z;
+    acc.w += w * v.w;
+  }
+  *reinterpret_cast<float4*>(&red[warp * kD + 4 * lane]) = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float4 sum = *reinterpret_cast<const float4*>(&red[4 * lane]);
+#pragma unroll
+    for (int w = 1; w < NW; ++w) {
+      const float4 t = *reinterpret_cast<const float4*>(&red[w * kD + 4 * lane]);
+      sum.x += t.x;
+      sum.y += t.y;
+      sum.z += t.z;
+      sum.w += t.w;
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    const int64_t base = out_row * kD + 4 * lane;
+    store_out(out, base + 0, sum.x * inv, out_f32);
+    store_out(out, base + 1, sum.y * inv, out_f32);
+    store_out(out, base + 2, sum.z * inv, out_f32);
+    store_out(out, base + 3, sum.w * inv, out_f32);
+  }
+  __syncthreads();
+}
+
 // --------------------------------------------------------------------------
 // Page math.  A policy object holds one warp's running state over the pages
 // it is dealt in a chunk:
@@ -330,24 +421,6 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_h2(uint32_t v) {
   __half2 h = *reinterpret_cast<__half2*>(&v);
   return __half22float2(h);
-}
-
-// Hardware base-2 exponential (MUFU), relative error ~2^-22; -inf -> 0.
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// 2^e for e in [-126, 127], built from the exponent bits.
-__device__ __forceinline__ float pow2i(int e) {
-  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-}
-
-// For x > 0 normal: the e with x = f * 2^e, f in [0.5, 1); x <= 2^-126 -> -125.
-__device__ __forceinline__ int exp_frexp(float x) {
-  const int be = static_cast<int>((__float_as_uint(x) >> 23) & 0xFF);
-  return be == 0 ? -125 : be - 126;
 }
 
 constexpr uint32_t kBias1152 = 0x64806480u;  // fp16 (1152, 1152)
@@ -729,36 +802,51 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       }
     }
   }
+  if (single) return;
+
+  // ---- split: the last CTA of this (sequence, KV group) to finish merges
+  // every chunk's partial (threadfence-then-ticket; no CTA ever waits).
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned int ticket = atomicAdd(
+        &p.ws_ctr[static_cast<int64_t>(b) * p.num_q_heads + kvh * G], 1u);
+    s_last = ticket == static_cast<unsigned int>(nchunks - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float* red = reinterpret_cast<float*>(smem);  // records no longer needed
+  for (int h = 0; h < G; ++h) {
+    const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + kvh * G + h;
+    merge_head<NW>(p.ws_ml + bh * p.max_chunks * 2,
+                   p.ws_o + bh * p.max_chunks * kD, nchunks, p.out, bh,
+                   p.out_f32, red);
+  }
 }
 
 // --------------------------------------------------------------------------
-// Split reduce: one CTA of 128 threads (one per output dim) per (b, hq).
+// Standalone split reduce: one CTA of kReduceNW warps per (b, hq), the same
+// merge routine (and warp count) as the fused merge of the decode kernel.
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(128)
+constexpr int kReduceNW = 4;
+
+__global__ void __launch_bounds__(kReduceNW * 32)
 split_reduce_kernel(const float* __restrict__ ws_ml,
                     const float* __restrict__ ws_o,
                     const int32_t* __restrict__ context_lens, int32_t num_q_heads,
                     int32_t chunk_tokens, int32_t max_chunks, void* out,
                     int32_t out_f32) {
+  __shared__ __align__(16) float red[kReduceNW * kD + 2];
   const int bh = blockIdx.x;
   const int b = bh / num_q_heads;
   const int n = context_lens[b];
   const int nchunks = (n + chunk_tokens - 1) / chunk_tokens;
   if (nchunks <= 1) return;
-  const int d = threadIdx.x;
-  const float* ml = ws_ml + static_cast<int64_t>(bh) * max_chunks * 2;
-  const float* o = ws_o + static_cast<int64_t>(bh) * max_chunks * kD;
-  float M = -INFINITY;
-  for (int c = 0; c < nchunks; ++c) M = fmaxf(M, ml[2 * c]);
-  float L = 0.0f, O = 0.0f;
-  for (int c = 0; c < nchunks; ++c) {
-    const float mc = ml[2 * c];
-    const float e = (mc == -INFINITY) ? 0.0f : exp2f(mc - M);
-    L += ml[2 * c + 1] * e;
-    O += o[static_cast<int64_t>(c) * kD + d] * e;
-  }
-  store_out(out, static_cast<int64_t>(bh) * kD + d, L > 0.0f ? O / L : 0.0f,
-            out_f32);
+  merge_head<kReduceNW>(ws_ml + static_cast<int64_t>(bh) * max_chunks * 2,
+                        ws_o + static_cast<int64_t>(bh) * max_chunks * kD,
+                        nchunks, out, bh, out_f32, red);
 }
 
 template <int G, int NW, int SPW, class Math>
@@ -787,6 +875,7 @@ int launch_group(const DecodeParams& p, const CUtensorMap& tmk,
   // fastest for the tensor-core form on all of them.
   if (variant == 1)
     return launch_decode_kernel<G, 4, 4, SimtMath<G>>(p, tmk, tmv, stream);
+  static_assert(kReduceNW == 4, "fused and standalone merges must match");
   return launch_decode_kernel<G, 4, 2, MmaMath<G>>(p, tmk, tmv, stream);
 }
 
@@ -813,11 +902,21 @@ size_t workspace_ml_bytes(int32_t batch, int32_t num_q_heads,
   return (ml + 255) & ~size_t(255);
 }
 
+size_t workspace_o_bytes(int32_t batch, int32_t num_q_heads,
+                         int32_t max_chunks) {
+  return static_cast<size_t>(batch) * num_q_heads * max_chunks * kD *
+         sizeof(float);
+}
+
+size_t workspace_ctr_bytes(int32_t batch, int32_t num_q_heads) {
+  return static_cast<size_t>(batch) * num_q_heads * sizeof(uint32_t);
+}
+
 size_t workspace_total_bytes(int32_t batch, int32_t num_q_heads,
                              int32_t max_chunks) {
   return workspace_ml_bytes(batch, num_q_heads, max_chunks) +
-         static_cast<size_t>(batch) * num_q_heads * max_chunks * kD *
-             sizeof(float);
+         workspace_o_bytes(batch, num_q_heads, max_chunks) +
+         workspace_ctr_bytes(batch, num_q_heads);
 }
 
 int launch_decode(const DecodeParams& p, const CUtensorMap& tmk,
@@ -840,7 +939,7 @@ int launch_split_reduce(const float* ws_ml, const float* ws_o,
                         cudaStream_t stream) {
   const int64_t nbh = static_cast<int64_t>(batch) * num_q_heads;
   if (nbh == 0) return 0;
-  split_reduce_kernel<<<static_cast<unsigned>(nbh), kD, 0, stream>>>(
+  split_reduce_kernel<<<static_cast<unsigned>(nbh), kReduceNW * 32, 0, stream>>>(
       ws_ml, ws_o, context_lens, num_q_heads, chunk_tokens, max_chunks, out,
       out_f32);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;

@@ -23,6 +23,8 @@ struct DecodeParams {
   const int32_t* context_lens;  // [B]
   float* ws_ml;                 // [B][Hq][max_chunks][2] (m, l), base-2
   float* ws_o;                  // [B][Hq][max_chunks][128]
+  uint32_t* ws_ctr;             // [B][Hq] tickets (index b*Hq + first head
+                                // of the KV group), zero at launch
   void* out;                    // [B][Hq][128] bf16 or f32
   int32_t batch;
   int32_t num_q_heads;
@@ -37,6 +39,9 @@ struct DecodeParams {
 // Workspace carve-up shared by the decode and reduce launchers.
 size_t workspace_ml_bytes(int32_t batch, int32_t num_q_heads,
                           int32_t max_chunks);
+size_t workspace_o_bytes(int32_t batch, int32_t num_q_heads,
+                         int32_t max_chunks);
+size_t workspace_ctr_bytes(int32_t batch, int32_t num_q_heads);
 size_t workspace_total_bytes(int32_t batch, int32_t num_q_heads,
                              int32_t max_chunks);
 

@@ -51,8 +51,10 @@ def test_workspace_bytes_closed_form():
     import paged_int8_kv_b200 as pk
     # batch 64, 32 q heads, 32K context, chunks of 512 -> 64 chunks
     ws = pk.kv8_decode_workspace_bytes(64, 32, 128, 32768, 512)
-    ml = 64 * 32 * 64 * 2 * 4
-    assert ws == ((ml + 255) // 256) * 256 + 64 * 32 * 64 * 128 * 4
+    ml = 64 * 32 * 64 * 2 * 4          # (m, l) per (sequence, head, chunk)
+    o = 64 * 32 * 64 * 128 * 4         # unnormalised output per chunk
+    tickets = 64 * 32 * 4              # one merge ticket per (sequence, head)
+    assert ws == ((ml + 255) // 256) * 256 + o + tickets
     assert pk.kv8_decode_workspace_bytes(64, 32, 128, 512, 512) == 0
     assert pk.kv8_decode_workspace_bytes(64, 32, 128, 32768, 0) == 0
     assert pk.kv8_decode_workspace_bytes(64, 32, 64, 32768, 512) == 0
