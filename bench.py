@@ -158,6 +158,21 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def max_over_ranks(vals, dist=None, device=None):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    if dist is None:
+        return list(vals)
+    import torch
+    t = torch.tensor(list(vals), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Units all ranks processed per second, over the slowest rank's time."""
+    return units_per_rank * world / (ms_per_step * 1e-3)
+
+
 # ------------------------------------------------------------- CPU oracle
 def oracle_sample_seconds(w: W.Workload, seqs) -> tuple[float, str]:
     """Time the oracle's decode step (append of the new token + attention
@@ -370,17 +385,14 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     barrier()
 
     # ---- max over ranks
-    if dist is not None:
-        t = torch.tensor([ms, dms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, dms, e2e_ms = t.tolist()
+    ms, dms, e2e_ms = max_over_ranks([ms, dms, e2e_ms], dist, dev)
 
     status = pk.kv8_read_device_status(clear=True)
     if rank != 0:
         return 0
 
     tokens = w.batch * world
-    value = tokens / (ms * 1e-3)
+    value = whole_job_rate(w.batch, world, ms)
     peak, peak_kind = measured_peaks()
     achieved = ab["total"] / (dms * 1e-3) / 1e9
     cpu = None
@@ -410,7 +422,7 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
                                "timed as the kv8_paged_decode_attention call",
                      "algorithmic_bytes": ab["total"],
                      "traffic": recorded_traffic(w.name)},
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
+        "e2e": {"value": whole_job_rate(w.batch, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
