@@ -7,10 +7,10 @@
 // v_hat = code * vs), out = softmax(q k_hat^T / sqrt(d)) v_hat, with fp32
 // accumulation [大模型推理加速：KV Cache与vLLM技术解析, §4.1].
 //
-// Work decomposition (one CTA per (context chunk, KV head, sequence)):
-//   * The chunk's 16-token pages are dealt round-robin to NW warps.  Each
-//     warp owns SPW shared-memory slots and streams its own pages through
-//     them: lane 0 resolves the page through the block table
+// Work decomposition (persistent CTAs of independent warps; one work item =
+// one (sequence, KV head, context chunk), handled by one warp):
+//   * A warp owns SPW shared-memory slots and streams its items' 16-token
+//     pages through them: lane 0 resolves each page through the block table
 //     [KV Cache 优化全景解析, §4.2] and issues two TMA tensor copies (the
 //     2 KB K page and the 2 KB V page, 128-byte swizzled so that the
 //     column reads below are bank-conflict free) plus two 64-byte bulk
@@ -23,10 +23,10 @@
 //     fp32 in registers, folds the token's K scale into the score, keeps a
 //     base-2 online softmax (running max m and sum l per head), folds the
 //     token's V scale into the probability and accumulates o += p * vc.
-//   * At the end of the chunk the NW warp states are merged through shared
-//     memory.  A sequence that fits one chunk writes the normalised output;
-//     otherwise (m, l, o) go to the workspace and kv8_split_reduce merges
-//     the chunks with a log-sum-exp.
+//   * At the end of its chunk the warp writes the result from registers: the
+//     normalised output for a sequence that fits one chunk, else the chunk's
+//     (m, l, o) partial; the last chunk of each (sequence, KV group) to
+//     finish (a ticket, never a wait) merges the partials by log-sum-exp.
 #include "kv8_common.cuh"
 #include "kv8_internal.h"
 
@@ -42,18 +42,17 @@ constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kPageTx = 2 * kPageBytes + 2 * kBS * sizeof(float);
 
 // --------------------------------------------------------------------------
-// Shared-memory plan of a decode CTA (base aligned to 1024 bytes):
+// Shared-memory plan of a decode CTA of WPC independent warps (base aligned
+// to 1024 bytes):
 //   per warp w: SPW slots of [K page 2048 B | V page 2048 B]   (tiles)
 //   per warp w: SPW slots of [ks 64 B | vs 64 B]              (scales)
 //   per warp w: SPW mbarriers
-// After its last page a warp reuses its own tiles as its merge record:
-//   o[G][128] fp32, m[G], l[G].
 // --------------------------------------------------------------------------
-template <int NW, int SPW>
+template <int WPC, int SPW>
 struct SmemPlan {
-  static constexpr int kTileBytes = NW * SPW * 2 * kPageBytes;
-  static constexpr int kScaleBytes = NW * SPW * 2 * kBS * 4;
-  static constexpr int kBarBytes = NW * SPW * 8;
+  static constexpr int kTileBytes = WPC * SPW * 2 * kPageBytes;
+  static constexpr int kScaleBytes = WPC * SPW * 2 * kBS * 4;
+  static constexpr int kBarBytes = WPC * SPW * 8;
   static constexpr int kBytes = kTileBytes + kScaleBytes + kBarBytes + 1024;
 };
 
@@ -116,49 +115,33 @@ __device__ __forceinline__ int exp_frexp(float x) {
 }
 
 // Log-sum-exp merge of one query head's C chunk partials into its output
-// row: chunk c holds m_c (base-2 max), l_c (sum of 2^(s - m_c)) and o_c[d]
-// (sum of 2^(s - m_c) v_hat[d]);
+// row, by one warp: chunk c holds m_c (base-2 max), l_c (sum of
+// 2^(s - m_c)) and o_c[d] (sum of 2^(s - m_c) v_hat[d]);
 //   M = max_c m_c,  L = sum_c l_c 2^(m_c - M),
 //   out[d] = sum_c o_c[d] 2^(m_c - M) / L.
-// Called by every thread of a CTA of NW warps (it synchronises the CTA);
-// `red` is NW*128 + 2 floats of shared memory.  Warp 0 finds M and L; then
-// warp w sums chunks w, w + NW, ... for 4 dims per lane with float4 loads,
-// and warp 0 adds the NW partial sums.  The fused merge of a split decode
-// and the standalone reduce kernel both use it with the same NW, so they
-// produce identical results.
-template <int NW>
-__device__ __forceinline__ void merge_head(const float* ml, const float* o,
-                                           int nchunks, void* out,
-                                           int64_t out_row, int out_f32,
-                                           float* red) {
+// Lanes split the chunks for M and L, then each lane accumulates 4 dims over
+// all chunks with float4 loads.  The fused merge of a split decode and the
+// standalone reduce kernel both call it, so they give identical results.
+__device__ __forceinline__ void merge_head_warp(const float* ml, const float* o,
+                                                int nchunks, void* out,
+                                                int64_t out_row, int out_f32) {
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  if (warp == 0) {
-    float mx = -INFINITY;
-    for (int c = lane; c < nchunks; c += 32) mx = fmaxf(mx, __ldcg(&ml[2 * c]));
+  float mx = -INFINITY;
+  for (int c = lane; c < nchunks; c += 32) mx = fmaxf(mx, __ldcg(&ml[2 * c]));
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1)
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-    float ls = 0.0f;
-    for (int c = lane; c < nchunks; c += 32) {
-      const float mc = __ldcg(&ml[2 * c]);
-      ls += (mc == -INFINITY) ? 0.0f : __ldcg(&ml[2 * c + 1]) * ex2(mc - mx);
-    }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) ls += __shfl_xor_sync(kFull, ls, m);
-    if (lane == 0) {
-      red[NW * kD] = mx;
-      red[NW * kD + 1] = ls;
-    }
-  }
-  __syncthreads();
-  const float M = red[NW * kD];
-  const float L = red[NW * kD + 1];
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int c = warp; c < nchunks; c += NW) {
+  for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+  float ls = 0.0f;
+  for (int c = lane; c < nchunks; c += 32) {
     const float mc = __ldcg(&ml[2 * c]);
-    const float w = (mc == -INFINITY) ? 0.0f : ex2(mc - M);
+    ls += (mc == -INFINITY) ? 0.0f : __ldcg(&ml[2 * c + 1]) * ex2(mc - mx);
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) ls += __shfl_xor_sync(kFull, ls, m);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+  for (int c = 0; c < nchunks; ++c) {
+    const float mc = __ldcg(&ml[2 * c]);
+    const float w = (mc == -INFINITY) ? 0.0f : ex2(mc - mx);
     const float4 v =
         __ldcg(reinterpret_cast<const float4*>(o + static_cast<int64_t>(c) * kD) + lane);
     acc.x += w * v.x;
@@ -166,27 +149,40 @@ __device__ __forceinline__ void merge_head(const float* ml, const float* o,
     acc.z += w * v.z;
     acc.w += w * v.w;
   }
-  *reinterpret_cast<float4*>(&red[warp * kD + 4 * lane]) = acc;
-  __syncthreads();
-  if (warp == 0) {
-    float4 sum = *reinterpret_cast<const float4*>(&red[4 * lane]);
-#pragma unroll
-    for (int w = 1; w < NW; ++w) {
-      const float4 t = *reinterpret_cast<const float4*>(&red[w * kD + 4 * lane]);
-      sum.x += t.x;
-      sum.y += t.y;
-      sum.z += t.z;
-      sum.w += t.w;
-    }
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-    const int64_t base = out_row * kD + 4 * lane;
-    store_out(out, base + 0, sum.x * inv, out_f32);
-    store_out(out, base + 1, sum.y * inv, out_f32);
-    store_out(out, base + 2, sum.z * inv, out_f32);
-    store_out(out, base + 3, sum.w * inv, out_f32);
-  }
-  __syncthreads();
+  const float inv = ls > 0.0f ? 1.0f / ls : 0.0f;
+  const int64_t base = out_row * kD + 4 * lane;
+  store_out(out, base + 0, acc.x * inv, out_f32);
+  store_out(out, base + 1, acc.y * inv, out_f32);
+  store_out(out, base + 2, acc.z * inv, out_f32);
+  store_out(out, base + 3, acc.w * inv, out_f32);
 }
+
+// Where a warp's finished chunk goes: the normalised output row (a context
+// that fits one chunk) or the chunk's partial (m, l, o) in the workspace.
+struct ChunkSink {
+  void* out;
+  float* ws_o;
+  float* ws_ml;
+  int64_t row0;  // b * H_q + first query head of the KV group
+  int64_t ci0;   // partial index of the first head: row0 * max_chunks + chunk
+  int max_chunks;
+  bool single;
+  int out_f32;
+
+  __device__ __forceinline__ void put_o(int h, int d, float o, float l) const {
+    if (single)
+      store_out(out, (row0 + h) * kD + d, l > 0.0f ? o / l : 0.0f, out_f32);
+    else
+      ws_o[(ci0 + static_cast<int64_t>(h) * max_chunks) * kD + d] = o;
+  }
+  __device__ __forceinline__ void put_ml(int h, float m, float l) const {
+    if (!single) {
+      const int64_t ci = ci0 + static_cast<int64_t>(h) * max_chunks;
+      ws_ml[2 * ci] = m;
+      ws_ml[2 * ci + 1] = l;
+    }
+  }
+};
 
 // --------------------------------------------------------------------------
 // Page math.  A policy object holds one warp's running state over the pages
@@ -195,8 +191,8 @@ __device__ __forceinline__ void merge_head(const float* ml, const float* o,
 //   page(tk, tv, ks, vs, nv)  fold in one 16-token page; tokens >= nv are
 //                             masked (their bytes may be stale or poison)
 //   reset()                   contribute nothing (after a failed wait)
-//   record(rec, lane)         write this warp's o[G][128] (relative to its
-//                             running max m, base 2), m[G] and l[G]
+//   finish(sink)              hand this warp's o[G][128] (relative to its
+//                             running max m, base 2), m[G] and l[G] to sink
 // --------------------------------------------------------------------------
 
 // CUDA-core form: codes become exact fp32 in registers, fp32 FMA.
@@ -205,6 +201,7 @@ __device__ __forceinline__ void merge_head(const float* ml, const float* o,
 //   G == 8: 8 dims (16 lanes per token, 2 tokens per pass, 8 passes).
 template <int G>
 struct SimtMath {
+  static constexpr int kWarpsPerSM = 0;  // no register cap
   static constexpr int DPL = (G <= 4) ? 16 : 8;  // dims per lane
   static constexpr int LPT = kD / DPL;           // lanes per token
   static constexpr int TPP = 32 / LPT;           // tokens per pass
@@ -331,7 +328,7 @@ struct SimtMath {
     }
   }
 
-  __device__ __forceinline__ void record(float* rec) {
+  __device__ __forceinline__ void finish(const ChunkSink& sk) {
 #pragma unroll
     for (int m = LPT; m < 32; m <<= 1) {
 #pragma unroll
@@ -346,25 +343,28 @@ struct SimtMath {
 #pragma unroll
     for (int m = LPT; m < 32; m <<= 1)
       l_lane += __shfl_xor_sync(kFull, l_lane, m);
-    if (tg == 0) {
 #pragma unroll
-      for (int h = 0; h < G; ++h)
+    for (int h = 0; h < G; ++h) {
+      const float lh = __shfl_sync(kFull, l_lane, h * HSTRIDE);
+      if (tg == 0) {
 #pragma unroll
-        for (int i = 0; i < DPL / 2; ++i)
-          *reinterpret_cast<float2*>(&rec[h * kD + dg * DPL + 2 * i]) = o2[h][i];
-      if (dg % HSTRIDE == 0) {
-        rec[G * kD + hh] = m_run;
-        rec[G * kD + G + hh] = l_lane;
+        for (int i = 0; i < DPL / 2; ++i) {
+          sk.put_o(h, dg * DPL + 2 * i, o2[h][i].x, lh);
+          sk.put_o(h, dg * DPL + 2 * i + 1, o2[h][i].y, lh);
+        }
       }
     }
+    if (tg == 0 && dg % HSTRIDE == 0) sk.put_ml(hh, m_run, l_lane);
   }
 };
 
 // Tensor-core form (mma.sync m16n8k16, fp16 operands, fp32 accumulation).
 // Per 16-token page a warp computes
-//   S^T[16 x 8]   = K_code[16 x 128] . q'^T[128 x 8]    rows = the 16 tokens
+//   S^T[16 x 8]   = K_code[16 x 128] . Q^T[128 x 8]     rows = the 16 tokens
 //   O^T[128 x 8] += V_code^T[128 x 16] . P''^T[16 x 8]   cols = query heads
-// i.e. 8 k-steps for the scores and 8 m-tiles x (hi, lo) for the output;
+// i.e. 4 k-steps x 3 digit planes of int8 mma for the scores (the K codes
+// are the A operand exactly as loaded) and 8 m-tiles x (hi, lo) of fp16 mma
+// for the output;
 // columns >= G carry zero q and are never stored.  Thread (r = lane/4,
 // c = lane%4) owns, in both products, heads 2c and 2c+1: it holds their
 // scores for tokens r and 8+r, keeps their running max, and holds their
@@ -373,19 +373,19 @@ struct SimtMath {
 // to the B-operand layout of the p.v mma with two 8x8 movmatrix transposes
 // per fp16 half.
 // Exactness of the operands:
-//   * codes -> fp16 exactly: the byte c+128 is placed under the fp16
+//   * q.k is exact integer arithmetic on q rounded to 22 bits per head
+//     (see init());
+//   * V codes -> fp16 exactly: the byte c+128 is placed under the fp16
 //     exponent of 1024, giving 1152 + c exactly, then 1152 is subtracted;
-//   * q is scaled per head by a power of two so that max|q'| lies in
-//     [2^14, 2^15) and converted to fp16 (exact for bf16 values down to
-//     2^-17 of that max); the power of two goes into the score factor;
 //   * P'' = 2^(s - m) * vs_t * 2^-E is split into fp16 hi + lo (about 22
 //     significant bits); E, a per-warp power of two that only grows, keeps
 //     P'' inside the fp16 range (the accumulators are rescaled exactly);
 //   * m and E are moved lazily (see page()), so most pages skip the
 //     rescale of the accumulators.
 // Index maps (any bijection works as long as both operands agree):
-//   q.k: k index -> dim 32c + 4s + {0,2 | 1,3} in k-step s, so a thread
-//        reads 32 contiguous code bytes of each of its tokens r and 8+r;
+//   q.k: k index 4c+j / 16+4c+j -> dim 32c + 8s + j / 32c + 8s + 4 + j in
+//        k-step s, so a thread reads 32 contiguous code bytes of each of its
+//        tokens r and 8+r and feeds them to the mma unchanged;
 //   p.v: row r / r+8 of m-tile 2w+j -> dim 16r + 4w + 2j + {0 | 1}, so a
 //        thread reads one 16-byte chunk of each of tokens 2c, 2c+1, 8+2c,
 //        9+2c.
@@ -396,6 +396,17 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0,
   asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
       "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Integer mma: D[16x8] (s32) += A[16x32] (s8, row) . B[32x8] (s8, col).
+__device__ __forceinline__ void mma16832_s8(int (&d)[4], uint32_t a0,
+                                            uint32_t a1, uint32_t a2,
+                                            uint32_t a3, uint32_t b0,
+                                            uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, "
+      "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
@@ -444,10 +455,11 @@ __device__ __forceinline__ uint32_t word_of(const uint4& a, int i) {
 
 template <int G>
 struct MmaMath {
+  static constexpr int kWarpsPerSM = 12;  // cap registers at 168 per thread
   static constexpr float kSlack = 8.0f;  // log2 units
   static constexpr int kVSlack = 4;
   int lane, r, c;
-  uint2 qk[8];      // B fragments of q'^T (head r): k-step s
+  uint2 qd[3][4];   // B fragments of Q^T, head r: digit plane p, k-step s
   float qf0, qf1;   // score factors of heads 2c, 2c+1
   float ot[8][4];   // O^T fragments: heads 2c, 2c+1 at two dims per m-tile
   float m0, m1;     // reference max of heads 2c, 2c+1 (base 2)
@@ -456,6 +468,12 @@ struct MmaMath {
   float vlim;       // 2^(e_run + kVSlack)
   float fs;         // 2^-e_run
 
+  // q of head r, dims [32c, 32c+32), as Q = rint(q * 2^sh) with max|Q| in
+  // [2^21, 2^22), written in three balanced base-256 digits
+  // Q = 65536 d2 + 256 d1 + d0 (each an int8).  q.k is then exact integer
+  // arithmetic on the int8 tensor cores, S = 2^-sh (65536 C2 + 256 C1 + C0)
+  // with C_p = sum_d d_p[d] code[d]; the rounding of q to 22 bits relative
+  // to its head's max (<= 2^-23 max|q| per element) is the only error.
   __device__ __forceinline__ void init(const __nv_bfloat16* qg, float q_scale,
                                        int lane_) {
     lane = lane_;
@@ -483,14 +501,31 @@ struct MmaMath {
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qv[i]));
     amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-    // q' = q * 2^sh with max|q'| in [2^14, 2^15); applied as two exact
-    // power-of-two factors so that each stays representable
-    const int sh = amax > 0.0f ? 15 - exp_frexp(amax) : 0;
+    // max|q| * 2^sh in [2^21, 2^22), applied as two exact powers of two
+    const int sh = amax > 0.0f ? 22 - exp_frexp(amax) : 0;
     const float f1 = pow2i(sh / 2), f2 = pow2i(sh - sh / 2);
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      qk[s].x = pack_h2(qv[4 * s + 0] * f1 * f2, qv[4 * s + 2] * f1 * f2);
-      qk[s].y = pack_h2(qv[4 * s + 1] * f1 * f2, qv[4 * s + 3] * f1 * f2);
+    for (int s = 0; s < 4; ++s) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t w0 = 0, w1 = 0, w2 = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int Q = __float2int_rn(qv[8 * s + 4 * half + j] * f1 * f2);
+          const int d0 = static_cast<int>(static_cast<int8_t>(Q & 0xFF));
+          const int q1 = (Q - d0) >> 8;
+          const int d1 = static_cast<int>(static_cast<int8_t>(q1 & 0xFF));
+          const int d2 = (q1 - d1) >> 8;
+          w0 |= (static_cast<uint32_t>(d0) & 0xFFu) << (8 * j);
+          w1 |= (static_cast<uint32_t>(d1) & 0xFFu) << (8 * j);
+          w2 |= (static_cast<uint32_t>(d2) & 0xFFu) << (8 * j);
+        }
+        if (half == 0) {
+          qd[0][s].x = w0; qd[1][s].x = w1; qd[2][s].x = w2;
+        } else {
+          qd[0][s].y = w0; qd[1][s].y = w1; qd[2][s].y = w2;
+        }
+      }
     }
     const float qf = q_scale * pow2i(-(sh / 2)) * pow2i(-(sh - sh / 2));
     // this thread's score columns are heads 2c and 2c+1 (quads 2c, 2c+1)
@@ -522,13 +557,24 @@ struct MmaMath {
     const uint4 ka1 = *reinterpret_cast<const uint4*>(ra + (((2 * c + 1) ^ sw) << 4));
     const uint4 kb0 = *reinterpret_cast<const uint4*>(rb + (((2 * c) ^ sw) << 4));
     const uint4 kb1 = *reinterpret_cast<const uint4*>(rb + (((2 * c + 1) ^ sw) << 4));
-    float st[4] = {0.f, 0.f, 0.f, 0.f};
+    // k-step s covers k = 4c..4c+3 -> word 2s and k = 16+4c.. -> word 2s+1
+    // of each token's 32-byte slice (dims 32c + 8s .. 32c + 8s + 7)
+    int acc[3][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      uint32_t ea, oa, eb, ob;
-      k_word_to_h2(word_of(s < 4 ? ka0 : ka1, s & 3), ea, oa);
-      k_word_to_h2(word_of(s < 4 ? kb0 : kb1, s & 3), eb, ob);
-      mma16816(st, ea, eb, oa, ob, qk[s].x, qk[s].y);
+    for (int s = 0; s < 4; ++s) {
+      const uint32_t a0 = word_of(s < 2 ? ka0 : ka1, (2 * s) & 3);
+      const uint32_t a1 = word_of(s < 2 ? kb0 : kb1, (2 * s) & 3);
+      const uint32_t a2 = word_of(s < 2 ? ka0 : ka1, (2 * s + 1) & 3);
+      const uint32_t a3 = word_of(s < 2 ? kb0 : kb1, (2 * s + 1) & 3);
+#pragma unroll
+      for (int pl = 0; pl < 3; ++pl)
+        mma16832_s8(acc[pl], a0, a1, a2, a3, qd[pl][s].x, qd[pl][s].y);
+    }
+    float st[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int low = acc[1][e] * 256 + acc[0][e];  // |low| < 2^30
+      st[e] = __int2float_rn(acc[2][e]) * 65536.0f + __int2float_rn(low);
     }
     // st: [0] token r head 2c, [1] token r head 2c+1,
     //     [2] token 8+r head 2c, [3] token 8+r head 2c+1
@@ -631,7 +677,7 @@ struct MmaMath {
     }
   }
 
-  __device__ __forceinline__ void record(float* rec) {
+  __device__ __forceinline__ void finish(const ChunkSink& sk) {
     float s0 = l0, s1 = l1;
 #pragma unroll
     for (int m = 4; m < 32; m <<= 1) {
@@ -646,60 +692,78 @@ struct MmaMath {
       const int dA = 16 * r + 4 * w + 2 * j;  // row r
       const int dB = dA + 1;                  // row r + 8
       if (h0 < G) {
-        rec[h0 * kD + dA] = ot[i][0] * f;
-        rec[h0 * kD + dB] = ot[i][2] * f;
+        sk.put_o(h0, dA, ot[i][0] * f, s0);
+        sk.put_o(h0, dB, ot[i][2] * f, s0);
       }
       if (h1 < G) {
-        rec[h1 * kD + dA] = ot[i][1] * f;
-        rec[h1 * kD + dB] = ot[i][3] * f;
+        sk.put_o(h1, dA, ot[i][1] * f, s1);
+        sk.put_o(h1, dB, ot[i][3] * f, s1);
       }
     }
     if (r == 0) {
-      if (h0 < G) {
-        rec[G * kD + h0] = m0;
-        rec[G * kD + G + h0] = s0;
-      }
-      if (h1 < G) {
-        rec[G * kD + h1] = m1;
-        rec[G * kD + G + h1] = s1;
-      }
+      if (h0 < G) sk.put_ml(h0, m0, s0);
+      if (h1 < G) sk.put_ml(h1, m1, s1);
     }
   }
 };
 
 // --------------------------------------------------------------------------
-// The decode kernel: pipeline, merge and write; the page math is `Math`.
+// The decode kernel.  Persistent: a grid of (SMs x resident CTAs) CTAs of
+// WPC independent warps.  A work item is one (sequence, KV head, context
+// chunk); items are numbered chunk-major, i = (chunk * H_kv + kvh) * B + b,
+// and warp gw of W takes items gw, gw + W, ... (skipping chunks past a
+// sequence's end), so every warp sees a mix of chunk positions.  A warp
+// streams its items' pages through its own SPW-slot ring back to back: the
+// issue cursor runs SPW pages ahead of the compute cursor, across item
+// boundaries, so the ring never drains between chunks.  There are no CTA
+// barriers: each warp writes its chunk's result straight from registers.
 // --------------------------------------------------------------------------
-template <int G, int NW, int SPW, class Math>
-__global__ void __launch_bounds__(NW * 32)
+struct Item {
+  int64_t idx;
+  int b, kvh, chunk, n, tok0, tok1, npages, nchunks;
+};
+
+// Decode item idx; false if the chunk lies past its sequence (a context of
+// length 0 keeps chunk 0, with no pages, so that its zero row is written).
+__device__ __forceinline__ bool item_load(const DecodeParams& p, Item& it) {
+  const int64_t per_chunk = static_cast<int64_t>(p.num_kv_heads) * p.batch;
+  it.chunk = static_cast<int>(it.idx / per_chunk);
+  const int64_t rem = it.idx - static_cast<int64_t>(it.chunk) * per_chunk;
+  it.kvh = static_cast<int>(rem / p.batch);
+  it.b = static_cast<int>(rem - static_cast<int64_t>(it.kvh) * p.batch);
+  it.n = p.context_lens[it.b];
+  it.tok0 = it.chunk * p.chunk_tokens;
+  if (it.tok0 >= it.n && !(it.n == 0 && it.chunk == 0)) return false;
+  it.tok1 = min(it.n, it.tok0 + p.chunk_tokens);
+  it.npages = (it.tok1 - it.tok0 + kBS - 1) / kBS;
+  it.nchunks = (it.n + p.chunk_tokens - 1) / p.chunk_tokens;
+  return true;
+}
+
+__device__ __forceinline__ void item_next(const DecodeParams& p, Item& it,
+                                          int64_t stride, int64_t n_items) {
+  do {
+    it.idx += stride;
+  } while (it.idx < n_items && !item_load(p, it));
+}
+
+template <int G, int WPC, int SPW, class Math>
+__global__ void __launch_bounds__(WPC * 32,
+                                  Math::kWarpsPerSM / WPC > 0 ? Math::kWarpsPerSM / WPC : 1)
 decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
               const __grid_constant__ CUtensorMap tmv) {
-  using Plan = SmemPlan<NW, SPW>;
+  using Plan = SmemPlan<WPC, SPW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-  const int chunk = blockIdx.x;
-  const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  const int n = p.context_lens[b];
-  const int tok0 = chunk * p.chunk_tokens;
-  if (tok0 >= n && !(n == 0 && chunk == 0)) return;
-  const int tok1 = min(n, tok0 + p.chunk_tokens);
-  const int npages = (tok1 - tok0 + kBS - 1) / kBS;
-  const int nchunks = (n + p.chunk_tokens - 1) / p.chunk_tokens;
-  const int my_pages = warp < npages ? (npages - warp + NW - 1) / NW : 0;
-
   uint8_t* tiles = smem + warp * SPW * 2 * kPageBytes;
   float* scl = reinterpret_cast<float*>(smem + Plan::kTileBytes) +
                warp * SPW * 2 * kBS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kTileBytes +
                                                Plan::kScaleBytes) +
                    warp * SPW;
-
   if (lane == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
@@ -709,20 +773,35 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   }
   __syncwarp();
 
-  // ---- page issue: block-table entries are fetched 32 at a time
-  const int32_t* bt = p.block_tables +
-                      static_cast<int64_t>(b) * p.max_blocks_per_seq +
-                      tok0 / kBS + warp;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * WPC;
+  const int64_t n_items =
+      static_cast<int64_t>(p.max_chunks) * p.num_kv_heads * p.batch;
+  Item cmp;
+  cmp.idx = static_cast<int64_t>(blockIdx.x) * WPC + warp;
+  if (cmp.idx < n_items && !item_load(p, cmp)) item_next(p, cmp, stride, n_items);
+
+  // ---- issue cursor: SPW pages ahead of the compute cursor
+  Item iss = cmp;
+  int iss_page = 0;
   int bt_reg = 0;
-  auto issue = [&](int k) {
-    if ((k & 31) == 0) {
-      const int kk = k + lane;
-      bt_reg = kk < my_pages ? bt[kk * NW] : 0;
+  uint32_t k_iss = 0;
+  auto issue_one = [&]() {
+    while (iss.idx < n_items && iss_page >= iss.npages) {
+      item_next(p, iss, stride, n_items);
+      iss_page = 0;
     }
-    const int blk = __shfl_sync(kFull, bt_reg, k & 31);
+    if (iss.idx >= n_items) return;
+    if ((iss_page & 31) == 0) {
+      const int j = iss_page + lane;
+      bt_reg = j < iss.npages
+                   ? p.block_tables[static_cast<int64_t>(iss.b) * p.max_blocks_per_seq +
+                                    iss.tok0 / kBS + j]
+                   : 0;
+    }
+    const int blk = __shfl_sync(kFull, bt_reg, iss_page & 31);
     if (lane == 0) {
-      const int s = k % SPW;
-      const int page = blk * p.num_kv_heads + kvh;
+      const int s = k_iss % SPW;
+      const int page = blk * p.num_kv_heads + iss.kvh;
       mbar_arrive_expect_tx(&bars[s], kPageTx);
       uint8_t* tk = tiles + s * 2 * kPageBytes;
       tma_load_3d(tk, &tmk, 0, 0, page, &bars[s]);
@@ -733,150 +812,128 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       bulk_g2s(sc + kBS, p.v_scales + static_cast<int64_t>(page) * kBS,
                kBS * sizeof(float), &bars[s]);
     }
+    ++k_iss;
+    ++iss_page;
   };
-  const int pre = my_pages < SPW ? my_pages : SPW;
-  for (int k = 0; k < pre; ++k) issue(k);
+#pragma unroll 1
+  for (int s = 0; s < SPW; ++s) issue_one();
 
   Math math;
-  math.init(p.q + (static_cast<int64_t>(b) * p.num_q_heads + kvh * G) * kD,
-            p.q_scale, lane);
-
+  uint32_t k_cmp = 0;
   bool ok = true;
-  int k = 0;
-  for (; k < my_pages; ++k) {
-    const int s = k % SPW;
-    if (!mbar_wait(&bars[s], (k / SPW) & 1, &g_device_status)) {
-      ok = false;
-      break;
+  while (cmp.idx < n_items) {
+    const int64_t row0 = static_cast<int64_t>(cmp.b) * p.num_q_heads + cmp.kvh * G;
+    math.init(p.q + row0 * kD, p.q_scale, lane);
+    for (int j = 0; j < cmp.npages; ++j) {
+      const int s = k_cmp % SPW;
+      if (!mbar_wait(&bars[s], (k_cmp / SPW) & 1, &g_device_status)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* tk = tiles + s * 2 * kPageBytes;
+      const float* ks = scl + s * 2 * kBS;
+      math.page(tk, tk + kPageBytes, ks, ks + kBS,
+                min(kBS, cmp.tok1 - (cmp.tok0 + j * kBS)));
+      __syncwarp();
+      issue_one();
+      ++k_cmp;
     }
-    const uint8_t* tk = tiles + s * 2 * kPageBytes;
-    const float* ks = scl + s * 2 * kBS;
-    const int tbase = tok0 + (warp + k * NW) * kBS;
-    math.page(tk, tk + kPageBytes, ks, ks + kBS, min(kBS, tok1 - tbase));
-    __syncwarp();
-    if (k + SPW < my_pages) issue(k + SPW);
-  }
-  if (!ok) {
-    // A copy never landed: drain what is still in flight (bounded), then
-    // contribute nothing to the merge.  The sticky status word reports it.
-    for (int kk = k + 1; kk < my_pages && kk < k + SPW; ++kk)
-      mbar_wait(&bars[kk % SPW], (kk / SPW) & 1, &g_device_status);
-    math.reset();
-  }
+    if (!ok) break;
 
-  // ---- warp record in this warp's own (now idle) tiles, then merge
-  __syncwarp();
-  math.record(reinterpret_cast<float*>(tiles));
-  __syncthreads();
+    ChunkSink sk;
+    sk.out = p.out;
+    sk.ws_o = p.ws_o;
+    sk.ws_ml = p.ws_ml;
+    sk.row0 = row0;
+    sk.ci0 = row0 * p.max_chunks + cmp.chunk;
+    sk.max_chunks = p.max_chunks;
+    sk.single = cmp.nchunks <= 1;
+    sk.out_f32 = p.out_f32;
+    math.finish(sk);
 
-  const bool single = nchunks <= 1;
-  for (int idx = threadIdx.x; idx < G * kD; idx += NW * 32) {
-    const int h = idx / kD;
-    const int d = idx % kD;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float* rw = reinterpret_cast<const float*>(smem + w * SPW * 2 * kPageBytes);
-      M = fmaxf(M, rw[G * kD + h]);
-    }
-    float L = 0.0f, O = 0.0f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float* rw = reinterpret_cast<const float*>(smem + w * SPW * 2 * kPageBytes);
-      const float mw = rw[G * kD + h];
-      const float e = (mw == -INFINITY) ? 0.0f : ex2(mw - M);
-      L += rw[G * kD + G + h] * e;
-      O += rw[h * kD + d] * e;
-    }
-    const int hq = kvh * G + h;
-    if (single) {
-      const int64_t oi = (static_cast<int64_t>(b) * p.num_q_heads + hq) * kD + d;
-      store_out(p.out, oi, L > 0.0f ? O / L : 0.0f, p.out_f32);
-    } else {
-      const int64_t ci =
-          (static_cast<int64_t>(b) * p.num_q_heads + hq) * p.max_chunks + chunk;
-      p.ws_o[ci * kD + d] = O;
-      if (d == 0) {
-        p.ws_ml[2 * ci] = M;
-        p.ws_ml[2 * ci + 1] = L;
+    if (!sk.single) {
+      // the last chunk of this (sequence, KV group) to finish merges them
+      __threadfence();
+      __syncwarp();
+      unsigned int ticket = 0;
+      if (lane == 0) ticket = atomicAdd(&p.ws_ctr[row0], 1u);
+      ticket = __shfl_sync(kFull, ticket, 0);
+      if (ticket == static_cast<unsigned int>(cmp.nchunks - 1)) {
+        __threadfence();
+        for (int h = 0; h < G; ++h)
+          merge_head_warp(p.ws_ml + (row0 + h) * p.max_chunks * 2,
+                          p.ws_o + (row0 + h) * p.max_chunks * kD, cmp.nchunks,
+                          p.out, row0 + h, p.out_f32);
       }
     }
+    item_next(p, cmp, stride, n_items);
   }
-  if (single) return;
-
-  // ---- split: the last CTA of this (sequence, KV group) to finish merges
-  // every chunk's partial (threadfence-then-ticket; no CTA ever waits).
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned int ticket = atomicAdd(
-        &p.ws_ctr[static_cast<int64_t>(b) * p.num_q_heads + kvh * G], 1u);
-    s_last = ticket == static_cast<unsigned int>(nchunks - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  float* red = reinterpret_cast<float*>(smem);  // records no longer needed
-  for (int h = 0; h < G; ++h) {
-    const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + kvh * G + h;
-    merge_head<NW>(p.ws_ml + bh * p.max_chunks * 2,
-                   p.ws_o + bh * p.max_chunks * kD, nchunks, p.out, bh,
-                   p.out_f32, red);
+  if (!ok) {
+    // A copy never landed: drain the other copies in flight (bounded) and
+    // stop.  The sticky status word reports it.
+    for (uint32_t k = k_cmp + 1; k < k_iss; ++k)
+      mbar_wait(&bars[k % SPW], (k / SPW) & 1, &g_device_status);
   }
 }
 
 // --------------------------------------------------------------------------
-// Standalone split reduce: one CTA of kReduceNW warps per (b, hq), the same
-// merge routine (and warp count) as the fused merge of the decode kernel.
+// Standalone split reduce: one warp per (b, hq), the same merge routine as
+// the fused merge of the decode kernel.
 // --------------------------------------------------------------------------
-constexpr int kReduceNW = 4;
-
-__global__ void __launch_bounds__(kReduceNW * 32)
+__global__ void __launch_bounds__(32)
 split_reduce_kernel(const float* __restrict__ ws_ml,
                     const float* __restrict__ ws_o,
                     const int32_t* __restrict__ context_lens, int32_t num_q_heads,
                     int32_t chunk_tokens, int32_t max_chunks, void* out,
                     int32_t out_f32) {
-  __shared__ __align__(16) float red[kReduceNW * kD + 2];
   const int bh = blockIdx.x;
   const int b = bh / num_q_heads;
   const int n = context_lens[b];
   const int nchunks = (n + chunk_tokens - 1) / chunk_tokens;
   if (nchunks <= 1) return;
-  merge_head<kReduceNW>(ws_ml + static_cast<int64_t>(bh) * max_chunks * 2,
-                        ws_o + static_cast<int64_t>(bh) * max_chunks * kD,
-                        nchunks, out, bh, out_f32, red);
+  merge_head_warp(ws_ml + static_cast<int64_t>(bh) * max_chunks * 2,
+                  ws_o + static_cast<int64_t>(bh) * max_chunks * kD, nchunks,
+                  out, bh, out_f32);
 }
 
-template <int G, int NW, int SPW, class Math>
+template <int G, int WPC, int SPW, class Math>
 int launch_decode_kernel(const DecodeParams& p, const CUtensorMap& tmk,
                          const CUtensorMap& tmv, cudaStream_t stream) {
-  auto kern = decode_kernel<G, NW, SPW, Math>;
-  constexpr int smem = SmemPlan<NW, SPW>::kBytes;
-  static bool attr_done = false;  // per instantiation; benign race
-  if (!attr_done) {
+  auto kern = decode_kernel<G, WPC, SPW, Math>;
+  constexpr int smem = SmemPlan<WPC, SPW>::kBytes;
+  static int resident = 0;  // CTAs per SM for this instantiation
+  static int sms = 0;
+  if (resident == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
       return -1;
-    attr_done = true;
+    int nsm = 0, occ = 0;
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, WPC * 32,
+                                                      smem) != cudaSuccess)
+      return -1;
+    sms = nsm;
+    resident = occ > 0 ? occ : 1;
   }
-  dim3 grid(p.max_chunks, p.num_kv_heads, p.batch);
-  kern<<<grid, NW * 32, smem, stream>>>(p, tmk, tmv);
+  const int64_t n_items =
+      static_cast<int64_t>(p.max_chunks) * p.num_kv_heads * p.batch;
+  int64_t ctas = static_cast<int64_t>(sms) * resident;
+  const int64_t need = (n_items + WPC - 1) / WPC;
+  if (ctas > need) ctas = need;
+  if (ctas < 1) ctas = 1;
+  kern<<<static_cast<unsigned>(ctas), WPC * 32, smem, stream>>>(p, tmk, tmv);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 template <int G>
 int launch_group(const DecodeParams& p, const CUtensorMap& tmk,
                  const CUtensorMap& tmv, int32_t variant, cudaStream_t stream) {
-  // CTA shape from a sweep on B200 over (warps, slots per warp) in
-  // {1,2,4,8} x {2,3,4,6,8} on the four multi-sequence workloads: 4 warps
-  // with 2 slots each (8 pages, 33 KB in flight per CTA; 4 CTAs per SM) was
-  // fastest for the tensor-core form on all of them.
   if (variant == 1)
     return launch_decode_kernel<G, 4, 4, SimtMath<G>>(p, tmk, tmv, stream);
-  static_assert(kReduceNW == 4, "fused and standalone merges must match");
-  return launch_decode_kernel<G, 4, 2, MmaMath<G>>(p, tmk, tmv, stream);
+  return launch_decode_kernel<G, 4, 3, MmaMath<G>>(p, tmk, tmv, stream);
 }
 
 }  // namespace
@@ -939,7 +996,7 @@ int launch_split_reduce(const float* ws_ml, const float* ws_o,
                         cudaStream_t stream) {
   const int64_t nbh = static_cast<int64_t>(batch) * num_q_heads;
   if (nbh == 0) return 0;
-  split_reduce_kernel<<<static_cast<unsigned>(nbh), kReduceNW * 32, 0, stream>>>(
+  split_reduce_kernel<<<static_cast<unsigned>(nbh), 32, 0, stream>>>(
       ws_ml, ws_o, context_lens, num_q_heads, chunk_tokens, max_chunks, out,
       out_f32);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
