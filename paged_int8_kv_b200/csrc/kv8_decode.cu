@@ -358,34 +358,33 @@ struct SimtMath {
   }
 };
 
-// Tensor-core form (mma.sync m16n8k16, fp16 operands, fp32 accumulation).
-// Per 16-token page a warp computes
-//   S^T[16 x 8]   = K_code[16 x 128] . Q^T[128 x 8]     rows = the 16 tokens
-//   O^T[128 x 8] += V_code^T[128 x 16] . P''^T[16 x 8]   cols = query heads
-// i.e. 4 k-steps x 3 digit planes of int8 mma for the scores (the K codes
-// are the A operand exactly as loaded) and 8 m-tiles x (hi, lo) of fp16 mma
-// for the output;
-// columns >= G carry zero q and are never stored.  Thread (r = lane/4,
-// c = lane%4) owns, in both products, heads 2c and 2c+1: it holds their
-// scores for tokens r and 8+r, keeps their running max, and holds their
-// O^T columns, so the softmax bookkeeping never leaves the thread except
-// on a (rare) change of the reference max.  P'' moves from the S^T layout
-// to the B-operand layout of the p.v mma with two 8x8 movmatrix transposes
-// per fp16 half.
-// Exactness of the operands:
-//   * q.k is exact integer arithmetic on q rounded to 22 bits per head
-//     (see init());
-//   * V codes -> fp16 exactly: the byte c+128 is placed under the fp16
-//     exponent of 1024, giving 1152 + c exactly, then 1152 is subtracted;
-//   * P'' = 2^(s - m) * vs_t * 2^-E is split into fp16 hi + lo (about 22
-//     significant bits); E, a per-warp power of two that only grows, keeps
-//     P'' inside the fp16 range (the accumulators are rescaled exactly);
-//   * m and E are moved lazily (see page()), so most pages skip the
-//     rescale of the accumulators.
+// Tensor-core form.  Per 16-token page a warp computes
+//   S[16 x 16]    = Qd[16 x 128] . K_code^T[128 x 16]   (int8 mma, exact)
+//   O^T[128 x 8] += V_code^T[128 x 16] . P''^T[16 x 8]   (fp16 mma, fp32 acc)
+// * q.k: the rows of Qd are (query head, digit plane): q of head h is
+//   rounded to Q = rint(q * 2^sh) with max|Q| in [2^29, 2^30) and written
+//   as four balanced int8 digits Q = 2^24 d3 + 2^16 d2 + 2^8 d1 + d0; m-tile
+//   0 holds (d3 | d2) and m-tile 1 (d1 | d0) of heads 0..7 in rows r / r+8.
+//   The K codes enter as the B operand exactly as loaded (a thread's two
+//   32-bit words of a token are one B fragment), the int32 products are
+//   exact, and S = 2^-sh (2^16 (2^8 C3 + C2) + (2^8 C1 + C0)).  The only
+//   approximation is the rounding of q to 30 bits of its head's max.
+//   2 m-tiles x 2 n-tiles (tokens 0..7, 8..15) x 4 k-steps = 16 mma.
+// * Thread (r = lane/4, c = lane%4) then holds head r's scores for tokens
+//   2c, 2c+1, 8+2c, 9+2c: exactly its B fragment of P''^T for the p.v mma,
+//   so the probabilities never move between lanes.
+// * p.v: V codes -> fp16 exactly (the byte c+128 under the fp16 exponent of
+//   1024 gives 1152 + c; 1152 is subtracted); P'' = 2^(s - m) vs_t 2^-E is
+//   split into fp16 hi + lo (about 22 bits); 8 m-tiles x (hi, lo) = 16 mma.
+//   The O^T columns are heads 2c, 2c+1.
+// * Softmax: base 2, one running max and sum per head (quad r), moved
+//   lazily: only when a score exceeds the reference by more than kSlack or
+//   a V scale exceeds 2^(E + kVSlack) are the references moved and the
+//   accumulators rescaled (exactly, by powers of two and one exp2).
 // Index maps (any bijection works as long as both operands agree):
 //   q.k: k index 4c+j / 16+4c+j -> dim 32c + 8s + j / 32c + 8s + 4 + j in
 //        k-step s, so a thread reads 32 contiguous code bytes of each of its
-//        tokens r and 8+r and feeds them to the mma unchanged;
+//        tokens r and 8+r;
 //   p.v: row r / r+8 of m-tile 2w+j -> dim 16r + 4w + 2j + {0 | 1}, so a
 //        thread reads one 16-byte chunk of each of tokens 2c, 2c+1, 8+2c,
 //        9+2c.
@@ -456,24 +455,18 @@ __device__ __forceinline__ uint32_t word_of(const uint4& a, int i) {
 template <int G>
 struct MmaMath {
   static constexpr int kWarpsPerSM = 12;  // cap registers at 168 per thread
-  static constexpr float kSlack = 8.0f;  // log2 units
+  static constexpr float kSlack = 8.0f;   // log2 units
   static constexpr int kVSlack = 4;
   int lane, r, c;
-  uint2 qd[3][4];   // B fragments of Q^T, head r: digit plane p, k-step s
-  float qf0, qf1;   // score factors of heads 2c, 2c+1
+  uint4 qa[2][4];   // A fragments of Qd (head r): m-tile t, k-step s
+  float qf;         // score factor of head r: 2^-sh * softmax_scale * log2(e)
   float ot[8][4];   // O^T fragments: heads 2c, 2c+1 at two dims per m-tile
-  float m0, m1;     // reference max of heads 2c, 2c+1 (base 2)
-  float l0, l1;     // this thread's partial sums of heads 2c, 2c+1
+  float m_run;      // reference max of head r (base 2)
+  float l_run;      // this thread's partial sum of head r
   int e_run;        // P'' carries 2^-e_run (warp-uniform)
   float vlim;       // 2^(e_run + kVSlack)
   float fs;         // 2^-e_run
 
-  // q of head r, dims [32c, 32c+32), as Q = rint(q * 2^sh) with max|Q| in
-  // [2^21, 2^22), written in three balanced base-256 digits
-  // Q = 65536 d2 + 256 d1 + d0 (each an int8).  q.k is then exact integer
-  // arithmetic on the int8 tensor cores, S = 2^-sh (65536 C2 + 256 C1 + C0)
-  // with C_p = sum_d d_p[d] code[d]; the rounding of q to 22 bits relative
-  // to its head's max (<= 2^-23 max|q| per element) is the only error.
   __device__ __forceinline__ void init(const __nv_bfloat16* qg, float q_scale,
                                        int lane_) {
     lane = lane_;
@@ -501,42 +494,45 @@ struct MmaMath {
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qv[i]));
     amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-    // max|q| * 2^sh in [2^21, 2^22), applied as two exact powers of two
-    const int sh = amax > 0.0f ? 22 - exp_frexp(amax) : 0;
+    // max|q| * 2^sh in [2^29, 2^30), applied as two exact powers of two
+    const int sh = amax > 0.0f ? 30 - exp_frexp(amax) : 0;
     const float f1 = pow2i(sh / 2), f2 = pow2i(sh - sh / 2);
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        uint32_t w0 = 0, w1 = 0, w2 = 0;
+        uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int Q = __float2int_rn(qv[8 * s + 4 * half + j] * f1 * f2);
           const int d0 = static_cast<int>(static_cast<int8_t>(Q & 0xFF));
           const int q1 = (Q - d0) >> 8;
           const int d1 = static_cast<int>(static_cast<int8_t>(q1 & 0xFF));
-          const int d2 = (q1 - d1) >> 8;
+          const int q2 = (q1 - d1) >> 8;
+          const int d2 = static_cast<int>(static_cast<int8_t>(q2 & 0xFF));
+          const int d3 = (q2 - d2) >> 8;
           w0 |= (static_cast<uint32_t>(d0) & 0xFFu) << (8 * j);
           w1 |= (static_cast<uint32_t>(d1) & 0xFFu) << (8 * j);
           w2 |= (static_cast<uint32_t>(d2) & 0xFFu) << (8 * j);
+          w3 |= (static_cast<uint32_t>(d3) & 0xFFu) << (8 * j);
         }
+        // k = 4c..4c+3 (word 2s: a0/a1), k = 16+4c.. (word 2s+1: a2/a3)
         if (half == 0) {
-          qd[0][s].x = w0; qd[1][s].x = w1; qd[2][s].x = w2;
+          qa[0][s].x = w3; qa[0][s].y = w2;
+          qa[1][s].x = w1; qa[1][s].y = w0;
         } else {
-          qd[0][s].y = w0; qd[1][s].y = w1; qd[2][s].y = w2;
+          qa[0][s].z = w3; qa[0][s].w = w2;
+          qa[1][s].z = w1; qa[1][s].w = w0;
         }
       }
     }
-    const float qf = q_scale * pow2i(-(sh / 2)) * pow2i(-(sh - sh / 2));
-    // this thread's score columns are heads 2c and 2c+1 (quads 2c, 2c+1)
-    qf0 = __shfl_sync(kFull, qf, 8 * c);
-    qf1 = __shfl_sync(kFull, qf, 8 * c + 4);
+    qf = q_scale * pow2i(-(sh / 2)) * pow2i(-(sh - sh / 2));
     reset();
   }
 
   __device__ __forceinline__ void reset() {
-    m0 = m1 = -INFINITY;
-    l0 = l1 = 0.0f;
+    m_run = -INFINITY;
+    l_run = 0.0f;
     e_run = -126;
     vlim = 0.0f;
     fs = 1.0f;
@@ -549,7 +545,8 @@ struct MmaMath {
   __device__ __forceinline__ void page(const uint8_t* tk, const uint8_t* tv,
                                        const float* ks, const float* vs,
                                        int nv) {
-    // ---- S^T = K q'^T: rows r (token r) and r+8 (token 8+r)
+    // ---- S = Qd K^T: n-tile 0 = tokens 0..7 (this thread feeds token r),
+    //                  n-tile 1 = tokens 8..15 (token 8 + r)
     const uint8_t* ra = tk + r * 128;
     const uint8_t* rb = tk + (8 + r) * 128;
     const int sw = r & 7;  // (8 + r) & 7 == r & 7
@@ -557,95 +554,96 @@ struct MmaMath {
     const uint4 ka1 = *reinterpret_cast<const uint4*>(ra + (((2 * c + 1) ^ sw) << 4));
     const uint4 kb0 = *reinterpret_cast<const uint4*>(rb + (((2 * c) ^ sw) << 4));
     const uint4 kb1 = *reinterpret_cast<const uint4*>(rb + (((2 * c + 1) ^ sw) << 4));
-    // k-step s covers k = 4c..4c+3 -> word 2s and k = 16+4c.. -> word 2s+1
-    // of each token's 32-byte slice (dims 32c + 8s .. 32c + 8s + 7)
-    int acc[3][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}};
+    int acc[2][2][4];
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[t][j][e] = 0;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      const uint32_t a0 = word_of(s < 2 ? ka0 : ka1, (2 * s) & 3);
-      const uint32_t a1 = word_of(s < 2 ? kb0 : kb1, (2 * s) & 3);
-      const uint32_t a2 = word_of(s < 2 ? ka0 : ka1, (2 * s + 1) & 3);
-      const uint32_t a3 = word_of(s < 2 ? kb0 : kb1, (2 * s + 1) & 3);
+      const uint4& ka = s < 2 ? ka0 : ka1;
+      const uint4& kb = s < 2 ? kb0 : kb1;
+      const uint32_t a0 = (s & 1) ? ka.z : ka.x, a1 = (s & 1) ? ka.w : ka.y;
+      const uint32_t b0 = (s & 1) ? kb.z : kb.x, b1 = (s & 1) ? kb.w : kb.y;
 #pragma unroll
-      for (int pl = 0; pl < 3; ++pl)
-        mma16832_s8(acc[pl], a0, a1, a2, a3, qd[pl][s].x, qd[pl][s].y);
+      for (int t = 0; t < 2; ++t) {
+        mma16832_s8(acc[t][0], qa[t][s].x, qa[t][s].y, qa[t][s].z, qa[t][s].w, a0, a1);
+        mma16832_s8(acc[t][1], qa[t][s].x, qa[t][s].y, qa[t][s].z, qa[t][s].w, b0, b1);
+      }
     }
+    // head r, tokens 2c, 2c+1 (n-tile 0) and 8+2c, 9+2c (n-tile 1)
     float st[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int low = acc[1][e] * 256 + acc[0][e];  // |low| < 2^30
-      st[e] = __int2float_rn(acc[2][e]) * 65536.0f + __int2float_rn(low);
-    }
-    // st: [0] token r head 2c, [1] token r head 2c+1,
-    //     [2] token 8+r head 2c, [3] token 8+r head 2c+1
-    const bool va = r < nv, vb = 8 + r < nv;
-    const float ksa = ks[r], ksb = ks[8 + r];
-    const float vsa = va ? vs[r] : 0.0f, vsb = vb ? vs[8 + r] : 0.0f;
-    float sc[4];
-    sc[0] = va ? st[0] * qf0 * ksa : -INFINITY;
-    sc[1] = va ? st[1] * qf1 * ksa : -INFINITY;
-    sc[2] = vb ? st[2] * qf0 * ksb : -INFINITY;
-    sc[3] = vb ? st[3] * qf1 * ksb : -INFINITY;
-
-    // Lazy rescaling: the reference maxima (per head) and the exponent
-    // e_run (per warp) move only when a score exceeds its reference by
-    // more than kSlack or a V scale exceeds 2^(e_run + kVSlack); otherwise
-    // probabilities up to 2^kSlack are accumulated against the stale
-    // reference, which keeps every P'' below 2^(kSlack + kVSlack).
-    const float lm0 = fmaxf(sc[0], sc[2]);
-    const float lm1 = fmaxf(sc[1], sc[3]);
-    const float lv = fmaxf(vsa, vsb);
-    const bool move = lm0 > m0 + kSlack || lm1 > m1 + kSlack || lv > vlim;
-    if (__any_sync(kFull, move)) {
-      float x0 = lm0, x1 = lm1, vx = lv;
+    for (int j = 0; j < 2; ++j)
 #pragma unroll
-      for (int m = 4; m < 32; m <<= 1) {
-        x0 = fmaxf(x0, __shfl_xor_sync(kFull, x0, m));
-        x1 = fmaxf(x1, __shfl_xor_sync(kFull, x1, m));
-        vx = fmaxf(vx, __shfl_xor_sync(kFull, vx, m));
+      for (int e = 0; e < 2; ++e) {
+        const int hi = acc[0][j][e] * 256 + acc[0][j][2 + e];  // d3, d2
+        const int lo = acc[1][j][e] * 256 + acc[1][j][2 + e];  // d1, d0
+        st[2 * j + e] = __int2float_rn(hi) * 65536.0f + __int2float_rn(lo);
       }
-      const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
-      // every lane sees the same 16 tokens' scales: e_new is warp-uniform
+    const int t0 = 2 * c, t2 = 8 + 2 * c;
+    const float2 ksa = *reinterpret_cast<const float2*>(ks + t0);
+    const float2 ksb = *reinterpret_cast<const float2*>(ks + t2);
+    const float2 vsa = *reinterpret_cast<const float2*>(vs + t0);
+    const float2 vsb = *reinterpret_cast<const float2*>(vs + t2);
+    const bool v0 = t0 < nv, v1 = t0 + 1 < nv, v2 = t2 < nv, v3 = t2 + 1 < nv;
+    float sc[4];
+    sc[0] = v0 ? st[0] * qf * ksa.x : -INFINITY;
+    sc[1] = v1 ? st[1] * qf * ksa.y : -INFINITY;
+    sc[2] = v2 ? st[2] * qf * ksb.x : -INFINITY;
+    sc[3] = v3 ? st[3] * qf * ksb.y : -INFINITY;
+    float vsv[4];
+    vsv[0] = v0 ? vsa.x : 0.0f;
+    vsv[1] = v1 ? vsa.y : 0.0f;
+    vsv[2] = v2 ? vsb.x : 0.0f;
+    vsv[3] = v3 ? vsb.y : 0.0f;
+
+    const float lm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    const float lv = fmaxf(fmaxf(vsv[0], vsv[1]), fmaxf(vsv[2], vsv[3]));
+    if (__any_sync(kFull, lm > m_run + kSlack || lv > vlim)) {
+      float x = fmaxf(lm, __shfl_xor_sync(kFull, lm, 1));
+      x = fmaxf(x, __shfl_xor_sync(kFull, x, 2));
+      float vx = fmaxf(lv, __shfl_xor_sync(kFull, lv, 1));
+      vx = fmaxf(vx, __shfl_xor_sync(kFull, vx, 2));
+      const float n = fmaxf(m_run, x);
+      // every quad sees all 16 tokens' scales: e_new is warp-uniform
       const int e_new = vx > vlim ? exp_frexp(vx) : e_run;
-      const float ef = pow2i(max(e_run - e_new, -126));
-      const float a0 = (n0 == m0) ? 1.0f : ex2(m0 - n0);
-      const float a1 = (n1 == m1) ? 1.0f : ex2(m1 - n1);
-      l0 *= a0;
-      l1 *= a1;
-      m0 = n0;
-      m1 = n1;
+      const float a = (n == m_run) ? 1.0f : ex2(m_run - n);
+      const float a_o = a * pow2i(max(e_run - e_new, -126));
+      l_run *= a;
+      m_run = n;
       e_run = e_new;
       vlim = pow2i(min(e_new + kVSlack, 127));
       fs = pow2i(-e_new);
-      const float b0 = a0 * ef, b1 = a1 * ef;
+      const float ae = __shfl_sync(kFull, a_o, 8 * c);      // head 2c
+      const float ao = __shfl_sync(kFull, a_o, 8 * c + 4);  // head 2c+1
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        ot[i][0] *= b0;
-        ot[i][1] *= b1;
-        ot[i][2] *= b0;
-        ot[i][3] *= b1;
+        ot[i][0] *= ae;
+        ot[i][1] *= ao;
+        ot[i][2] *= ae;
+        ot[i][3] *= ao;
       }
     }
-    const float u0 = m0 == -INFINITY ? 0.0f : m0;
-    const float u1 = m1 == -INFINITY ? 0.0f : m1;
-    const float p0 = ex2(sc[0] - u0), p1 = ex2(sc[1] - u1);
-    const float p2 = ex2(sc[2] - u0), p3 = ex2(sc[3] - u1);
-    l0 += p0 + p2;
-    l1 += p1 + p3;
-    const float wa = vsa * fs, wb = vsb * fs;
-    const float q0 = p0 * wa, q1 = p1 * wa, q2 = p2 * wb, q3 = p3 * wb;
-    // fp16 hi/lo in the S^T layout (rows = tokens, cols = heads) ...
-    const uint32_t ha = pack_h2(q0, q1), hb = pack_h2(q2, q3);
-    const float2 fa = unpack_h2(ha), fb = unpack_h2(hb);
-    const uint32_t la = pack_h2(q0 - fa.x, q1 - fa.y);
-    const uint32_t lb = pack_h2(q2 - fb.x, q3 - fb.y);
-    // ... transposed to B fragments of P''^T: head r, tokens {2c, 2c+1}
-    // (tokens 0..7 matrix) and {8+2c, 9+2c} (tokens 8..15 matrix)
-    const uint32_t h0 = movmatrix_t(ha), h2 = movmatrix_t(hb);
-    const uint32_t g0 = movmatrix_t(la), g2 = movmatrix_t(lb);
+    const float mu = m_run == -INFINITY ? 0.0f : m_run;
+    float pr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pr[i] = ex2(sc[i] - mu);
+    l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    float pp[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pp[i] = pr[i] * (vsv[i] * fs);
+    // B fragments of P''^T (head r): tokens {2c, 2c+1} and {8+2c, 9+2c}
+    const uint32_t h0 = pack_h2(pp[0], pp[1]);
+    const uint32_t h2 = pack_h2(pp[2], pp[3]);
+    const float2 f0 = unpack_h2(h0);
+    const float2 f2 = unpack_h2(h2);
+    const uint32_t g0 = pack_h2(pp[0] - f0.x, pp[1] - f0.y);
+    const uint32_t g2 = pack_h2(pp[2] - f2.x, pp[3] - f2.y);
 
     // ---- O^T += V^T P''^T: tokens 2c, 2c+1, 8+2c, 9+2c, 16-byte chunk r
-    const int t0 = 2 * c, t2 = 8 + 2 * c;
     const int cr0 = (r ^ (2 * c)) << 4;      // tokens 2c and 8+2c
     const int cr1 = (r ^ (2 * c + 1)) << 4;  // tokens 2c+1 and 9+2c
     const uint4 vA = *reinterpret_cast<const uint4*>(tv + t0 * 128 + cr0);
@@ -660,15 +658,13 @@ struct MmaMath {
       const uint32_t Y = prmt(A, B, 0x7362u) ^ 0x80808080u;  // bytes 2,3
       const uint32_t Z = prmt(C, D, 0x5140u) ^ 0x80808080u;
       const uint32_t U = prmt(C, D, 0x7362u) ^ 0x80808080u;
-      // m-tile 2w: rows r / r+8 = byte 0 / byte 1
-      {
+      {  // m-tile 2w: rows r / r+8 = byte 0 / byte 1
         const uint32_t a0 = v_pair(X, 0x4140u), a1 = v_pair(X, 0x4342u);
         const uint32_t a2 = v_pair(Z, 0x4140u), a3 = v_pair(Z, 0x4342u);
         mma16816(ot[2 * w], a0, a1, a2, a3, h0, h2);
         mma16816(ot[2 * w], a0, a1, a2, a3, g0, g2);
       }
-      // m-tile 2w+1: rows r / r+8 = byte 2 / byte 3
-      {
+      {  // m-tile 2w+1: rows r / r+8 = byte 2 / byte 3
         const uint32_t a0 = v_pair(Y, 0x4140u), a1 = v_pair(Y, 0x4342u);
         const uint32_t a2 = v_pair(U, 0x4140u), a3 = v_pair(U, 0x4342u);
         mma16816(ot[2 * w + 1], a0, a1, a2, a3, h0, h2);
@@ -678,12 +674,14 @@ struct MmaMath {
   }
 
   __device__ __forceinline__ void finish(const ChunkSink& sk) {
-    float s0 = l0, s1 = l1;
-#pragma unroll
-    for (int m = 4; m < 32; m <<= 1) {
-      s0 += __shfl_xor_sync(kFull, s0, m);
-      s1 += __shfl_xor_sync(kFull, s1, m);
-    }
+    float l = l_run;
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+    // this thread's O^T columns are heads 2c (quad 2c) and 2c+1 (quad 2c+1)
+    const float s0 = __shfl_sync(kFull, l, 8 * c);
+    const float s1 = __shfl_sync(kFull, l, 8 * c + 4);
+    const float m0 = __shfl_sync(kFull, m_run, 8 * c);
+    const float m1 = __shfl_sync(kFull, m_run, 8 * c + 4);
     const float f = pow2i(e_run);
     const int h0 = 2 * c, h1 = 2 * c + 1;
 #pragma unroll
@@ -785,6 +783,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   int iss_page = 0;
   int bt_reg = 0;
   uint32_t k_iss = 0;
+  int slot_iss = 0;
   auto issue_one = [&]() {
     while (iss.idx < n_items && iss_page >= iss.npages) {
       item_next(p, iss, stride, n_items);
@@ -800,7 +799,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     }
     const int blk = __shfl_sync(kFull, bt_reg, iss_page & 31);
     if (lane == 0) {
-      const int s = k_iss % SPW;
+      const int s = slot_iss;
       const int page = blk * p.num_kv_heads + iss.kvh;
       mbar_arrive_expect_tx(&bars[s], kPageTx);
       uint8_t* tk = tiles + s * 2 * kPageBytes;
@@ -814,29 +813,35 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     }
     ++k_iss;
     ++iss_page;
+    slot_iss = slot_iss + 1 == SPW ? 0 : slot_iss + 1;
   };
 #pragma unroll 1
   for (int s = 0; s < SPW; ++s) issue_one();
 
   Math math;
   uint32_t k_cmp = 0;
+  int slot = 0;
+  uint32_t phase = 0;
   bool ok = true;
   while (cmp.idx < n_items) {
     const int64_t row0 = static_cast<int64_t>(cmp.b) * p.num_q_heads + cmp.kvh * G;
     math.init(p.q + row0 * kD, p.q_scale, lane);
     for (int j = 0; j < cmp.npages; ++j) {
-      const int s = k_cmp % SPW;
-      if (!mbar_wait(&bars[s], (k_cmp / SPW) & 1, &g_device_status)) {
+      if (!mbar_wait(&bars[slot], phase, &g_device_status)) {
         ok = false;
         break;
       }
-      const uint8_t* tk = tiles + s * 2 * kPageBytes;
-      const float* ks = scl + s * 2 * kBS;
+      const uint8_t* tk = tiles + slot * 2 * kPageBytes;
+      const float* ks = scl + slot * 2 * kBS;
       math.page(tk, tk + kPageBytes, ks, ks + kBS,
                 min(kBS, cmp.tok1 - (cmp.tok0 + j * kBS)));
       __syncwarp();
       issue_one();
       ++k_cmp;
+      if (++slot == SPW) {
+        slot = 0;
+        phase ^= 1u;
+      }
     }
     if (!ok) break;
 
