@@ -443,7 +443,7 @@ def main():
     ap.add_argument("--impl", default="kv8", choices=["kv8", "reference"])
     ap.add_argument("--workload", default="llama8b_b64_32k", choices=sorted(W.NAMED))
     ap.add_argument("--chunk", type=int, default=512)
-    ap.add_argument("--kernel", type=int, default=0, help="0 auto, 1 CUDA-core, 2 tensor-core")
+    ap.add_argument("--kernel", type=int, default=0, help="0 auto, 1 CUDA-core, 2 mma.sync tensor-core, 3 tcgen05")
     ap.add_argument("--cpu-seqs", type=int, default=4)
     ap.add_argument("--ref-seqs", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -180,12 +180,16 @@ KV8_API int32_t kv8_split_reduce(const void *workspace, size_t workspace_bytes,
 
 /*
  * kv8_set_decode_kernel -- choose how kv8_paged_decode_attention computes a
- * page (process-wide, for tuning and for comparing the two forms):
+ * page (process-wide, for tuning and for comparing the forms):
  *   0  automatic (default),
  *   1  CUDA-core form: codes converted to fp32 in registers, fp32 FMA,
- *   2  tensor-core form: codes converted exactly to fp16, q.k and p.v on
- *      mma tiles with fp32 accumulation.
- * Both compute the same function; results differ only by rounding order.
+ *   2  warp tensor-core form (mma.sync): q.k as int8 products of the K codes
+ *      with exact int8 digit planes of q; p.v on V codes converted exactly
+ *      to fp16 with fp32 accumulation,
+ *   3  tcgen05 form: q.k and p.v both as int8 products on the 5th-generation
+ *      tensor cores (digit planes of q and of the probabilities), int32
+ *      accumulators in tensor memory, K and V codes read as TMA stages them.
+ * All compute the same function; results differ only by rounding order.
  * Returns KV8_ERR_INVALID_ARG for any other value.  Not thread-safe with
  * respect to concurrent decode calls.
  */

@@ -74,7 +74,7 @@ void split_shape(int32_t max_context_len, int32_t chunk_tokens,
   }
 }
 
-int32_t g_decode_kernel = 0;  // 0 auto, 1 CUDA-core FMA, 2 tensor-core mma
+int32_t g_decode_kernel = 0;  // 0 auto, 1 CUDA-core, 2 mma.sync, 3 tcgen05
 
 }  // namespace
 
@@ -214,7 +214,9 @@ int32_t kv8_paged_decode_attention(
       cudaMemsetAsync(ws_ctr, 0, kv8::workspace_ctr_bytes(batch, num_q_heads),
                       st) != cudaSuccess)
     return KV8_ERR_CUDA;
-  int rc = kv8::launch_decode(p, tmk, tmv, g_decode_kernel, st);
+  int rc = g_decode_kernel == 3
+               ? kv8::launch_decode_tc(p, tmk, tmv, st)
+               : kv8::launch_decode(p, tmk, tmv, g_decode_kernel, st);
   if (rc == -2) return KV8_ERR_UNSUPPORTED;
   if (rc != 0) return KV8_ERR_CUDA;
   return KV8_OK;
@@ -252,7 +254,7 @@ int32_t kv8_split_reduce(const void* workspace, size_t workspace_bytes,
 }
 
 int32_t kv8_set_decode_kernel(int32_t kind) {
-  if (kind < 0 || kind > 2) return KV8_ERR_INVALID_ARG;
+  if (kind < 0 || kind > 3) return KV8_ERR_INVALID_ARG;
   g_decode_kernel = kind;
   return KV8_OK;
 }

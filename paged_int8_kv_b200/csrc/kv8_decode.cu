@@ -29,6 +29,7 @@
 //     finish (a ticket, never a wait) merges the partials by log-sum-exp.
 #include "kv8_common.cuh"
 #include "kv8_internal.h"
+#include "kv8_merge.cuh"
 
 namespace kv8 {
 
@@ -86,75 +87,6 @@ __device__ __forceinline__ float reduce_heads(float (&v)[G], int lane) {
 template <int G, int LPT>
 __device__ __forceinline__ int lane_head(int dg) {
   return dg / (LPT / G);
-}
-
-__device__ __forceinline__ void store_out(void* out, int64_t idx, float v,
-                                          int out_f32) {
-  if (out_f32)
-    static_cast<float*>(out)[idx] = v;
-  else
-    static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
-}
-
-// Hardware base-2 exponential (MUFU), relative error ~2^-22; -inf -> 0.
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// 2^e for e in [-126, 127], built from the exponent bits.
-__device__ __forceinline__ float pow2i(int e) {
-  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-}
-
-// For x > 0 normal: the e with x = f * 2^e, f in [0.5, 1); x <= 2^-126 -> -125.
-__device__ __forceinline__ int exp_frexp(float x) {
-  const int be = static_cast<int>((__float_as_uint(x) >> 23) & 0xFF);
-  return be == 0 ? -125 : be - 126;
-}
-
-// Log-sum-exp merge of one query head's C chunk partials into its output
-// row, by one warp: chunk c holds m_c (base-2 max), l_c (sum of
-// 2^(s - m_c)) and o_c[d] (sum of 2^(s - m_c) v_hat[d]);
-//   M = max_c m_c,  L = sum_c l_c 2^(m_c - M),
-//   out[d] = sum_c o_c[d] 2^(m_c - M) / L.
-// Lanes split the chunks for M and L, then each lane accumulates 4 dims over
-// all chunks with float4 loads.  The fused merge of a split decode and the
-// standalone reduce kernel both call it, so they give identical results.
-__device__ __forceinline__ void merge_head_warp(const float* ml, const float* o,
-                                                int nchunks, void* out,
-                                                int64_t out_row, int out_f32) {
-  const int lane = threadIdx.x & 31;
-  float mx = -INFINITY;
-  for (int c = lane; c < nchunks; c += 32) mx = fmaxf(mx, __ldcg(&ml[2 * c]));
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-  float ls = 0.0f;
-  for (int c = lane; c < nchunks; c += 32) {
-    const float mc = __ldcg(&ml[2 * c]);
-    ls += (mc == -INFINITY) ? 0.0f : __ldcg(&ml[2 * c + 1]) * ex2(mc - mx);
-  }
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) ls += __shfl_xor_sync(kFull, ls, m);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-  for (int c = 0; c < nchunks; ++c) {
-    const float mc = __ldcg(&ml[2 * c]);
-    const float w = (mc == -INFINITY) ? 0.0f : ex2(mc - mx);
-    const float4 v =
-        __ldcg(reinterpret_cast<const float4*>(o + static_cast<int64_t>(c) * kD) + lane);
-    acc.x += w * v.x;
-    acc.y += w * v.y;
-    acc.z += w * v.z;
-    acc.w += w * v.w;
-  }
-  const float inv = ls > 0.0f ? 1.0f / ls : 0.0f;
-  const int64_t base = out_row * kD + 4 * lane;
-  store_out(out, base + 0, acc.x * inv, out_f32);
-  store_out(out, base + 1, acc.y * inv, out_f32);
-  store_out(out, base + 2, acc.z * inv, out_f32);
-  store_out(out, base + 3, acc.w * inv, out_f32);
 }
 
 // Where a warp's finished chunk goes: the normalised output row (a context
@@ -914,6 +846,11 @@ int launch_decode_kernel(const DecodeParams& p, const CUtensorMap& tmk,
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
       return -1;
+    // all of the unified L1 / shared storage as shared memory, so that the
+    // occupancy computed below is what the launch gets
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return -1;
     int nsm = 0, occ = 0;
     if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) !=
             cudaSuccess ||
@@ -954,6 +891,9 @@ int read_device_status(uint32_t* value, int clear) {
         cudaSuccess)
       return -1;
   }
+  uint32_t tc = 0;
+  if (read_tc_status(&tc, clear) != 0) return -1;
+  *value |= tc;
   return 0;
 }
 

@@ -63,8 +63,17 @@ int launch_split_reduce(const float* ws_ml, const float* ws_o,
                         int32_t max_chunks, void* out, int32_t out_f32,
                         cudaStream_t stream);
 
-// Reads (and optionally clears) the sticky device status word after a
-// device-wide synchronize.  Returns 0, or -1 on a CUDA error.
+// Decode on the tcgen05 tensor cores (kv8_decode_tc.cu); same contract as
+// launch_decode.
+int launch_decode_tc(const DecodeParams& p, const CUtensorMap& tmk,
+                     const CUtensorMap& tmv, cudaStream_t stream);
+
+// Sticky status word of the tcgen05 decode kernel (no synchronize).
+int read_tc_status(uint32_t* value, int clear);
+
+// Reads (and optionally clears) the sticky device status words of every
+// decode kernel after a device-wide synchronize, OR-ed together.  Returns 0,
+// or -1 on a CUDA error.
 int read_device_status(uint32_t* value, int clear);
 
 }  // namespace kv8

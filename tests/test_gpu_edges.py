@@ -42,7 +42,7 @@ def _ref(oracle_mod, w):
                                        w.context_lens)
 
 
-@pytest.mark.parametrize("kind", [1, 2], ids=["cudacore", "tensorcore"])
+@pytest.mark.parametrize("kind", [1, 2, 3], ids=["cudacore", "mmasync", "tcgen05"])
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (8, 2), (16, 2), (4, 1)])
 @pytest.mark.parametrize("chunk", [0, 16, 512])
 def test_ragged_groups_chunks(pk, oracle_mod, hq, hkv, chunk, kind):
@@ -79,7 +79,7 @@ def test_tensorcore_extreme_magnitudes(pk, oracle_mod, scale):
     w.private_kv = scaled
     ref = _ref(oracle_mod, w)
     cache, qd, bt, cl = U.device_inputs(w)
-    for kind in (1, 2):
+    for kind in (1, 2, 3):
         pk.kv8_set_decode_kernel(kind)
         gpu = U.gpu_decode(cache, qd, bt, cl, w, chunk_tokens=256)
         denom = max(np.abs(ref).max(), 1e-30)
@@ -92,11 +92,12 @@ def test_tensorcore_matches_cudacore(pk):
                         outliers=(4, 8.0))
     cache, q, bt, cl = U.device_inputs(w)
     outs = []
-    for kind in (1, 2):
+    for kind in (1, 2, 3):
         pk.kv8_set_decode_kernel(kind)
         outs.append(U.gpu_decode(cache, q, bt, cl, w, chunk_tokens=512))
     pk.kv8_set_decode_kernel(0)
     assert np.abs(outs[0] - outs[1]).max() < 1e-4
+    assert np.abs(outs[0] - outs[2]).max() < 1e-4
 
 
 def test_block_permutation_bit_identical(pk):
