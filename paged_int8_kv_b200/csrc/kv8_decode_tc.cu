@@ -23,20 +23,25 @@
 //
 // A CTA is persistent over work items (sequence, KV head, chunk) numbered
 // chunk-major; a chunk is taken in groups of 8 pages (128 tokens) that cycle
-// through NB shared-memory buffers.  Warp roles:
-//   producer (1 warp)   TMA of each group's K and V pages and scales;
-//   issuer (1 warp)     builds the q digit planes of each item (q loaded one
-//                       item ahead) and issues q.k of group g, then p.v of
-//                       group g-1, one thread issuing, completion signalled
-//                       by tcgen05.commit;
-//   softmax (4 warps)   thread t takes token t of a group: reads S from
-//                       tensor memory, runs the base-2 online softmax with
-//                       lazy moves of the reference max m and of the V-scale
-//                       exponent E, writes the P'' planes; drains O (thread
-//                       t = dim t) into fp32 registers only when m or E move
-//                       and at the end of the item.
-// Roles hand over through mbarriers only.  Every wait is bounded in time and
-// records a status bit on timeout.
+// through NB shared-memory buffers.  Warp roles (8 warps):
+//   producer (1)   TMA of each group's K and V pages and both scale rows;
+//   q planes (1)   the q digit planes of each item, up to two items ahead
+//                  of q.k, from q loaded one item before that;
+//   issuer (1)     one thread issues q.k and p.v from a non-blocking event
+//                  loop (p.v first); completion is signalled by
+//                  tcgen05.commit on mbarriers;
+//   softmax (4)    thread t takes token t of a group: reads S from tensor
+//                  memory, runs the base-2 online softmax with lazy moves of
+//                  the reference max m and of the V-scale exponent E, writes
+//                  the P'' planes; drains O (thread t = dim t) into fp32
+//                  registers when m or E move, and at the end of the item
+//                  after the next item's first group is handed over (O has
+//                  two tensor-memory slots, by item parity);
+//   epilogue (1)   per split item, the merge ticket and, for the last chunk,
+//                  the log-sum-exp merge.
+// Roles hand over through mbarriers (and one shared counter for the
+// epilogue) only.  Every wait is bounded in time and records a status bit
+// on timeout.
 #include "kv8_common.cuh"
 #include "kv8_internal.h"
 #include "kv8_merge.cuh"
@@ -71,8 +76,8 @@ struct TcPlan {
   static constexpr int kPd = kQd + 2 * N * kD;                     // [2][N x 128 B]
   static constexpr int kQf = kPd + 2 * N * kD;                     // [2][8] f32
   static constexpr int kPacc = kQf + 64;                           // [2] u32
-  static constexpr int kRed = kPacc + 16;                          // 160 f32
-  static constexpr int kBar = kRed + 160 * 4;                      // mbarriers
+  static constexpr int kRed = kPacc + 16;                          // 176 f32
+  static constexpr int kBar = kRed + 176 * 4;                      // mbarriers
   static constexpr int kBarCount = 2 * NB + 14;
   static constexpr int kEnd = kBar + kBarCount * 8 + 16;           // + tmem slot
   static constexpr int kBytes = kEnd + 1024;                       // align slack
@@ -311,6 +316,21 @@ __device__ __forceinline__ float warp_max(float v) {
   return r;
 }
 
+// Waits for phase `parity` of `bar` for about `ns` nanoseconds at most (the
+// thread is suspended meanwhile); true once the phase has completed.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
+                                                   uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Non-blocking probe of phase `parity` of `bar`.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -414,7 +434,8 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t tO = tmem + 2 * N;  // S slots at tmem and tmem + N
+  // tensor memory: S slots at columns [0, N) and [N, 2N); O slots (by item
+  // parity) at [2N, 3N) and [3N, 4N)
 
   TcCursor cur;
   cur.start(p);
@@ -459,8 +480,10 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       mbar_wait_ns(&full[k % NB], (k / NB) & 1);
   } else if (warp == 5) {
     // ======================================================= MMA issuer
+    uint32_t obits = 0;  // O slot (item parity) of group g at bit g % 32
     auto issue_pv = [&](uint32_t g) {  // pfull of g observed
       const int s = g & 1;
+      const uint32_t tO = tmem + (2 + ((obits >> (g & 31)) & 1u)) * N;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t acc = pacc[s];
@@ -521,6 +544,7 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
             if (qk_j == qk_groups - 1) mma_commit(&qempty[qs]);
           }
           __syncwarp();
+          obits = (obits & ~(1u << (ngrp & 31))) | ((nitem & 1u) << (ngrp & 31));
           ++ngrp;
           if (++qk_j == qk_groups) {
             qk_j = 0;
@@ -534,9 +558,16 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
           continue;
         }
       }
-      // idle
+      // idle: sleep briefly on the barrier most likely to complete next
+      if (lane == 0) {
+        if (gv < ngrp)
+          mbar_try_wait_hint(&pfull[gv & 1], (gv >> 1) & 1, 256);
+        else if (qk_left)
+          mbar_try_wait_hint(&full[ngrp % NB], (ngrp / NB) & 1, 256);
+      }
+      __syncwarp();
       if (spins == 0) t_idle = global_ns();
-      if ((++spins & 63) == 0 && global_ns() - t_idle > kWaitNs) {
+      if ((++spins & 15) == 0 && global_ns() - t_idle > kWaitNs) {
         if (lane == 0) atomicOr(&g_tc_status, KV8_DEV_WAIT_TIMEOUT);
         break;
       }
@@ -653,10 +684,63 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     const int t = tid;  // token of a group in the softmax, dim in the output
     const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
     uint32_t nitem = 0, nout = 0;
+    // The previous item's O (tensor-memory slot by item parity) is drained
+    // and its output written only after this item's first group has been
+    // handed to the tensor cores, so its last p.v is never waited for.
+    // (m and l of the pending item, the same in every thread, stay in the
+    // shared l-sum area of its parity: l at [0, 32), m at [32, 40))
+    bool pn_on = false, pn_drain = false, pn_single = false;
+    int64_t pn_row0 = 0;
+    int pn_chunk = 0, pn_e = 0;
+    uint32_t pn_g = 0, pn_slot = 0;
+    const float* pn_red = red;
+    float pn_o[GP];
+    auto drain_into = [&](uint32_t oslot, uint32_t glast, float (&acc)[GP]) {
+      // O (int32 planes) of the p.v up to group glast, added into acc
+      wait_or_fail(&pempty[glast & 1], (glast >> 1) & 1, failed);
+      tc_fence_after();
+      uint32_t orr[N];
+      tmem_ld_row(tmem + (2 + oslot) * N + lane_base, orr);
+#pragma unroll
+      for (int h = 0; h < GP; ++h) {
+        const float v =
+            (__int2float_rn(static_cast<int>(orr[3 * GP + h])) * 256.0f +
+             __int2float_rn(static_cast<int>(orr[2 * GP + h]))) * 65536.0f +
+            (__int2float_rn(static_cast<int>(orr[GP + h])) * 256.0f +
+             __int2float_rn(static_cast<int>(orr[h])));
+        acc[h] += v;
+      }
+    };
+    auto finish_pending = [&]() {
+      if (!pn_on) return;
+      if (pn_drain) drain_into(pn_slot, pn_g, pn_o);
+      const float2 os = pow2pair(pn_e - kPFrac);  // O = acc 2^(E - 24)
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float o = pn_o[h] * os.x * os.y;
+        const float L = (pn_red[h] + pn_red[8 + h]) + (pn_red[16 + h] + pn_red[24 + h]);
+        if (pn_single) {
+          store_out(p.out, (pn_row0 + h) * kD + t, L > 0.0f ? o / L : 0.0f, p.out_f32);
+        } else {
+          const int64_t ci = (pn_row0 + h) * p.max_chunks + pn_chunk;
+          p.ws_o[ci * kD + t] = o;
+          if (t == 0) {
+            p.ws_ml[2 * ci] = pn_red[32 + h];
+            p.ws_ml[2 * ci + 1] = L;
+          }
+        }
+      }
+      if (!pn_single) {  // partials written: hand the item to the epilogue warp
+        __syncwarp();
+        if (lane == 0) done_add(&s_done);
+      }
+      pn_on = false;
+    };
     for (; cur.valid(); cur.next()) {
       const TcItem it = cur.it;
       const int64_t row0 = static_cast<int64_t>(it.b) * p.num_q_heads + it.kvh * G;
       const int ngroups = (it.npages + kGroupPages - 1) / kGroupPages;
+      const uint32_t oslot = nitem & 1;
       float qf[GP];
       if (ngroups > 0) {
         const int qs = nitem & 1;
@@ -677,24 +761,6 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       float vlim = 0.0f;
       bool o_fresh = true;  // next p.v overwrites O
       int o_groups = 0;     // groups accumulated in O since the last drain
-
-      auto drain_o = [&]() {  // O (int32 planes, current units) into o_acc
-        wait_or_fail(&pempty[(ngrp - 1) & 1], ((ngrp - 1) >> 1) & 1, failed);
-        tc_fence_after();
-        uint32_t orr[N];
-        tmem_ld_row(tO + lane_base, orr);
-#pragma unroll
-        for (int h = 0; h < GP; ++h) {
-          const float v =
-              (__int2float_rn(static_cast<int>(orr[3 * GP + h])) * 256.0f +
-               __int2float_rn(static_cast<int>(orr[2 * GP + h]))) * 65536.0f +
-              (__int2float_rn(static_cast<int>(orr[GP + h])) * 256.0f +
-               __int2float_rn(static_cast<int>(orr[h])));
-          o_acc[h] += v;
-        }
-        o_fresh = true;
-        o_groups = 0;
-      };
 
       for (int g = 0; g < ngroups; ++g, ++ngrp) {
         const int s = ngrp & 1;
@@ -727,7 +793,11 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
           }
           float vx = warp_max(vs);
           if (lane == 0) red[64 + warp] = vx;
-          if (!o_fresh) drain_o();
+          if (!o_fresh) {  // O so far into o_acc at the old references
+            drain_into(oslot, ngrp - 1, o_acc);
+            o_fresh = true;
+            o_groups = 0;
+          }
           consumers_sync();
           vx = fmaxf(fmaxf(red[64], red[65]), fmaxf(red[66], red[67]));
           const int e_new = vx > vlim ? exp_frexp(vx) : e_run;  // vs < 2^E
@@ -765,42 +835,35 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
         warp_arrive(&pfull[s], lane);
         o_fresh = false;
         ++o_groups;
+        if (g == 0) finish_pending();
       }
-      // ---- end of the chunk: drain O, sum l over tokens, write
-      if (!o_fresh) drain_o();
-      float* lred = red + 96 + (nout & 1) * 32;  // alternating l-sum areas
+      // ---- end of the chunk: sum l over tokens; O and the output follow
+      // the next item's first group
+      float* lred = red + 96 + (nout & 1) * 40;  // alternating l-sum areas
 #pragma unroll
       for (int h = 0; h < GP; ++h) {
         float x = l_part[h];
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(kFull, x, m);
         if (lane == 0) lred[warp * 8 + h] = x;
+        if (t == 0) lred[32 + h] = m_ref[h];
       }
-      tc_fence_before();
-      consumers_sync();  // l sums visible; O read before the next p.v
+      consumers_sync();  // l sums visible
       ++nout;
-      const bool single = it.nchunks <= 1;
-      const float2 os = pow2pair(e_run - kPFrac);  // O = o_acc 2^(E - 24)
+      finish_pending();  // an item without groups leaves one behind
+      pn_on = true;
+      pn_drain = !o_fresh;
+      pn_single = it.nchunks <= 1;
+      pn_row0 = row0;
+      pn_chunk = it.chunk;
+      pn_e = e_run;
+      pn_g = ngrp - 1;
+      pn_slot = oslot;
+      pn_red = lred;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float L = (lred[h] + lred[8 + h]) + (lred[16 + h] + lred[24 + h]);
-        const float o = o_acc[h] * os.x * os.y;
-        if (single) {
-          store_out(p.out, (row0 + h) * kD + t, L > 0.0f ? o / L : 0.0f, p.out_f32);
-        } else {
-          const int64_t ci = (row0 + h) * p.max_chunks + it.chunk;
-          p.ws_o[ci * kD + t] = o;
-          if (t == 0) {
-            p.ws_ml[2 * ci] = m_ref[h];
-            p.ws_ml[2 * ci + 1] = L;
-          }
-        }
-      }
-      if (!single) {  // partials written: hand the item to the epilogue warp
-        __syncwarp();
-        if (lane == 0) done_add(&s_done);
-      }
+      for (int h = 0; h < GP; ++h) pn_o[h] = o_acc[h];
     }
+    finish_pending();
   }
   tc_fence_before();
   __syncthreads();

@@ -7,7 +7,8 @@
     sampled ones of the 32K workload, in the split-K launch the bench times,
     within the tolerance stated by the method's target: |gpu - oracle| <= 2e-3
     for fp32 output, plus half a bf16 ulp of the exact value for bf16 output
-    (the rounding of the output itself).
+    (the rounding of the output itself); both for the default decode form
+    and for the tcgen05 form.
 """
 import numpy as np
 import pytest
@@ -61,9 +62,20 @@ def test_quantize_bit_exact(built, oracle_mod, name):
     assert np.array_equal(_u32(cache.v_scales.cpu().numpy()), _u32(vs))
 
 
+KINDS = pytest.mark.parametrize("kind", [0, 3], ids=["default", "tcgen05"])
+
+
+@pytest.fixture
+def kind_set(built, kind):
+    built.kv8_set_decode_kernel(kind)
+    yield kind
+    built.kv8_set_decode_kernel(0)
+
+
+@KINDS
 @pytest.mark.parametrize("name", SMALL)
 @pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
-def test_decode_all_pairs(built, oracle_mod, name, out_dtype):
+def test_decode_all_pairs(built, oracle_mod, name, out_dtype, kind_set):
     w, (cache, q, bt, cl), (kc, vc, ks, vs) = _setup(name, oracle_mod)
     ref = oracle_mod.decode_attention(w.q(), kc, vc, ks, vs, w.block_tables,
                                       w.context_lens)
@@ -100,8 +112,9 @@ def test_big_quantize_sampled_sequences(big, oracle_mod):
         assert np.array_equal(_u32(cache.v_scales[blocks].cpu().numpy()), _u32(vs))
 
 
+@KINDS
 @pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
-def test_big_decode_sampled(big, oracle_mod, out_dtype):
+def test_big_decode_sampled(big, oracle_mod, out_dtype, kind_set):
     w, (cache, q, bt, cl) = big
     dt = torch.float32 if out_dtype == "f32" else torch.bfloat16
     gpu = U.gpu_decode(cache, q, bt, cl, w, out_dtype=dt)
