@@ -65,6 +65,19 @@ def algorithmic_bytes(w: W.Workload) -> dict:
             "total": kv + q + out + tables}
 
 
+def unique_kv_bytes(w: W.Workload) -> int:
+    """Codes + scales of the distinct (physical block, KV head) pages the
+    launch attends: a block shared by several sequences (a common prefix)
+    counts once, with the most tokens any sequence uses of it."""
+    used = {}
+    for b in range(w.batch):
+        t = int(w.context_lens[b])
+        for j in range(math.ceil(t / w.block_size)):
+            blk = int(w.block_tables[b, j])
+            used[blk] = max(used.get(blk, 0), min(w.block_size, t - j * w.block_size))
+    return sum(used.values()) * w.num_kv_heads * BYTES_PER_TOKEN_HEAD
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -419,6 +432,9 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
         "data": "synthetic (seeded N(0,1) bf16 q/K/V, shuffled blocks)",
         "config": bench_config(w, args),
         "hbm_gbs": achieved,
+        **({"hbm_gbs_unique_bytes": (uniq + ab["total"] - ab["kv"]) / (dms * 1e-3) / 1e9,
+            "unique_bytes": uniq + ab["total"] - ab["kv"]}
+           if (uniq := unique_kv_bytes(w)) < ab["kv"] else {}),
         "hbm_frac_of_measured": achieved / peak,
         "hbm_frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
         "decode_us": dms * 1e3,
