@@ -187,11 +187,17 @@ def whole_job_rate(units_per_rank: int, world: int, ms_per_step: float) -> float
 
 
 # ------------------------------------------------------------- CPU oracle
-def oracle_sample_seconds(w: W.Workload, seqs) -> tuple[float, str]:
+def oracle_sample_seconds(w: W.Workload, seqs, threads: int = 1) -> tuple[float, str]:
     """Time the oracle's decode step (append of the new token + attention
-    for every query head) on sequences ``seqs``; cache build excluded."""
+    for every query head) on sequences ``seqs``; cache build excluded.
+
+    With ``threads`` > 1 the attention calls, one per (sequence, KV head),
+    run on a pool of that many threads (the oracle is plain single-threaded
+    C; its calls release the interpreter lock, so the pool spreads them over
+    the host cores)."""
     import oracle
-    total = 0.0
+    from concurrent.futures import ThreadPoolExecutor
+    prep = []
     for b in seqs:
         k, v = w.sequence_kv(b)
         n = k.shape[0]
@@ -204,17 +210,41 @@ def oracle_sample_seconds(w: W.Workload, seqs) -> tuple[float, str]:
         slots = np.arange(n, dtype=np.int64)
         oracle.quantize_append(k[:-1], slots[:-1], kc, ks)
         oracle.quantize_append(v[:-1], slots[:-1], vc, vs)
-        table = np.arange(nblk, dtype=np.int32)[None, :]
-        t0 = time.perf_counter()
+        prep.append((b, k, v, slots, kc, vc, ks, vs))
+    g = w.group
+    tasks = [(i, kvh) for i in range(len(prep)) for kvh in range(w.num_kv_heads)]
+
+    def attend(task):
+        i, kvh = task
+        b, k, v, slots, kc, vc, ks, vs = prep[i]
+        table = np.arange(kc.shape[0], dtype=np.int32)[None, :]
+        oracle.decode_attention(w.q()[b:b + 1], kc, vc, ks, vs, table,
+                                w.context_lens[b:b + 1],
+                                pairs=[(0, h) for h in range(kvh * g, (kvh + 1) * g)])
+
+    t0 = time.perf_counter()
+    for b, k, v, slots, kc, vc, ks, vs in prep:
         oracle.quantize_append(k[-1:], slots[-1:], kc, ks)
         oracle.quantize_append(v[-1:], slots[-1:], vc, vs)
-        oracle.decode_attention(w.q()[b:b + 1], kc, vc, ks, vs, table,
-                                w.context_lens[b:b + 1])
-        total += time.perf_counter() - t0
+    if threads > 1:
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(attend, tasks))
+    else:
+        for t in tasks:
+            attend(t)
+    total = time.perf_counter() - t0
     desc = (f"{len(seqs)} of {w.batch} sequences of {w.name}: append 1 token "
             f"+ attention for all {w.num_q_heads} query heads over "
-            f"{int(w.context_lens[list(seqs)].sum())} tokens (fp64, 1 thread)")
+            f"{int(w.context_lens[list(seqs)].sum())} tokens (fp64, "
+            f"{threads} thread{'s' if threads > 1 else ''})")
     return total, desc
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
 
 
 def run_reference(args, w: W.Workload, rank: int):
@@ -222,14 +252,15 @@ def run_reference(args, w: W.Workload, rank: int):
         return 0
     import oracle
     oracle.build()
+    cores = host_cores()
     nseq = max(1, args.ref_seqs)
-    seqs = list(range(nseq))
+    seqs = list(range(min(nseq, w.batch)))
     for _ in range(args.warmup):
-        oracle_sample_seconds(w, seqs[:1])
+        oracle_sample_seconds(w, seqs[:1], cores)
     times = []
     desc = ""
     for i in range(args.steps):
-        s, desc = oracle_sample_seconds(w, [seqs[i % nseq]])
+        s, desc = oracle_sample_seconds(w, [seqs[i % len(seqs)]], cores)
         times.append(s)
     sec = sum(times) / len(times)
     value = 1.0 / sec
@@ -238,10 +269,9 @@ def run_reference(args, w: W.Workload, rank: int):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": bench_config(w, args),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1,
-                         "kind": "oracle",
-                         "sample": "per step: " + desc.replace("1 of", "1 of")},
+        "config": bench_config(w, args, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores,
+                         "kind": "oracle", "sample": "per step: " + desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -249,41 +279,148 @@ def run_reference(args, w: W.Workload, rank: int):
     return 0
 
 
-def bench_config(w: W.Workload, args) -> dict:
+def bench_config(w: W.Workload, args, world: int) -> dict:
     return {"workload": w.name, "batch": w.batch,
             "context_lens": (int(w.context_lens.min()), int(w.context_lens.max())),
             "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "block_size": w.block_size,
             "chunk_tokens": args.chunk, "num_blocks": w.num_blocks,
-            "parallelism": f"replica x{args.gpus} (sequences independent)",
+            "parallelism": (f"{world} ranks, one GPU each, every rank its own "
+                            "batch (sequences independent)" if world > 1 else
+                            "1 GPU"),
             "l2": "no flush: the cache read each step is larger than L2"
                   if algorithmic_bytes(w)["total"] > 126e6 * 4 else
                   "L2 flushed between steps"}
 
 
 # -------------------------------------------------------------- GPU bench
+class DeviceWorkload:
+    """One workload's cache and decode inputs on the GPU."""
+
+    def __init__(self, w: W.Workload, dev, chunk: int):
+        import torch
+        from paged_int8_kv_b200.runtime import PagedKV8Cache, fill_from_host
+        self.w = w
+        self.chunk = chunk
+        self.cache = PagedKV8Cache(w.num_blocks, w.num_kv_heads, device=dev)
+        fill_from_host(self.cache, w.fill_segments())
+        kn, vn, sl = w.step_tokens()
+        self.host_step = (kn, vn, sl)
+        self.k_new = torch.from_numpy(kn).view(torch.bfloat16).to(dev)
+        self.v_new = torch.from_numpy(vn).view(torch.bfloat16).to(dev)
+        self.slots = torch.from_numpy(sl).to(dev)
+        self.q = torch.from_numpy(w.q()).view(torch.bfloat16).to(dev)
+        self.bt = torch.from_numpy(w.block_tables).to(dev)
+        self.cl = torch.from_numpy(w.context_lens).to(dev)
+        self.out = torch.empty(self.q.shape, dtype=torch.bfloat16, device=dev)
+        self.ws = self.cache.workspace(w.batch, w.num_q_heads,
+                                       w.max_context_len, chunk)
+
+    def append(self, k=None, v=None, s=None):
+        self.cache.append(self.k_new if k is None else k,
+                          self.v_new if v is None else v,
+                          self.slots if s is None else s)
+
+    def decode(self, form, q=None, bt=None, cl=None):
+        import paged_int8_kv_b200 as pk
+        c = self.cache
+        pk.kv8_paged_decode_attention_form(
+            self.q if q is None else q, c.k_cache, c.v_cache, c.k_scales,
+            c.v_scales, self.bt if bt is None else bt,
+            self.cl if cl is None else cl, self.out, self.w.max_context_len,
+            chunk_tokens=self.chunk, workspace=self.ws, form=form)
+
+    def step(self, form):
+        self.append()
+        self.decode(form)
+
+
+def pick_chunk(w: W.Workload, requested: int) -> int:
+    """The split a workload is timed with: the config's own chunk when it
+    names one (``requested`` > 0), else the library's suggestion for this
+    device (kv8_decode_chunk_tokens)."""
+    if requested > 0:
+        return requested
+    import paged_int8_kv_b200 as pk
+    return pk.kv8_decode_chunk_tokens(w.batch, w.num_kv_heads, w.max_context_len)
+
+
+def time_decode_calls(dw: DeviceWorkload, form: int, calls: int, warmup: int,
+                      flush) -> list[float]:
+    """Per-call device time (ms) of the decode entry point, CUDA events on
+    the launching stream, the L2 flushed before each call when ``flush`` is
+    a buffer larger than L2."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        dw.decode(form)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(calls)]
+    for i in range(calls):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        dw.decode(form)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def rate_record(w: W.Workload, dec_ms: float, peak: float) -> dict:
+    ab = algorithmic_bytes(w)
+    gbs = ab["total"] / (dec_ms * 1e-3) / 1e9
+    rec = {"decode_us": dec_ms * 1e3,
+           "tokens_per_s": w.batch / (dec_ms * 1e-3),
+           "kv_tokens_per_s": float(w.context_lens.sum()) / (dec_ms * 1e-3),
+           "algorithmic_bytes": ab["total"], "hbm_gbs": gbs,
+           "frac_of_measured": gbs / peak,
+           "frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS}
+    uniq = unique_kv_bytes(w)
+    if uniq < ab["kv"]:
+        ub = uniq + ab["total"] - ab["kv"]
+        rec["unique_bytes"] = ub
+        rec["hbm_gbs_unique_bytes"] = ub / (dec_ms * 1e-3) / 1e9
+        rec["frac_of_measured_unique_bytes"] = rec["hbm_gbs_unique_bytes"] / peak
+    return rec
+
+
+PER_WORKLOAD = ("tiny", "llama8b_b32", "pruned_compact", "prefix_shared_70b")
+
+
+def run_per_workload(args, dev, peak: float) -> dict:
+    """Decode µs, tokens/s and GB/s of every other configured workload,
+    timed one decode call at a time (median of ``--calls`` calls, L2
+    flushed before each call: these caches fit in or near L2)."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    for name in PER_WORKLOAD:
+        w = W.NAMED[name]()
+        dw = DeviceWorkload(w, dev, pick_chunk(w, 0))
+        dw.append()
+        ms = time_decode_calls(dw, args.kernel, args.calls, 10, flush)
+        rec = rate_record(w, statistics.median(ms), peak)
+        rec.update({"workload": w.name, "chunk_tokens": dw.chunk,
+                    "calls": len(ms), "l2": "flushed before each call",
+                    "stat": "median"})
+        res[name] = rec
+        del dw
+        torch.cuda.empty_cache()
+    del flush
+    return res
+
+
 def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     import torch
     import paged_int8_kv_b200 as pk
-    from paged_int8_kv_b200.runtime import PagedKV8Cache, fill_from_host
 
     dev = torch.device("cuda", _env_int("LOCAL_RANK", 0))
     torch.cuda.set_device(dev)
-    pk.kv8_set_decode_kernel(args.kernel)
     stream = torch.cuda.current_stream()
-
-    cache = PagedKV8Cache(w.num_blocks, w.num_kv_heads, device=dev)
-    fill_from_host(cache, w.fill_segments())
-    kn, vn, sl = w.step_tokens()
-    k_new = torch.from_numpy(kn).view(torch.bfloat16).to(dev)
-    v_new = torch.from_numpy(vn).view(torch.bfloat16).to(dev)
-    slots = torch.from_numpy(sl).to(dev)
-    q = torch.from_numpy(w.q()).view(torch.bfloat16).to(dev)
-    bt = torch.from_numpy(w.block_tables).to(dev)
-    cl = torch.from_numpy(w.context_lens).to(dev)
-    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
-    maxlen = w.max_context_len
-    ws = cache.workspace(w.batch, w.num_q_heads, maxlen, args.chunk)
+    form = args.kernel
+    dw = DeviceWorkload(w, dev, pick_chunk(w, args.chunk))
+    args.chunk = dw.chunk
     flush = None
     ab = algorithmic_bytes(w)
     if ab["total"] <= 4 * 126e6:
@@ -291,21 +428,14 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     # per step: the quantize-append kernel and the decode kernel (a split
     # launch also enqueues a small memset of its merge tickets)
     launches_per_step = 2
-    memsets_per_step = 1 if ws is not None else 0
-
-    def step():
-        cache.append(k_new, v_new, slots)
-        pk.kv8_paged_decode_attention(q, cache.k_cache, cache.v_cache,
-                                      cache.k_scales, cache.v_scales, bt, cl,
-                                      out, maxlen, chunk_tokens=args.chunk,
-                                      workspace=ws)
+    memsets_per_step = 1 if dw.ws is not None else 0
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
     for _ in range(args.warmup):
-        step()
+        dw.step(form)
     torch.cuda.synchronize()
 
     # ---- device-resident timed region
@@ -328,7 +458,7 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     t0 = time.perf_counter()
     while time.perf_counter() - t0 < 1.0:
         for _ in range(20):
-            step()
+            dw.step(form)
         torch.cuda.synchronize()
     barrier()
     t_start = torch.cuda.Event(enable_timing=True)
@@ -338,12 +468,9 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
         if flush is not None:
             flush.fill_(i & 0xFF)
         ev[i][0].record(stream)
-        cache.append(k_new, v_new, slots)
+        dw.append()
         dec[i][0].record(stream)
-        pk.kv8_paged_decode_attention(q, cache.k_cache, cache.v_cache,
-                                      cache.k_scales, cache.v_scales, bt, cl,
-                                      out, maxlen, chunk_tokens=args.chunk,
-                                      workspace=ws)
+        dw.decode(form)
         dec[i][1].record(stream)
         ev[i][1].record(stream)
     t_end.record(stream)
@@ -358,14 +485,15 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     dms = sum(dec_ms) / len(dec_ms)
 
     # ---- end to end through the public API: host buffers in, result out
+    kn, vn, sl = dw.host_step
     pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
     h_k, h_v, h_s = pin(kn), pin(vn), pin(sl)
     h_q, h_bt, h_cl = pin(w.q()), pin(w.block_tables), pin(w.context_lens)
-    h_out = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    h_out = torch.empty(dw.q.shape, dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (h_k, h_v, h_s, h_q, h_bt, h_cl))
     d2h = h_out.numel() * h_out.element_size()
-    d_k, d_v, d_s = torch.empty_like(k_new), torch.empty_like(v_new), torch.empty_like(slots)
-    d_q, d_bt, d_cl = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(cl)
+    d_k, d_v, d_s = torch.empty_like(dw.k_new), torch.empty_like(dw.v_new), torch.empty_like(dw.slots)
+    d_q, d_bt, d_cl = torch.empty_like(dw.q), torch.empty_like(dw.bt), torch.empty_like(dw.cl)
 
     def e2e_step():
         d_k.view(torch.int16).copy_(h_k.view(torch.int16), non_blocking=True)
@@ -374,12 +502,9 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
         d_q.view(torch.int16).copy_(h_q.view(torch.int16), non_blocking=True)
         d_bt.copy_(h_bt, non_blocking=True)
         d_cl.copy_(h_cl, non_blocking=True)
-        cache.append(d_k, d_v, d_s)
-        pk.kv8_paged_decode_attention(d_q, cache.k_cache, cache.v_cache,
-                                      cache.k_scales, cache.v_scales, d_bt,
-                                      d_cl, out, maxlen, chunk_tokens=args.chunk,
-                                      workspace=ws)
-        h_out.copy_(out, non_blocking=True)
+        dw.append(d_k, d_v, d_s)
+        dw.decode(form, d_q, d_bt, d_cl)
+        h_out.copy_(dw.out, non_blocking=True)
 
     # the same lead-in as the device-timed region: about a second of the same
     # steps under load while the clock sampler runs, so that both numbers
@@ -409,28 +534,38 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     ms, dms, e2e_ms = max_over_ranks([ms, dms, e2e_ms], dist, dev)
 
     status = pk.kv8_read_device_status(clear=True)
+    peak, peak_kind = measured_peaks()
+    del dw, flush
+    torch.cuda.empty_cache()
+    # the other workloads, one GPU each rank (rank 0 reports them)
+    per = None
+    if not args.no_per_workload:
+        per = run_per_workload(args, dev, peak)
     if rank != 0:
         return 0
 
-    tokens = w.batch * world
     value = whole_job_rate(w.batch, world, ms)
-    peak, peak_kind = measured_peaks()
     achieved = ab["total"] / (dms * 1e-3) / 1e9
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
         seqs = list(range(min(args.cpu_seqs, w.batch)))
-        sec, desc = oracle_sample_seconds(w, seqs)
-        cpu = {"value": len(seqs) / sec, "unit": UNIT, "cores": 1,
-               "kind": "oracle", "sample": desc}
+        cores = host_cores()
+        sec, desc = oracle_sample_seconds(w, seqs, cores)
+        sec1, desc1 = oracle_sample_seconds(w, seqs, 1)
+        cpu = {"value": len(seqs) / sec, "unit": UNIT, "cores": cores,
+               "kind": "oracle", "sample": desc,
+               "single_thread": {"value": len(seqs) / sec1, "unit": UNIT,
+                                 "cores": 1, "sample": desc1}}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "kv_dtype": "int8", "out_dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 q/K/V, shuffled blocks)",
-        "config": bench_config(w, args),
+        "config": bench_config(w, args, world),
+        "decode_form": form,
         "hbm_gbs": achieved,
         **({"hbm_gbs_unique_bytes": (uniq + ab["total"] - ab["kv"]) / (dms * 1e-3) / 1e9,
             "unique_bytes": uniq + ab["total"] - ab["kv"]}
@@ -438,11 +573,13 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
         "hbm_frac_of_measured": achieved / peak,
         "hbm_frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
         "decode_us": dms * 1e3,
+        "decode_us_x_sm_mhz": (dms * 1e3 * clocks["sm_mhz"]
+                               if clocks and clocks.get("sm_mhz") else None),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                                     if peak_kind == "measured" else "fallback 6650 GB/s",
-                     "kernel": "decode_kernel (split-K pages + fused chunk merge), "
+                     "kernel": "decode kernel (split-K pages + fused chunk merge), "
                                "timed as the kv8_paged_decode_attention call",
                      "algorithmic_bytes": ab["total"],
                      "traffic": recorded_traffic(w.name)},
@@ -453,10 +590,51 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
         "memsets": memsets_per_step * args.steps,
         "clocks": clocks,
         "device_status": status,
+        "per_workload": per,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def run_dry_cpu(args, rank: int, world: int, dist):
+    """The launch and rank logic alone, on CPU ranks over gloo: every rank
+    times a trivial host step, the max over ranks is taken, rank 0 prints a
+    line marked as a dry run (no measurement: value is null)."""
+    for _ in range(args.warmup):
+        time.sleep(0.001)
+    if dist is not None:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time.sleep(0.001)
+    ms = (time.perf_counter() - t0) * 1e3 / args.steps
+    ms = max_over_ranks([ms], dist, None)[0]
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "metric": METRIC, "value": None,
+                          "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                          "warmup": args.warmup, "ms_per_step_host": ms,
+                          "ranks_seen": world}), flush=True)
+    return 0
+
+
+def _free_port() -> int:
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def spawn_ranks(n: int) -> int:
+    """Re-launch this command as n ranks, one process per GPU (the same
+    launch the multi-GPU driver uses), and return its exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(_free_port()), os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.call(cmd)
 
 
 def main():
@@ -466,28 +644,47 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kv8", choices=["kv8", "reference"])
     ap.add_argument("--workload", default="llama8b_b64_32k", choices=sorted(W.NAMED))
-    ap.add_argument("--chunk", type=int, default=512)
-    ap.add_argument("--kernel", type=int, default=0, help="0 auto, 1 CUDA-core, 2 mma.sync tensor-core, 3 tcgen05")
-    ap.add_argument("--cpu-seqs", type=int, default=4)
+    ap.add_argument("--chunk", type=int, default=512,
+                    help="chunk_tokens of the timed workload (0: the library's "
+                         "suggestion for this device)")
+    ap.add_argument("--kernel", type=int, default=0,
+                    help="decode form: 0 auto, 1 CUDA-core, 2 mma.sync tensor-core, 3 tcgen05")
+    ap.add_argument("--calls", type=int, default=50,
+                    help="timed decode calls per workload in per_workload")
+    ap.add_argument("--cpu-seqs", type=int, default=8)
     ap.add_argument("--ref-seqs", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true")
+    ap.add_argument("--dry-run-cpu", action="store_true",
+                    help="rank/launch logic only, on CPU over gloo (no GPU work, "
+                         "no measurement)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    w = W.NAMED[args.workload]()
 
     world = _env_int("WORLD_SIZE", 1)
     rank = _env_int("RANK", 0)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return spawn_ranks(args.gpus)
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}",
+              file=sys.stderr)
+        return 2
     if args.impl == "reference":
-        return run_reference(args, w, rank)
+        return run_reference(args, W.NAMED[args.workload](), rank)
     dist = None
     if world > 1:
         import datetime
-        import torch
         import torch.distributed as dist
-        torch.cuda.set_device(_env_int("LOCAL_RANK", 0))
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        if args.dry_run_cpu:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        else:
+            import torch
+            torch.cuda.set_device(_env_int("LOCAL_RANK", 0))
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        return run_kv8(args, w, rank, world, dist)
+        if args.dry_run_cpu:
+            return run_dry_cpu(args, rank, world, dist)
+        return run_kv8(args, W.NAMED[args.workload](), rank, world, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()

@@ -16,7 +16,8 @@
  * Conventions shared by every entry point
  *   - Every pointer argument except the stream is a DEVICE pointer owned by
  *     the caller.  The library allocates nothing and keeps no state between
- *     calls.
+ *     calls that changes a result (it caches only per-device facts such as
+ *     the SM count, and the device status word below).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is enqueued asynchronously; a KV8_OK return means the
  *     work was launched, not that it finished.
@@ -109,6 +110,24 @@ KV8_API size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
                                   int32_t chunk_tokens);
 
 /*
+ * kv8_decode_chunk_tokens -- a chunk_tokens for kv8_paged_decode_attention
+ * that keeps every SM of the current device busy.
+ *
+ * The split is a scheduling choice the pages leave open.  A decode launch
+ * hands one (sequence, KV head, chunk) to each warp at a time, about 12
+ * warps per SM; with few sequences or short contexts whole chunks leave
+ * warps idle and make the slowest warp's chain of pages the launch time.
+ * This returns the chunk length, a multiple of 16 between 64 and 512, that
+ * cuts max_context_len into equal chunks so that batch * num_kv_heads *
+ * chunks is at least about three times the resident warps of the current
+ * device (148 SMs are assumed when no device can be queried), or 0 (no
+ * split) when max_context_len <= 64.  Size the workspace with the returned
+ * value (kv8_decode_workspace_bytes).  Returns 0 for non-positive arguments.
+ */
+KV8_API int32_t kv8_decode_chunk_tokens(int32_t batch, int32_t num_kv_heads,
+                                        int32_t max_context_len);
+
+/*
  * kv8_paged_decode_attention -- one decode step of GQA attention over the
  * paged INT8 cache, for one new query token per sequence.
  *
@@ -178,22 +197,47 @@ KV8_API int32_t kv8_split_reduce(const void *workspace, size_t workspace_bytes,
                          int32_t max_context_len, int32_t chunk_tokens,
                          void *out, int32_t out_dtype, void *stream);
 
+/* Decode forms for kv8_paged_decode_attention_form. */
+#define KV8_FORM_AUTO 0      /* what kv8_paged_decode_attention uses */
+#define KV8_FORM_CUDA_CORE 1 /* codes converted to fp32, fp32 FMA */
+#define KV8_FORM_MMA_F16PV 2 /* warp mma: int8 q.k, fp16 p.v */
+#define KV8_FORM_TCGEN05 3   /* 5th-generation tensor cores, TMEM accumulators */
+#define KV8_FORM_MMA_I8 4    /* warp mma: int8 q.k, int8 p.v on raw V codes */
+
 /*
- * kv8_set_decode_kernel -- choose how kv8_paged_decode_attention computes a
- * page (process-wide, for tuning and for comparing the forms):
- *   0  automatic (default),
- *   1  CUDA-core form: codes converted to fp32 in registers, fp32 FMA,
- *   2  warp tensor-core form (mma.sync): q.k as int8 products of the K codes
- *      with exact int8 digit planes of q; p.v on V codes converted exactly
- *      to fp16 with fp32 accumulation,
- *   3  tcgen05 form: q.k and p.v both as int8 products on the 5th-generation
- *      tensor cores (digit planes of q and of the probabilities), int32
- *      accumulators in tensor memory, K and V codes read as TMA stages them.
- * All compute the same function; results differ only by rounding order.
- * Returns KV8_ERR_INVALID_ARG for any other value.  Not thread-safe with
- * respect to concurrent decode calls.
+ * kv8_paged_decode_attention_form -- kv8_paged_decode_attention with the
+ * decode form chosen by the caller, for every call separately:
+ *   KV8_FORM_AUTO       the form kv8_paged_decode_attention uses,
+ *   KV8_FORM_CUDA_CORE  codes converted to fp32 in registers, fp32 FMA,
+ *   KV8_FORM_MMA_F16PV  warp tensor cores (mma.sync): q.k as int8 products
+ *                       of the K codes with exact int8 digit planes of q;
+ *                       p.v on V codes converted exactly to fp16, fp32
+ *                       accumulation,
+ *   KV8_FORM_TCGEN05    q.k and p.v both as int8 products on the
+ *                       5th-generation tensor cores (digit planes of q and of
+ *                       the probabilities), int32 accumulators in tensor
+ *                       memory, K and V codes read as TMA stages them,
+ *   KV8_FORM_MMA_I8     warp tensor cores (mma.sync), both products int8:
+ *                       q.k as in KV8_FORM_MMA_F16PV; p.v multiplies the V
+ *                       codes as stored (a transposing shared-memory load)
+ *                       by exact byte planes of the integer-rounded
+ *                       probabilities, int32 accumulation.  Groups of 1, 2
+ *                       or 4 query heads per KV head; a group of 8 runs
+ *                       KV8_FORM_MMA_F16PV.
+ * Every form computes the same function; results differ only by rounding
+ * order, each within the accuracy kv8_paged_decode_attention states.  Any
+ * other `form` returns KV8_ERR_INVALID_ARG.  The choice lives in the call:
+ * the library keeps no selector between calls.
  */
-KV8_API int32_t kv8_set_decode_kernel(int32_t kind);
+KV8_API int32_t kv8_paged_decode_attention_form(
+    const void *q, const int8_t *k_cache, const int8_t *v_cache,
+    const float *k_scales, const float *v_scales, const int32_t *block_tables,
+    const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void *workspace,
+    size_t workspace_bytes, void *out, int32_t out_dtype, int32_t form,
+    void *stream);
 
 /*
  * kv8_read_device_status -- synchronise the current device, then read the
@@ -224,11 +268,15 @@ KV8_API int32_t kv8_read_device_status(uint32_t *status, int32_t clear);
  *     same arguments) returns KV8_ERR_WORKSPACE and launches nothing; use a
  *     larger chunk_tokens (fewer chunks) or the allocating entry point.
  *   - The first call on each device looks up the array's device address on
- *     that device (cudaGetSymbolAddress); make that first call before any
- *     stream capture.
- *   - Every call shares the one array, which keeps the last call's contents;
- *     nothing in it has to start at zero.  Calls whose kernels overlap on the
- *     GPU (e.g. on unordered streams) race on it: order them.
+ *     that device (cudaGetSymbolAddress) and keeps it; make that first call
+ *     before any stream capture.  Resetting the device after that first call
+ *     is not supported (the kept address would be stale).
+ *   - Every call shares the one array, which keeps the last call's contents.
+ *     The chunk partials need no initial value; the merge tickets at the end
+ *     of the array must start at zero, and each call clears them on its
+ *     stream before its kernel.  Calls whose kernels overlap on the GPU
+ *     (e.g. on unordered streams) race on the partials and the tickets:
+ *     order them.
  */
 #define KV8_NOALLOC_WORKSPACE_BYTES (16u << 20) /* 16 MiB per device */
 

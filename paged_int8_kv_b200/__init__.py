@@ -14,11 +14,15 @@ import importlib
 
 _BINDING_NAMES = {
     "EXPORTED", "KV8_ERR_CUDA", "KV8_ERR_INVALID_ARG", "KV8_ERR_UNSUPPORTED",
-    "KV8_ERR_WORKSPACE", "KV8_OK", "KV8_OUT_BF16", "KV8_OUT_F32", "LIB_PATH",
-    "Kv8Error", "default_softmax_scale", "kv8_decode_workspace_bytes",
-    "kv8_paged_decode_attention", "kv8_paged_decode_attention_noalloc",
+    "KV8_ERR_WORKSPACE", "KV8_FORM_AUTO", "KV8_FORM_CUDA_CORE",
+    "KV8_FORM_MMA_F16PV", "KV8_FORM_MMA_I8", "KV8_FORM_TCGEN05", "KV8_OK", "KV8_OUT_BF16",
+    "KV8_OUT_F32", "LIB_PATH",
+    "Kv8Error", "default_softmax_scale", "kv8_decode_chunk_tokens",
+    "kv8_decode_workspace_bytes",
+    "kv8_paged_decode_attention", "kv8_paged_decode_attention_form",
+    "kv8_paged_decode_attention_noalloc",
     "kv8_quantize_append",
-    "kv8_read_device_status", "kv8_set_decode_kernel", "kv8_split_reduce",
+    "kv8_read_device_status", "kv8_split_reduce",
     "kv8_status_string",
 }
 _RUNTIME_NAMES = {"PagedKV8Cache", "fill_from_host"}

@@ -24,14 +24,20 @@ KV8_ERR_WORKSPACE = 3
 KV8_ERR_CUDA = 4
 KV8_OUT_BF16 = 0
 KV8_OUT_F32 = 1
+KV8_FORM_AUTO = 0
+KV8_FORM_CUDA_CORE = 1
+KV8_FORM_MMA_F16PV = 2
+KV8_FORM_TCGEN05 = 3
+KV8_FORM_MMA_I8 = 4
 
 EXPORTED = (
     "kv8_status_string",
     "kv8_quantize_append",
     "kv8_decode_workspace_bytes",
+    "kv8_decode_chunk_tokens",
     "kv8_paged_decode_attention",
     "kv8_split_reduce",
-    "kv8_set_decode_kernel",
+    "kv8_paged_decode_attention_form",
     "kv8_read_device_status",
     "kv8_paged_decode_attention_noalloc",
 )
@@ -57,14 +63,18 @@ def _load() -> ctypes.CDLL:
     lib.kv8_quantize_append.argtypes = [P, P, P, i64, i32, i32, i32, i64, P, P, P, P, P]
     lib.kv8_decode_workspace_bytes.restype = sz
     lib.kv8_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    lib.kv8_decode_chunk_tokens.restype = i32
+    lib.kv8_decode_chunk_tokens.argtypes = [i32, i32, i32]
     lib.kv8_paged_decode_attention.restype = i32
     lib.kv8_paged_decode_attention.argtypes = [
         P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
         P, sz, P, i32, P]
     lib.kv8_split_reduce.restype = i32
     lib.kv8_split_reduce.argtypes = [P, sz, P, i32, i32, i32, i32, i32, P, i32, P]
-    lib.kv8_set_decode_kernel.restype = i32
-    lib.kv8_set_decode_kernel.argtypes = [i32]
+    lib.kv8_paged_decode_attention_form.restype = i32
+    lib.kv8_paged_decode_attention_form.argtypes = [
+        P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
+        P, sz, P, i32, i32, P]
     lib.kv8_paged_decode_attention_noalloc.restype = i32
     lib.kv8_paged_decode_attention_noalloc.argtypes = [
         P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
@@ -117,6 +127,26 @@ def kv8_decode_workspace_bytes(batch: int, num_q_heads: int, head_dim: int,
                                               max_context_len, chunk_tokens))
 
 
+def kv8_decode_chunk_tokens(batch: int, num_kv_heads: int,
+                            max_context_len: int) -> int:
+    """Suggested chunk_tokens for this device (0: no split)."""
+    return int(lib.kv8_decode_chunk_tokens(batch, num_kv_heads, max_context_len))
+
+
+def _decode_args(q, k_cache, v_cache, k_scales, v_scales, block_tables,
+                 context_lens, out, max_context_len, chunk_tokens, workspace,
+                 softmax_scale):
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    out_dtype = KV8_OUT_F32 if out.dtype == torch.float32 else KV8_OUT_BF16
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return (_p(q), _p(k_cache), _p(v_cache), _p(k_scales), _p(v_scales),
+            _p(block_tables), _p(context_lens), B, hq, hkv, d, bs,
+            block_tables.shape[1], nb, int(max_context_len),
+            float(softmax_scale), int(chunk_tokens), _p(workspace), ws_bytes,
+            _p(out), out_dtype)
+
+
 def kv8_paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor,
                                v_cache: torch.Tensor, k_scales: torch.Tensor,
                                v_scales: torch.Tensor,
@@ -127,16 +157,32 @@ def kv8_paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor,
                                softmax_scale: float = 0.0,
                                stream=None) -> torch.Tensor:
     """q bf16 [B, H_q, D]; out bf16 or fp32 [B, H_q, D] (written in place)."""
-    B, hq, d = q.shape
-    nb, hkv, bs, _ = k_cache.shape
-    out_dtype = KV8_OUT_F32 if out.dtype == torch.float32 else KV8_OUT_BF16
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("kv8_paged_decode_attention", lib.kv8_paged_decode_attention(
-        _p(q), _p(k_cache), _p(v_cache), _p(k_scales), _p(v_scales),
-        _p(block_tables), _p(context_lens), B, hq, hkv, d, bs,
-        block_tables.shape[1], nb, int(max_context_len), float(softmax_scale),
-        int(chunk_tokens), _p(workspace), ws_bytes, _p(out), out_dtype,
-        _stream(stream)))
+        *_decode_args(q, k_cache, v_cache, k_scales, v_scales, block_tables,
+                      context_lens, out, max_context_len, chunk_tokens,
+                      workspace, softmax_scale), _stream(stream)))
+    return out
+
+
+def kv8_paged_decode_attention_form(q: torch.Tensor, k_cache: torch.Tensor,
+                                    v_cache: torch.Tensor,
+                                    k_scales: torch.Tensor,
+                                    v_scales: torch.Tensor,
+                                    block_tables: torch.Tensor,
+                                    context_lens: torch.Tensor,
+                                    out: torch.Tensor, max_context_len: int,
+                                    chunk_tokens: int = 512,
+                                    workspace: torch.Tensor | None = None,
+                                    softmax_scale: float = 0.0,
+                                    form: int = KV8_FORM_AUTO,
+                                    stream=None) -> torch.Tensor:
+    """kv8_paged_decode_attention with the decode form given for this call."""
+    _check("kv8_paged_decode_attention_form",
+           lib.kv8_paged_decode_attention_form(
+               *_decode_args(q, k_cache, v_cache, k_scales, v_scales,
+                             block_tables, context_lens, out, max_context_len,
+                             chunk_tokens, workspace, softmax_scale),
+               int(form), _stream(stream)))
     return out
 
 
@@ -175,10 +221,6 @@ def kv8_split_reduce(workspace: torch.Tensor, context_lens: torch.Tensor,
         _p(context_lens), B, hq, d, int(max_context_len), int(chunk_tokens),
         _p(out), out_dtype, _stream(stream)))
     return out
-
-
-def kv8_set_decode_kernel(kind: int) -> None:
-    _check("kv8_set_decode_kernel", lib.kv8_set_decode_kernel(int(kind)))
 
 
 def kv8_read_device_status(clear: bool = True) -> int:

@@ -1,11 +1,15 @@
 """Build libkv8.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-    python -m paged_int8_kv_b200.build [--force] [--verbose]
+    python -m paged_int8_kv_b200.build [--force] [--verbose] [--test-hooks]
 
 Each ``csrc/*.cu`` is compiled by nvcc for ``sm_100a`` and the objects are
 linked into ``paged_int8_kv_b200/libkv8.so`` with the CUDA runtime linked
 statically, so the library needs nothing at load time beyond the driver.
 nvcc cross-compiles, so this runs on a machine without a GPU.
+
+``--test-hooks`` builds ``libkv8_testhooks.so`` instead: the same sources
+with ``-DKV8_TEST_HOOKS`` (short bounded waits and the switches declared in
+``csrc/kv8_test_hooks.h``), loaded only by the tests of the give-up path.
 """
 from __future__ import annotations
 
@@ -19,6 +23,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libkv8.so")
+TEST_LIB = os.path.join(HERE, "libkv8_testhooks.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -46,39 +51,43 @@ def _deps():
             [os.path.join(ROOT, "include", "kv8.h"), __file__])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          test_hooks: bool = False) -> str:
+    lib = TEST_LIB if test_hooks else LIB
+    if not force and up_to_date(lib):
+        return lib
+    bdir = os.path.join(BUILD, "testhooks") if test_hooks else BUILD
+    os.makedirs(bdir, exist_ok=True)
     nvcc = _nvcc()
+    extra = ["-DKV8_TEST_HOOKS"] if test_hooks else []
     objs = []
     for src in _sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
+        cmd = [nvcc, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
         if ptxas_info:
             cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
            "-cudart", "static", "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
-          ptxas_info="--ptxas-info" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                ptxas_info="--ptxas-info" in sys.argv,
+                test_hooks="--test-hooks" in sys.argv))

@@ -8,6 +8,7 @@
 
 #include "../../include/kv8.h"
 #include "kv8_internal.h"
+#include "kv8_test_hooks.h"
 
 namespace {
 
@@ -74,8 +75,6 @@ void split_shape(int32_t max_context_len, int32_t chunk_tokens,
   }
 }
 
-int32_t g_decode_kernel = 0;  // 0 auto, 1 CUDA-core, 2 mma.sync, 3 tcgen05
-
 }  // namespace
 
 extern "C" {
@@ -129,6 +128,35 @@ size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
   return kv8::workspace_total_bytes(batch, num_q_heads, max_chunks);
 }
 
+int32_t kv8_decode_chunk_tokens(int32_t batch, int32_t num_kv_heads,
+                                int32_t max_context_len) {
+  if (batch <= 0 || num_kv_heads <= 0 || max_context_len <= 0) return 0;
+  constexpr int32_t kMinChunk = 4 * kBlockSize, kMaxChunk = 32 * kBlockSize;
+  constexpr int64_t kWarpsPerSM = 12;
+  if (max_context_len <= kMinChunk) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+          cudaSuccess ||
+      sms <= 0) {
+    cudaGetLastError();  // no device here: clear the sticky error
+    sms = 148;
+  }
+  const int64_t want_items = 3 * kWarpsPerSM * sms;
+  const int64_t units = static_cast<int64_t>(batch) * num_kv_heads;
+  const int64_t splits = (want_items + units - 1) / units;
+  int64_t chunk = (max_context_len + splits - 1) / splits;
+  chunk = (chunk + kBlockSize - 1) / kBlockSize * kBlockSize;
+  if (chunk < kMinChunk) chunk = kMinChunk;
+  if (chunk > kMaxChunk) {
+    // equal chunks of at most kMaxChunk tokens
+    const int64_t n = (max_context_len + kMaxChunk - 1) / kMaxChunk;
+    chunk = (max_context_len + n - 1) / n;
+    chunk = (chunk + kBlockSize - 1) / kBlockSize * kBlockSize;
+  }
+  return static_cast<int32_t>(chunk);
+}
+
 int32_t kv8_paged_decode_attention(
     const void* q, const int8_t* k_cache, const int8_t* v_cache,
     const float* k_scales, const float* v_scales, const int32_t* block_tables,
@@ -137,6 +165,24 @@ int32_t kv8_paged_decode_attention(
     int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
     float softmax_scale, int32_t chunk_tokens, void* workspace,
     size_t workspace_bytes, void* out, int32_t out_dtype, void* stream) {
+  return kv8_paged_decode_attention_form(
+      q, k_cache, v_cache, k_scales, v_scales, block_tables, context_lens,
+      batch, num_q_heads, num_kv_heads, head_dim, block_size,
+      max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+      chunk_tokens, workspace, workspace_bytes, out, out_dtype, KV8_FORM_AUTO,
+      stream);
+}
+
+int32_t kv8_paged_decode_attention_form(
+    const void* q, const int8_t* k_cache, const int8_t* v_cache,
+    const float* k_scales, const float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void* workspace,
+    size_t workspace_bytes, void* out, int32_t out_dtype, int32_t form,
+    void* stream) {
+  if (form < KV8_FORM_AUTO || form > KV8_FORM_MMA_I8) return KV8_ERR_INVALID_ARG;
   // ---- shape checks
   if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
@@ -214,9 +260,9 @@ int32_t kv8_paged_decode_attention(
       cudaMemsetAsync(ws_ctr, 0, kv8::workspace_ctr_bytes(batch, num_q_heads),
                       st) != cudaSuccess)
     return KV8_ERR_CUDA;
-  int rc = g_decode_kernel == 3
+  int rc = form == KV8_FORM_TCGEN05
                ? kv8::launch_decode_tc(p, tmk, tmv, st)
-               : kv8::launch_decode(p, tmk, tmv, g_decode_kernel, st);
+               : kv8::launch_decode(p, tmk, tmv, form, st);
   if (rc == -2) return KV8_ERR_UNSUPPORTED;
   if (rc != 0) return KV8_ERR_CUDA;
   return KV8_OK;
@@ -253,11 +299,11 @@ int32_t kv8_split_reduce(const void* workspace, size_t workspace_bytes,
   return rc == 0 ? KV8_OK : KV8_ERR_CUDA;
 }
 
-int32_t kv8_set_decode_kernel(int32_t kind) {
-  if (kind < 0 || kind > 3) return KV8_ERR_INVALID_ARG;
-  g_decode_kernel = kind;
-  return KV8_OK;
+#ifdef KV8_TEST_HOOKS
+int32_t kv8_test_skip_first_copy(int32_t on) {
+  return kv8::test_skip_first_copy(on != 0) == 0 ? KV8_OK : KV8_ERR_CUDA;
 }
+#endif
 
 int32_t kv8_read_device_status(uint32_t* status, int32_t clear) {
   if (!status) return KV8_ERR_INVALID_ARG;

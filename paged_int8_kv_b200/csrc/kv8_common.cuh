@@ -21,8 +21,14 @@ enum : uint32_t {
 
 // Upper bound on mbarrier polls before a wait gives up (each poll may also
 // suspend the thread for a short hardware-chosen time): far above any real
-// latency of a 4 KB copy, a second or so in the worst case.
+// latency of a 4 KB copy, a second or so in the worst case.  The test-hook
+// build (KV8_TEST_HOOKS) gives up after a few milliseconds instead, so that
+// its test of the give-up path is short.
+#ifdef KV8_TEST_HOOKS
+constexpr uint32_t kMaxWaitPolls = 1u << 12;
+#else
 constexpr uint32_t kMaxWaitPolls = 1u << 24;
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

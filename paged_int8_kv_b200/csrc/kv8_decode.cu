@@ -27,6 +27,7 @@
 //     normalised output for a sequence that fits one chunk, else the chunk's
 //     (m, l, o) partial; the last chunk of each (sequence, KV group) to
 //     finish (a ticket, never a wait) merges the partials by log-sum-exp.
+#include "../../include/kv8.h"
 #include "kv8_common.cuh"
 #include "kv8_internal.h"
 #include "kv8_merge.cuh"
@@ -34,6 +35,13 @@
 namespace kv8 {
 
 __device__ uint32_t g_device_status = 0;
+
+#ifdef KV8_TEST_HOOKS
+// Test-hook build only: when set, warp 0 of CTA 0 arms the mbarrier of its
+// first page (expect-tx) but issues none of that page's copies, so its wait
+// for that page runs out; nothing is copied, nothing faults.
+__device__ int g_test_skip_first_copy = 0;
+#endif
 
 namespace {
 
@@ -47,14 +55,17 @@ constexpr uint32_t kPageTx = 2 * kPageBytes + 2 * kBS * sizeof(float);
 // to 1024 bytes):
 //   per warp w: SPW slots of [K page 2048 B | V page 2048 B]   (tiles)
 //   per warp w: SPW slots of [ks 64 B | vs 64 B]              (scales)
+//   per warp w: the page math's scratch (ScratchBytes, may be 0)
 //   per warp w: SPW mbarriers
 // --------------------------------------------------------------------------
-template <int WPC, int SPW>
+template <int WPC, int SPW, int ScratchBytes = 0>
 struct SmemPlan {
   static constexpr int kTileBytes = WPC * SPW * 2 * kPageBytes;
   static constexpr int kScaleBytes = WPC * SPW * 2 * kBS * 4;
+  static constexpr int kScratchBytes = WPC * ScratchBytes;
   static constexpr int kBarBytes = WPC * SPW * 8;
-  static constexpr int kBytes = kTileBytes + kScaleBytes + kBarBytes + 1024;
+  static constexpr int kBytes =
+      kTileBytes + kScaleBytes + kScratchBytes + kBarBytes + 1024;
 };
 
 // Transposed butterfly reduction of G per-lane partial sums over a group of
@@ -134,6 +145,7 @@ struct ChunkSink {
 template <int G>
 struct SimtMath {
   static constexpr int kWarpsPerSM = 0;  // no register cap
+  static constexpr int kScratchBytes = 0;
   static constexpr int DPL = (G <= 4) ? 16 : 8;  // dims per lane
   static constexpr int LPT = kD / DPL;           // lanes per token
   static constexpr int TPP = 32 / LPT;           // tokens per pass
@@ -142,6 +154,8 @@ struct SimtMath {
 
   int lane, tg, dg, hh;
   float2 q2[G][DPL / 2];
+
+  __device__ __forceinline__ void attach(uint8_t*) {}
   float2 o2[G][DPL / 2];
   float m_run, l_run;
 
@@ -196,6 +210,7 @@ struct SimtMath {
     }
   }
 
+  template <bool Full>
   __device__ __forceinline__ void page(const uint8_t* tk, const uint8_t* tv,
                                        const float* ks, const float* vs,
                                        int nv) {
@@ -387,6 +402,7 @@ __device__ __forceinline__ uint32_t word_of(const uint4& a, int i) {
 template <int G>
 struct MmaMath {
   static constexpr int kWarpsPerSM = 12;  // cap registers at 168 per thread
+  static constexpr int kScratchBytes = 0;
   static constexpr float kSlack = 8.0f;   // log2 units
   static constexpr int kVSlack = 4;
   int lane, r, c;
@@ -398,6 +414,8 @@ struct MmaMath {
   int e_run;        // P'' carries 2^-e_run (warp-uniform)
   float vlim;       // 2^(e_run + kVSlack)
   float fs;         // 2^-e_run
+
+  __device__ __forceinline__ void attach(uint8_t*) {}
 
   __device__ __forceinline__ void init(const __nv_bfloat16* qg, float q_scale,
                                        int lane_) {
@@ -474,6 +492,7 @@ struct MmaMath {
       for (int j = 0; j < 4; ++j) ot[i][j] = 0.0f;
   }
 
+  template <bool Full>
   __device__ __forceinline__ void page(const uint8_t* tk, const uint8_t* tv,
                                        const float* ks, const float* vs,
                                        int nv) {
@@ -637,6 +656,325 @@ struct MmaMath {
   }
 };
 
+// s8 x u8 integer mma: D[16x8] (s32) += A[16x16] (s8, row) . B[16x8] (u8, col).
+__device__ __forceinline__ void mma16816_s8u8(int (&d)[4], uint32_t a0,
+                                              uint32_t a1, uint32_t b0) {
+  asm("mma.sync.aligned.m16n8k16.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, "
+      "{%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+// Two 16 x 16 byte matrices from shared memory, each transposed into the A
+// fragment of an m16n8k16 int8 mma: lanes 0..15 address the 16 source rows
+// (16 bytes each) of matrix 0, lanes 16..31 those of matrix 1; thread
+// (g = lane / 4, t = lane % 4) receives source rows 4t..4t+3 of column g
+// (r0: matrix 0, r2: matrix 1) and of column g + 8 (r1, r3).
+__device__ __forceinline__ void ldsm_x2_trans_b8(uint32_t addr, uint32_t& r0,
+                                                 uint32_t& r1, uint32_t& r2,
+                                                 uint32_t& r3) {
+  asm volatile(
+      "ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(addr)
+      : "memory");
+}
+
+// Integer tensor-core form for groups of G <= 4 query heads: both products
+// on int8 mma, no code is converted on the CUDA cores.
+//   S[16 rows x 16 tok] = Qd[16 x 128] . K_code^T        (m16n8k32 s8, exact)
+//   O^T[128 x 16 col]  += V_code^T[128 x 16 tok] . Pd^T   (m16n8k16 s8.u8)
+// * Token <-> lane map: thread (r = lane/4, c = lane%4) ends up with the
+//   scores of tokens 4c..4c+3; q.k n-tile j column n is token
+//   4(n/2) + 2j + (n%2), and the p.v k index is the token itself.  Under the
+//   TMA's 128-byte swizzle every shared-memory read below is then
+//   bank-conflict free.
+// * q.k rows: thread row r holds head hr = (r % 4) % G; its rows r and r+8
+//   carry two of the four balanced int8 digit planes of q (Q = rint(q 2^sh),
+//   max|Q| in [2^29, 2^30), Q = sum_p 2^(8p) d_p): planes 3 and 1 for r < 4,
+//   2 and 0 for r >= 4.  Lanes L and L^16 hold the same head and add their
+//   two partial scores, so both end with the full score; 8 mma per page.
+//   The digits are the bytes of Q + 0x80808080, each minus 128: the unique
+//   balanced base-256 representation.
+// * p.v: P'' = 2^(s - m) vs 2^-e (lazy references as in MmaMath) is rounded
+//   to the integer P = rint(P'' 2^kF) < 2^31, whose four bytes are exact
+//   unsigned digit planes.  Column n of p.v n-tile t is (head hr(n), plane
+//   2t + n/4); the V codes enter as the A operand straight from shared
+//   memory through a transposing ldmatrix.  16 mma per page into int32
+//   accumulators (|acc| < 127 * 255 * tokens: no overflow below 66K tokens
+//   between drains).
+// * The int32 accumulators are drained (converted, weighted 2^(8p - kF),
+//   and added to fp32 partials kept in this warp's shared-memory scratch)
+//   when the references move and at the end of an item.  The two lanes
+//   c and c^2 hold complementary planes of the same outputs and are summed
+//   at the end.
+template <int G>
+struct I8Math {
+  static_assert(G == 1 || G == 2 || G == 4, "groups of 1, 2 or 4 heads");
+  static constexpr int kWarpsPerSM = 12;  // cap registers at 168 per thread
+  static constexpr int kScratchBytes = 32 * 32 * 4;  // fp32 [32][lane]
+  static constexpr float kSlack = 6.0f;   // log2 units
+  static constexpr int kVSlack = 2;
+  static constexpr int kF = 23;  // P'' < 2^(kSlack + kVSlack): P < 2^31
+  // lowest V-scale exponent tracked, so that 2^(kF - e) stays a normal
+  // float; V scales below 2^kMinE keep fewer bits of P (they are zero in
+  // any practical cache)
+  static constexpr int kMinE = kF - 127;
+  int lane, r, c, up;
+  uint32_t qa[4][4];  // A fragments of Qd per k-step: rows r / r+8, k halves
+  float qf;           // score factor of head hr: 2^-sh * softmax_scale * log2(e)
+  int acc[8][2][4];   // p.v int32 accumulators: m-tile, n-tile, fragment
+  float* of;          // this warp's drained fp32 partials, [32][lane]
+  float m_run, l_run;
+  int e_run;
+  float vlim;         // 2^(e_run + kVSlack)
+  float fsF;          // 2^(kF - e_run)
+  uint32_t psel;      // prmt selector of this thread's two P planes
+  bool started;       // the accumulators or the partials hold something
+  bool of_live;       // the partials hold something
+
+  __device__ __forceinline__ void attach(uint8_t* scratch) {
+    of = reinterpret_cast<float*>(scratch);
+  }
+
+  __device__ __forceinline__ void init(const __nv_bfloat16* qg, float q_scale,
+                                       int lane_) {
+    lane = lane_;
+    r = lane >> 2;
+    c = lane & 3;
+    up = r >> 2;
+    const int h = (r & 3) % G;
+    float qv[32];
+    const uint4* src = reinterpret_cast<const uint4*>(qg + h * kD + 32 * c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 raw = src[i];
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        qv[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+        qv[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qv[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+    const int sh = amax > 0.0f ? 30 - exp_frexp(amax) : 0;
+    const float f1 = pow2i(sh / 2), f2 = pow2i(sh - sh / 2);
+    // bytes (planes) this thread row keeps: rows r -> pa, rows r+8 -> pb
+    const uint32_t pa = up ? 2u : 3u, pb = up ? 0u : 1u;
+    const uint32_t sel = pa | ((4u + pa) << 4) | (pb << 8) | ((4u + pb) << 12);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // dims 32c + 4i .. 32c + 4i + 3
+      uint32_t u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        u[j] = static_cast<uint32_t>(__float2int_rn(qv[4 * i + j] * f1 * f2)) +
+               0x80808080u;
+      const uint32_t x = prmt(u[0], u[1], sel);
+      const uint32_t y = prmt(u[2], u[3], sel);
+      const uint32_t wa = prmt(x, y, 0x5410u) ^ 0x80808080u;
+      const uint32_t wb = prmt(x, y, 0x7632u) ^ 0x80808080u;
+      // k-step s = i / 2 covers dims 32c + 8s .. + 7: a0/a1 the first four
+      // (rows r / r+8), a2/a3 the next four
+      if (i & 1) {
+        qa[i >> 1][2] = wa;
+        qa[i >> 1][3] = wb;
+      } else {
+        qa[i >> 1][0] = wa;
+        qa[i >> 1][1] = wb;
+      }
+    }
+    qf = q_scale * pow2i(-(sh / 2)) * pow2i(-(sh - sh / 2));
+    psel = static_cast<uint32_t>(up) | ((4u + up) << 4) | ((2u + up) << 8) |
+           ((6u + up) << 12);
+    reset();
+  }
+
+  __device__ __forceinline__ void zero_acc() {
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[m][t][e] = 0;
+  }
+
+  __device__ __forceinline__ void reset() {
+    m_run = -INFINITY;
+    l_run = 0.0f;
+    e_run = kMinE;
+    vlim = 0.0f;
+    fsF = pow2i(kF - kMinE);
+    started = false;
+    of_live = false;
+    zero_acc();
+  }
+
+  // partials += planes of the accumulators (weighted), then *= scale of the
+  // output column's head (aA: column 2c, aB: column 2c+1); accumulators := 0
+  __device__ __forceinline__ void drain(float aA, float aB) {
+    const float w0 = pow2i(8 * (c >> 1) - kF);
+    const float w1 = pow2i(16 + 8 * (c >> 1) - kF);
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = m * 4 + e;
+        const float v = __int2float_rn(acc[m][0][e]) * w0 +
+                         __int2float_rn(acc[m][1][e]) * w1;
+        const float old = of_live ? of[k * 32 + lane] : 0.0f;
+        of[k * 32 + lane] = (old + v) * ((e & 1) ? aB : aA);
+      }
+    of_live = true;
+    zero_acc();
+  }
+
+  template <bool Full>
+  __device__ __forceinline__ void page(const uint8_t* tk, const uint8_t* tv,
+                                       const float* ks, const float* vs,
+                                       int nv) {
+    // ---- S = Qd K^T.  n-tile j, column n = r: token 4(r/2) + 2j + r%2
+    const int ta = 4 * (r >> 1) + (r & 1), tb = ta + 2;
+    const uint8_t* ra = tk + ta * 128;
+    const uint8_t* rb = tk + tb * 128;
+    const int sw = ta & 7, swb = tb & 7;
+    const uint4 ka0 = *reinterpret_cast<const uint4*>(ra + (((2 * c) ^ sw) << 4));
+    const uint4 ka1 = *reinterpret_cast<const uint4*>(ra + (((2 * c + 1) ^ sw) << 4));
+    const uint4 kb0 = *reinterpret_cast<const uint4*>(rb + (((2 * c) ^ swb) << 4));
+    const uint4 kb1 = *reinterpret_cast<const uint4*>(rb + (((2 * c + 1) ^ swb) << 4));
+    int sacc[2][4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[j][e] = 0;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const uint4& ka = s < 2 ? ka0 : ka1;
+      const uint4& kb = s < 2 ? kb0 : kb1;
+      mma16832_s8(sacc[0], qa[s][0], qa[s][1], qa[s][2], qa[s][3],
+                  (s & 1) ? ka.z : ka.x, (s & 1) ? ka.w : ka.y);
+      mma16832_s8(sacc[1], qa[s][0], qa[s][1], qa[s][2], qa[s][3],
+                  (s & 1) ? kb.z : kb.x, (s & 1) ? kb.w : kb.y);
+    }
+    // rows r / r+8 hold planes (3, 1) for up == 0 and (2, 0) for up == 1
+    const float wa = up ? 65536.0f : 16777216.0f;
+    const float wb = up ? 1.0f : 256.0f;
+    float st[4];  // tokens 4c + i, i = 2j + e
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float part = __fmaf_rn(__int2float_rn(sacc[j][e]), wa,
+                                     __int2float_rn(sacc[j][2 + e]) * wb);
+        st[2 * j + e] = part + __shfl_xor_sync(kFull, part, 16);
+      }
+    const float4 ks4 = *reinterpret_cast<const float4*>(ks + 4 * c);
+    const float4 vs4 = *reinterpret_cast<const float4*>(vs + 4 * c);
+    const float ksv[4] = {ks4.x, ks4.y, ks4.z, ks4.w};
+    const float vsr[4] = {vs4.x, vs4.y, vs4.z, vs4.w};
+    float sc[4], vsv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (Full) {
+        sc[i] = st[i] * qf * ksv[i];
+        vsv[i] = vsr[i];
+      } else {
+        const bool ok = 4 * c + i < nv;
+        sc[i] = ok ? st[i] * qf * ksv[i] : -INFINITY;
+        vsv[i] = ok ? vsr[i] : 0.0f;
+      }
+    }
+    const float lm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    const float lv = fmaxf(fmaxf(vsv[0], vsv[1]), fmaxf(vsv[2], vsv[3]));
+    if (__any_sync(kFull, lm > m_run + kSlack || lv > vlim)) {
+      float x = fmaxf(lm, __shfl_xor_sync(kFull, lm, 1));
+      x = fmaxf(x, __shfl_xor_sync(kFull, x, 2));
+      float vx = fmaxf(lv, __shfl_xor_sync(kFull, lv, 1));
+      vx = fmaxf(vx, __shfl_xor_sync(kFull, vx, 2));
+      const float n = fmaxf(m_run, x);
+      // every quad sees all 16 tokens' scales: e_new is warp-uniform
+      const int e_new = vx > vlim ? max(exp_frexp(vx), kMinE) : e_run;
+      const float a = (n == m_run) ? 1.0f : ex2(m_run - n);
+      const float a_o = a * pow2i(max(e_run - e_new, -126));
+      if (started) {
+        const int hA = ((2 * c) & 3) % G, hB = ((2 * c + 1) & 3) % G;
+        const float aA = __shfl_sync(kFull, a_o, 4 * hA);
+        const float aB = __shfl_sync(kFull, a_o, 4 * hB);
+        drain(aA, aB);
+      }
+      l_run *= a;
+      m_run = n;
+      e_run = e_new;
+      vlim = pow2i(min(e_new + kVSlack, 127));
+      fsF = pow2i(kF - e_new);
+    }
+    const float mu = m_run == -INFINITY ? 0.0f : m_run;
+    float pr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pr[i] = ex2(sc[i] - mu);
+    l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    uint32_t pi[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pi[i] = __float2uint_rn(pr[i] * (vsv[i] * fsF));
+    // B fragments: bytes = tokens 4c..4c+3, planes up (n-tile 0), 2+up (1)
+    const uint32_t x = prmt(pi[0], pi[1], psel);
+    const uint32_t y = prmt(pi[2], pi[3], psel);
+    const uint32_t b0 = prmt(x, y, 0x5410u);
+    const uint32_t b1 = prmt(x, y, 0x7632u);
+
+    // ---- O^T += V^T Pd^T: ldmatrix rows = tokens 0..15 (lanes 0..15 and
+    //      16..31 address the same tokens in m-tiles 2w and 2w+1)
+    const uint32_t vbase = smem_u32(tv) + (lane & 15) * 128;
+    const int vsw = lane & 7, vmt = lane >> 4;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x2_trans_b8(vbase + (((2 * w + vmt) ^ vsw) << 4), a0, a1, a2, a3);
+      mma16816_s8u8(acc[2 * w][0], a0, a1, b0);
+      mma16816_s8u8(acc[2 * w][1], a0, a1, b1);
+      mma16816_s8u8(acc[2 * w + 1][0], a2, a3, b0);
+      mma16816_s8u8(acc[2 * w + 1][1], a2, a3, b1);
+    }
+    started = true;
+  }
+
+  __device__ __forceinline__ void finish(const ChunkSink& sk) {
+    if (started) drain(1.0f, 1.0f);
+    float l = l_run;
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+    const int nA = 2 * c, nB = 2 * c + 1;  // output columns of this thread
+    const int hA = (nA & 3) % G, hB = (nB & 3) % G;
+    const float sA = __shfl_sync(kFull, l, 4 * hA);
+    const float sB = __shfl_sync(kFull, l, 4 * hB);
+    const float mA = __shfl_sync(kFull, m_run, 4 * hA);
+    const float mB = __shfl_sync(kFull, m_run, 4 * hB);
+    const float f = pow2i(e_run);
+    const bool wA = c < 2 && nA < G, wB = c < 2 && nB < G;
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = m * 4 + e;
+        float v = of_live ? of[k * 32 + lane] : 0.0f;
+        v += __shfl_xor_sync(kFull, v, 2);  // the complementary planes
+        const int d = 16 * m + r + ((e & 2) ? 8 : 0);
+        if (e & 1) {
+          if (wB) sk.put_o(nB, d, v * f, sB);
+        } else {
+          if (wA) sk.put_o(nA, d, v * f, sA);
+        }
+      }
+    if (r == 0) {
+      if (wA) sk.put_ml(nA, mA, sA);
+      if (wB) sk.put_ml(nB, mB, sB);
+    }
+  }
+};
+
 // --------------------------------------------------------------------------
 // The decode kernel.  Persistent: a grid of (SMs x resident CTAs) CTAs of
 // WPC independent warps.  A work item is one (sequence, KV head, context
@@ -649,32 +987,57 @@ struct MmaMath {
 // barriers: each warp writes its chunk's result straight from registers.
 // --------------------------------------------------------------------------
 struct Item {
-  int64_t idx;
-  int b, kvh, chunk, n, tok0, tok1, npages, nchunks;
+  int b, kvh, chunk, n, tok0, tok1, npages;
 };
 
-// Decode item idx; false if the chunk lies past its sequence (a context of
-// length 0 keeps chunk 0, with no pages, so that its zero row is written).
-__device__ __forceinline__ bool item_load(const DecodeParams& p, Item& it) {
+// The warp stride W = (dc * H_kv + dk) * B + db as mixed-radix digits, so
+// that stepping an item is a pair of compare-and-carry steps, no division.
+struct Stride {
+  int dc, dk, db;
+};
+
+__device__ __forceinline__ void item_set(const DecodeParams& p, int64_t idx,
+                                         Item& it) {
   const int64_t per_chunk = static_cast<int64_t>(p.num_kv_heads) * p.batch;
-  it.chunk = static_cast<int>(it.idx / per_chunk);
-  const int64_t rem = it.idx - static_cast<int64_t>(it.chunk) * per_chunk;
+  const int64_t c = idx / per_chunk;
+  const int64_t rem = idx - c * per_chunk;
+  it.chunk = c > p.max_chunks ? p.max_chunks : static_cast<int>(c);
   it.kvh = static_cast<int>(rem / p.batch);
   it.b = static_cast<int>(rem - static_cast<int64_t>(it.kvh) * p.batch);
+}
+
+__device__ __forceinline__ bool item_done(const DecodeParams& p,
+                                          const Item& it) {
+  return it.chunk >= p.max_chunks;
+}
+
+// Fill in the item's extent; false if the chunk lies past its sequence (a
+// context of length 0 keeps chunk 0, with no pages, so that its zero row is
+// written).
+__device__ __forceinline__ bool item_fill(const DecodeParams& p, Item& it) {
   it.n = p.context_lens[it.b];
   it.tok0 = it.chunk * p.chunk_tokens;
   if (it.tok0 >= it.n && !(it.n == 0 && it.chunk == 0)) return false;
   it.tok1 = min(it.n, it.tok0 + p.chunk_tokens);
   it.npages = (it.tok1 - it.tok0 + kBS - 1) / kBS;
-  it.nchunks = (it.n + p.chunk_tokens - 1) / p.chunk_tokens;
   return true;
 }
 
 __device__ __forceinline__ void item_next(const DecodeParams& p, Item& it,
-                                          int64_t stride, int64_t n_items) {
+                                          const Stride& st) {
   do {
-    it.idx += stride;
-  } while (it.idx < n_items && !item_load(p, it));
+    it.b += st.db;
+    it.kvh += st.dk;
+    it.chunk += st.dc;
+    if (it.b >= p.batch) {
+      it.b -= p.batch;
+      ++it.kvh;
+    }
+    if (it.kvh >= p.num_kv_heads) {
+      it.kvh -= p.num_kv_heads;
+      ++it.chunk;
+    }
+  } while (!item_done(p, it) && !item_fill(p, it));
 }
 
 template <int G, int WPC, int SPW, class Math>
@@ -682,7 +1045,7 @@ __global__ void __launch_bounds__(WPC * 32,
                                   Math::kWarpsPerSM / WPC > 0 ? Math::kWarpsPerSM / WPC : 1)
 decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
               const __grid_constant__ CUtensorMap tmv) {
-  using Plan = SmemPlan<WPC, SPW>;
+  using Plan = SmemPlan<WPC, SPW, Math::kScratchBytes>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -691,8 +1054,11 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   uint8_t* tiles = smem + warp * SPW * 2 * kPageBytes;
   float* scl = reinterpret_cast<float*>(smem + Plan::kTileBytes) +
                warp * SPW * 2 * kBS;
+  uint8_t* scratch =
+      smem + Plan::kTileBytes + Plan::kScaleBytes + warp * Math::kScratchBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kTileBytes +
-                                               Plan::kScaleBytes) +
+                                               Plan::kScaleBytes +
+                                               Plan::kScratchBytes) +
                    warp * SPW;
   if (lane == 0) {
     prefetch_tensormap(&tmk);
@@ -703,12 +1069,17 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   }
   __syncwarp();
 
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * WPC;
-  const int64_t n_items =
-      static_cast<int64_t>(p.max_chunks) * p.num_kv_heads * p.batch;
+  Stride st;
+  {
+    Item w;
+    item_set(p, static_cast<int64_t>(gridDim.x) * WPC, w);
+    st.dc = w.chunk;
+    st.dk = w.kvh;
+    st.db = w.b;
+  }
   Item cmp;
-  cmp.idx = static_cast<int64_t>(blockIdx.x) * WPC + warp;
-  if (cmp.idx < n_items && !item_load(p, cmp)) item_next(p, cmp, stride, n_items);
+  item_set(p, static_cast<int64_t>(blockIdx.x) * WPC + warp, cmp);
+  if (!item_done(p, cmp) && !item_fill(p, cmp)) item_next(p, cmp, st);
 
   // ---- issue cursor: SPW pages ahead of the compute cursor
   Item iss = cmp;
@@ -717,11 +1088,11 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   uint32_t k_iss = 0;
   int slot_iss = 0;
   auto issue_one = [&]() {
-    while (iss.idx < n_items && iss_page >= iss.npages) {
-      item_next(p, iss, stride, n_items);
+    while (!item_done(p, iss) && iss_page >= iss.npages) {
+      item_next(p, iss, st);
       iss_page = 0;
     }
-    if (iss.idx >= n_items) return;
+    if (item_done(p, iss)) return;
     if ((iss_page & 31) == 0) {
       const int j = iss_page + lane;
       bt_reg = j < iss.npages
@@ -730,10 +1101,15 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                    : 0;
     }
     const int blk = __shfl_sync(kFull, bt_reg, iss_page & 31);
-    if (lane == 0) {
+    bool issue_copies = true;
+#ifdef KV8_TEST_HOOKS
+    issue_copies = !(g_test_skip_first_copy && blockIdx.x == 0 && warp == 0 &&
+                     k_iss == 0);
+#endif
+    if (lane == 0) mbar_arrive_expect_tx(&bars[slot_iss], kPageTx);
+    if (lane == 0 && issue_copies) {
       const int s = slot_iss;
       const int page = blk * p.num_kv_heads + iss.kvh;
-      mbar_arrive_expect_tx(&bars[s], kPageTx);
       uint8_t* tk = tiles + s * 2 * kPageBytes;
       tma_load_3d(tk, &tmk, 0, 0, page, &bars[s]);
       tma_load_3d(tk + kPageBytes, &tmv, 0, 0, page, &bars[s]);
@@ -751,11 +1127,12 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   for (int s = 0; s < SPW; ++s) issue_one();
 
   Math math;
+  math.attach(scratch);
   uint32_t k_cmp = 0;
   int slot = 0;
   uint32_t phase = 0;
   bool ok = true;
-  while (cmp.idx < n_items) {
+  while (!item_done(p, cmp)) {
     const int64_t row0 = static_cast<int64_t>(cmp.b) * p.num_q_heads + cmp.kvh * G;
     math.init(p.q + row0 * kD, p.q_scale, lane);
     for (int j = 0; j < cmp.npages; ++j) {
@@ -765,8 +1142,11 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       }
       const uint8_t* tk = tiles + slot * 2 * kPageBytes;
       const float* ks = scl + slot * 2 * kBS;
-      math.page(tk, tk + kPageBytes, ks, ks + kBS,
-                min(kBS, cmp.tok1 - (cmp.tok0 + j * kBS)));
+      const int nv = cmp.tok1 - (cmp.tok0 + j * kBS);
+      if (nv >= kBS)
+        math.template page<true>(tk, tk + kPageBytes, ks, ks + kBS, kBS);
+      else
+        math.template page<false>(tk, tk + kPageBytes, ks, ks + kBS, nv);
       __syncwarp();
       issue_one();
       ++k_cmp;
@@ -784,7 +1164,8 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     sk.row0 = row0;
     sk.ci0 = row0 * p.max_chunks + cmp.chunk;
     sk.max_chunks = p.max_chunks;
-    sk.single = cmp.nchunks <= 1;
+    const int nchunks = (cmp.n + p.chunk_tokens - 1) / p.chunk_tokens;
+    sk.single = nchunks <= 1;
     sk.out_f32 = p.out_f32;
     math.finish(sk);
 
@@ -795,15 +1176,15 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       unsigned int ticket = 0;
       if (lane == 0) ticket = atomicAdd(&p.ws_ctr[row0], 1u);
       ticket = __shfl_sync(kFull, ticket, 0);
-      if (ticket == static_cast<unsigned int>(cmp.nchunks - 1)) {
+      if (ticket == static_cast<unsigned int>(nchunks - 1)) {
         __threadfence();
         for (int h = 0; h < G; ++h)
           merge_head_warp(p.ws_ml + (row0 + h) * p.max_chunks * 2,
-                          p.ws_o + (row0 + h) * p.max_chunks * kD, cmp.nchunks,
+                          p.ws_o + (row0 + h) * p.max_chunks * kD, nchunks,
                           p.out, row0 + h, p.out_f32);
       }
     }
-    item_next(p, cmp, stride, n_items);
+    item_next(p, cmp, st);
   }
   if (!ok) {
     // A copy never landed: drain the other copies in flight (bounded) and
@@ -837,10 +1218,13 @@ template <int G, int WPC, int SPW, class Math>
 int launch_decode_kernel(const DecodeParams& p, const CUtensorMap& tmk,
                          const CUtensorMap& tmv, cudaStream_t stream) {
   auto kern = decode_kernel<G, WPC, SPW, Math>;
-  constexpr int smem = SmemPlan<WPC, SPW>::kBytes;
-  static int resident = 0;  // CTAs per SM for this instantiation
-  static int sms = 0;
-  if (resident == 0) {
+  constexpr int smem = SmemPlan<WPC, SPW, Math::kScratchBytes>::kBytes;
+  static LaunchFacts table[kMaxDevices];  // per device, this instantiation
+  LaunchFacts* f = facts_for_current_device(table);
+  if (!f) return -1;
+  int resident = f->resident.load(std::memory_order_acquire);
+  int sms = f->sms.load(std::memory_order_acquire);
+  if (resident == 0 || sms == 0) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -859,6 +1243,8 @@ int launch_decode_kernel(const DecodeParams& p, const CUtensorMap& tmk,
       return -1;
     sms = nsm;
     resident = occ > 0 ? occ : 1;
+    f->sms.store(sms, std::memory_order_release);
+    f->resident.store(resident, std::memory_order_release);
   }
   const int64_t n_items =
       static_cast<int64_t>(p.max_chunks) * p.num_kv_heads * p.batch;
@@ -873,12 +1259,25 @@ int launch_decode_kernel(const DecodeParams& p, const CUtensorMap& tmk,
 template <int G>
 int launch_group(const DecodeParams& p, const CUtensorMap& tmk,
                  const CUtensorMap& tmv, int32_t variant, cudaStream_t stream) {
-  if (variant == 1)
+  if (variant == KV8_FORM_CUDA_CORE)
     return launch_decode_kernel<G, 4, 4, SimtMath<G>>(p, tmk, tmv, stream);
+  if constexpr (G <= 4) {
+    if (variant == KV8_FORM_MMA_I8)
+      return launch_decode_kernel<G, 4, 3, I8Math<G>>(p, tmk, tmv, stream);
+  }
   return launch_decode_kernel<G, 4, 3, MmaMath<G>>(p, tmk, tmv, stream);
 }
 
 }  // namespace
+
+#ifdef KV8_TEST_HOOKS
+int test_skip_first_copy(int on) {
+  return cudaMemcpyToSymbol(g_test_skip_first_copy, &on, sizeof(int)) ==
+                 cudaSuccess
+             ? 0
+             : -1;
+}
+#endif
 
 int read_device_status(uint32_t* value, int clear) {
   if (cudaDeviceSynchronize() != cudaSuccess) return -1;

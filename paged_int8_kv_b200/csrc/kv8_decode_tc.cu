@@ -879,8 +879,12 @@ int launch_tc(const DecodeParams& p, const CUtensorMap& tmk,
               const CUtensorMap& tmv, cudaStream_t stream) {
   auto kern = decode_tc_kernel<G, NB>;
   constexpr int smem = TcPlan<NB, 4 * (G < 4 ? 4 : G)>::kBytes;
-  static int resident = 0, sms = 0;
-  if (resident == 0) {
+  static LaunchFacts table[kMaxDevices];  // per device, this instantiation
+  LaunchFacts* f = facts_for_current_device(table);
+  if (!f) return -1;
+  int resident = f->resident.load(std::memory_order_acquire);
+  int sms = f->sms.load(std::memory_order_acquire);
+  if (resident == 0 || sms == 0) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -913,6 +917,8 @@ int launch_tc(const DecodeParams& p, const CUtensorMap& tmk,
     r = min(r, regs_sm / (warp_regs * (kThreads / 32)));
     r = min(r, 512 / kTmemCols);  // tensor-memory columns of the SM
     resident = r < 1 ? 1 : r;
+    f->sms.store(sms, std::memory_order_release);
+    f->resident.store(resident, std::memory_order_release);
   }
   const int64_t n_items =
       static_cast<int64_t>(p.max_chunks) * p.num_kv_heads * p.batch;

@@ -8,7 +8,28 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace kv8 {
+
+// Launch facts of one kernel on one device (resident CTAs per SM and the SM
+// count), found by its first launch on that device, with that device
+// current, after the kernel's attributes were set there.  Zero = not yet
+// known.  Racing first launches compute the same values.
+constexpr int kMaxDevices = 64;
+struct LaunchFacts {
+  std::atomic<int> resident{0};
+  std::atomic<int> sms{0};
+};
+
+// The facts slot of the current device (nullptr on a CUDA error or a
+// device ordinal beyond kMaxDevices).
+inline LaunchFacts* facts_for_current_device(LaunchFacts (&table)[kMaxDevices]) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return nullptr;
+  return &table[dev];
+}
 
 constexpr int kHeadDim = 128;
 constexpr int kBlockSize = 16;
@@ -75,5 +96,10 @@ int read_tc_status(uint32_t* value, int clear);
 // decode kernel after a device-wide synchronize, OR-ed together.  Returns 0,
 // or -1 on a CUDA error.
 int read_device_status(uint32_t* value, int clear);
+
+#ifdef KV8_TEST_HOOKS
+// Test-hook build only (see kv8_test_hooks.h).
+int test_skip_first_copy(int on);
+#endif
 
 }  // namespace kv8

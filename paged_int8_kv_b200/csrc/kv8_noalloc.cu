@@ -19,10 +19,16 @@
 // kernels as a plain pointer.
 //
 // Sharing rules: every call uses the same array, which keeps whatever the
-// last call left in it.  The split kernel writes every partial that the
-// reduce then reads, so nothing has to start at zero and nothing is
-// cleared.  Two calls whose kernels overlap on the GPU (for instance on two
-// streams without ordering between them) race on the array.
+// last call left in it.  The chunk partials need no initial value (the split
+// kernel writes every partial before the merge reads it); the merge tickets
+// at the end of the array must start at zero, and the call clears them on
+// its stream before its kernel, as the allocating entry point does with a
+// caller's workspace.  Two calls whose kernels overlap on the GPU (for
+// instance on two streams without ordering between them) race on both the
+// partials and the tickets.
+//
+// The cached device address stays valid for the life of the CUDA context;
+// a device reset after the first call on a device is not supported.
 #include <mutex>
 
 #include "../../include/kv8.h"
@@ -75,9 +81,12 @@ extern "C" int32_t kv8_paged_decode_attention_noalloc(
     ws = scratch_on_current_device();
     if (!ws) return KV8_ERR_CUDA;
   }
+  // the array's real size: the allocating entry point checks it against its
+  // own requirement too, so an oversized split is refused twice over
   return kv8_paged_decode_attention(
       q, k_cache, v_cache, k_scales, v_scales, block_tables, context_lens,
       batch, num_q_heads, num_kv_heads, head_dim, block_size,
       max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
-      chunk_tokens, ws, need, out, out_dtype, stream);
+      chunk_tokens, ws, ws ? static_cast<size_t>(KV8_NOALLOC_WORKSPACE_BYTES) : 0,
+      out, out_dtype, stream);
 }

@@ -62,15 +62,18 @@ class PagedKV8Cache:
                context_lens: torch.Tensor, max_context_len: int,
                chunk_tokens: int = 512, out: torch.Tensor | None = None,
                out_dtype: torch.dtype = torch.bfloat16,
-               softmax_scale: float = 0.0, stream=None) -> torch.Tensor:
+               softmax_scale: float = 0.0, form: int = B.KV8_FORM_AUTO,
+               stream=None) -> torch.Tensor:
+        """One decode step over this cache; ``form`` picks the decode form
+        for this call (KV8_FORM_AUTO: the library's default)."""
         if out is None:
             out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
         ws = self.workspace(q.shape[0], q.shape[1], max_context_len, chunk_tokens)
-        return B.kv8_paged_decode_attention(
+        return B.kv8_paged_decode_attention_form(
             q, self.k_cache, self.v_cache, self.k_scales, self.v_scales,
             block_tables, context_lens, out, max_context_len,
             chunk_tokens=chunk_tokens, workspace=ws,
-            softmax_scale=softmax_scale, stream=stream)
+            softmax_scale=softmax_scale, form=form, stream=stream)
 
 
 def fill_from_host(cache: PagedKV8Cache, segments, stream=None) -> int:

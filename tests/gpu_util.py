@@ -24,10 +24,10 @@ def device_inputs(w: W.Workload, device="cuda"):
 
 
 def gpu_decode(cache, q, bt, cl, w: W.Workload, chunk_tokens=None,
-               out_dtype=torch.float32):
+               out_dtype=torch.float32, form=0):
     ct = w.chunk_tokens if chunk_tokens is None else chunk_tokens
     out = cache.decode(q, bt, cl, w.max_context_len, chunk_tokens=ct,
-                       out_dtype=out_dtype)
+                       out_dtype=out_dtype, form=form)
     torch.cuda.synchronize()
     return out.float().cpu().numpy()
 

@@ -97,4 +97,32 @@ def test_host_validation_rejects_before_launch(lib):
     assert f(16, 16, 16, -1, 2, 128, 16, 8, 16, 16, 16, 16, 0) == 1
     assert f(16, 16, 16, 0, 2, 128, 16, 8, 16, 16, 16, 16, 0) == 0
     assert f(0, 16, 16, 4, 2, 128, 16, 8, 16, 16, 16, 16, 0) == 1
-    assert lib.kv8_set_decode_kernel(5) == 1
+    # the decode form is an argument of each call; unknown forms are refused
+    # before anything else is looked at
+    g = lib.kv8_paged_decode_attention_form
+    g.restype = i32
+    g.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32,
+                  ctypes.c_float, i32, P, ctypes.c_size_t, P, i32, i32, P]
+    for form in (-1, 99):
+        assert g(16, 16, 16, 16, 16, 16, 16, 1, 8, 2, 128, 16, 4, 8, 64, 0.0, 0,
+                 0, 0, 16, 0, form, 0) == 1
+    assert g(16, 16, 16, 16, 16, 16, 16, 1, 8, 2, 64, 16, 4, 8, 64, 0.0, 0,
+             0, 0, 16, 0, 2, 0) == 2                # head_dim unsupported
+
+
+def test_chunk_suggestion(lib):
+    # no GPU here: the suggestion assumes 148 SMs x 12 resident warps and
+    # cuts the longest context into equal block-aligned chunks of 64..512
+    # tokens so that sequences x KV heads x chunks >= 3 x 1776 warps
+    f = lib.kv8_decode_chunk_tokens
+    f.restype = ctypes.c_int32
+    f.argtypes = [ctypes.c_int32] * 3
+    assert f(64, 8, 32768) == 512          # 64 chunks: already 9x the warps
+    assert f(32, 8, 4017) == 192           # 21 chunks of <= 192 tokens
+    assert f(256, 8, 544) == 192           # 3 chunks: 192, 192, 160
+    assert f(2, 2, 256) == 64              # floor of 4 pages per chunk
+    assert f(1, 1, 64) == 0 and f(1, 1, 65) == 64
+    assert f(0, 8, 100) == 0 and f(4, 0, 100) == 0 and f(4, 8, 0) == 0
+    for b, h, t in ((1, 1, 10**6), (7, 3, 12345), (512, 8, 128)):
+        c = f(b, h, t)
+        assert c % 16 == 0 and 64 <= c <= 512

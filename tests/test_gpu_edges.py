@@ -31,7 +31,6 @@ def pk():
     from paged_int8_kv_b200 import build
     build.build()
     import paged_int8_kv_b200 as m
-    m.kv8_set_decode_kernel(0)
     yield m
     assert m.kv8_read_device_status(clear=True) == 0
 
@@ -42,7 +41,8 @@ def _ref(oracle_mod, w):
                                        w.context_lens)
 
 
-@pytest.mark.parametrize("kind", [1, 2, 3], ids=["cudacore", "mmasync", "tcgen05"])
+@pytest.mark.parametrize("kind", [1, 2, 3, 4],
+                         ids=["cudacore", "mmasync", "tcgen05", "mma_i8"])
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (8, 2), (16, 2), (4, 1)])
 @pytest.mark.parametrize("chunk", [0, 16, 512])
 def test_ragged_groups_chunks(pk, oracle_mod, hq, hkv, chunk, kind):
@@ -50,17 +50,13 @@ def test_ragged_groups_chunks(pk, oracle_mod, hq, hkv, chunk, kind):
                         extra_blocks=7, outliers=(3, 10.0), chunk_tokens=chunk)
     ref = _ref(oracle_mod, w)
     cache, q, bt, cl = U.device_inputs(w)
-    pk.kv8_set_decode_kernel(kind)
-    try:
-        for dt, bf in ((torch.float32, False), (torch.bfloat16, True)):
-            gpu = U.gpu_decode(cache, q, bt, cl, w, chunk_tokens=chunk,
-                               out_dtype=dt)
-            U.assert_close(gpu, ref, bf16=bf)
-            if not bf:
-                assert np.abs(gpu - ref).max() < 1e-4
-            assert np.all(gpu[0] == 0.0)  # empty context -> zeros
-    finally:
-        pk.kv8_set_decode_kernel(0)
+    for dt, bf in ((torch.float32, False), (torch.bfloat16, True)):
+        gpu = U.gpu_decode(cache, q, bt, cl, w, chunk_tokens=chunk,
+                           out_dtype=dt, form=kind)
+        U.assert_close(gpu, ref, bf16=bf)
+        if not bf:
+            assert np.abs(gpu - ref).max() < 1e-4
+        assert np.all(gpu[0] == 0.0)  # empty context -> zeros
 
 
 @pytest.mark.parametrize("scale", [2.0 ** -40, 1.0, 2.0 ** 20])
@@ -79,12 +75,10 @@ def test_tensorcore_extreme_magnitudes(pk, oracle_mod, scale):
     w.private_kv = scaled
     ref = _ref(oracle_mod, w)
     cache, qd, bt, cl = U.device_inputs(w)
-    for kind in (1, 2, 3):
-        pk.kv8_set_decode_kernel(kind)
-        gpu = U.gpu_decode(cache, qd, bt, cl, w, chunk_tokens=256)
+    for kind in (1, 2, 3, 4):
+        gpu = U.gpu_decode(cache, qd, bt, cl, w, chunk_tokens=256, form=kind)
         denom = max(np.abs(ref).max(), 1e-30)
         assert np.abs(gpu - ref).max() / denom < 1e-4, kind
-    pk.kv8_set_decode_kernel(0)
 
 
 def test_tensorcore_matches_cudacore(pk):
@@ -92,12 +86,11 @@ def test_tensorcore_matches_cudacore(pk):
                         outliers=(4, 8.0))
     cache, q, bt, cl = U.device_inputs(w)
     outs = []
-    for kind in (1, 2, 3):
-        pk.kv8_set_decode_kernel(kind)
-        outs.append(U.gpu_decode(cache, q, bt, cl, w, chunk_tokens=512))
-    pk.kv8_set_decode_kernel(0)
-    assert np.abs(outs[0] - outs[1]).max() < 1e-4
-    assert np.abs(outs[0] - outs[2]).max() < 1e-4
+    for kind in (1, 2, 3, 4):
+        outs.append(U.gpu_decode(cache, q, bt, cl, w, chunk_tokens=512,
+                                 form=kind))
+    for o in outs[1:]:
+        assert np.abs(outs[0] - o).max() < 1e-4
 
 
 def test_block_permutation_bit_identical(pk):

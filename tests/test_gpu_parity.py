@@ -35,7 +35,6 @@ def built():
     from paged_int8_kv_b200 import build
     build.build()
     import paged_int8_kv_b200 as pk
-    pk.kv8_set_decode_kernel(0)
     yield pk
     assert pk.kv8_read_device_status(clear=True) == 0
 
@@ -62,25 +61,19 @@ def test_quantize_bit_exact(built, oracle_mod, name):
     assert np.array_equal(_u32(cache.v_scales.cpu().numpy()), _u32(vs))
 
 
-KINDS = pytest.mark.parametrize("kind", [0, 3], ids=["default", "tcgen05"])
-
-
-@pytest.fixture
-def kind_set(built, kind):
-    built.kv8_set_decode_kernel(kind)
-    yield kind
-    built.kv8_set_decode_kernel(0)
+KINDS = pytest.mark.parametrize("kind", [0, 2, 3, 4],
+                                ids=["default", "mma_f16pv", "tcgen05", "mma_i8"])
 
 
 @KINDS
 @pytest.mark.parametrize("name", SMALL)
 @pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
-def test_decode_all_pairs(built, oracle_mod, name, out_dtype, kind_set):
+def test_decode_all_pairs(built, oracle_mod, name, out_dtype, kind):
     w, (cache, q, bt, cl), (kc, vc, ks, vs) = _setup(name, oracle_mod)
     ref = oracle_mod.decode_attention(w.q(), kc, vc, ks, vs, w.block_tables,
                                       w.context_lens)
     dt = torch.float32 if out_dtype == "f32" else torch.bfloat16
-    gpu = U.gpu_decode(cache, q, bt, cl, w, out_dtype=dt)
+    gpu = U.gpu_decode(cache, q, bt, cl, w, out_dtype=dt, form=kind)
     U.assert_close(gpu, ref, bf16=(out_dtype == "bf16"))
     if out_dtype == "f32":
         # the fp32 path is far inside the tolerance: a regression shows here
@@ -114,10 +107,10 @@ def test_big_quantize_sampled_sequences(big, oracle_mod):
 
 @KINDS
 @pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
-def test_big_decode_sampled(big, oracle_mod, out_dtype, kind_set):
+def test_big_decode_sampled(big, oracle_mod, out_dtype, kind):
     w, (cache, q, bt, cl) = big
     dt = torch.float32 if out_dtype == "f32" else torch.bfloat16
-    gpu = U.gpu_decode(cache, q, bt, cl, w, out_dtype=dt)
+    gpu = U.gpu_decode(cache, q, bt, cl, w, out_dtype=dt, form=kind)
     rng = np.random.default_rng(77)
     for b in BIG_SEQS:
         kc, vc, ks, vs, table = U.oracle_sequence_cache(oracle_mod, w, b)

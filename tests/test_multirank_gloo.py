@@ -71,3 +71,37 @@ def test_reference_arm_other_ranks_do_nothing():
         steps, warmup, ref_seqs, gpus = 1, 0, 1, 2
     # rank 1 returns immediately (no oracle work, no output)
     assert bench.run_reference(A(), W.tiny(), 1) == 0
+
+
+def test_bench_gpus_flag_spawns_ranks():
+    # `bench.py --gpus 2` started without a launcher starts its own two ranks
+    # (one process each); the dry run exercises that launch path on CPU ranks
+    # over gloo and must report both ranks, never one GPU under a 2-GPU label
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR",
+                        "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"),
+                        "--gpus", "2", "--dry-run-cpu", "--steps", "3",
+                        "--warmup", "3"], capture_output=True, text=True,
+                       timeout=300, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["dry_run"] is True and rec["value"] is None
+    assert rec["n_gpus"] == 2 and rec["ranks_seen"] == 2
+
+
+def test_bench_rejects_mismatched_world_size():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"),
+                        "--gpus", "4", "--dry-run-cpu"], capture_output=True,
+                       text=True, timeout=120, env=env, cwd=root)
+    assert r.returncode == 2 and "WORLD_SIZE=1" in r.stderr
