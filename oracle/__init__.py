@@ -55,6 +55,9 @@ def _load():
     lib.oracle_decode_attention.restype = ctypes.c_int
     lib.oracle_decode_attention.argtypes = [
         P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, f64, P, i64, P]
+    lib.oracle_extend_attention.restype = ctypes.c_int
+    lib.oracle_extend_attention.argtypes = [
+        P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, f64, P]
     lib.oracle_kv_cache_bytes.restype = f64
     lib.oracle_kv_cache_bytes.argtypes = [i64] * 7
     lib.oracle_kv8_scale_bytes.restype = f64
@@ -127,6 +130,39 @@ def decode_attention(q_bf16: np.ndarray, k_cache: np.ndarray,
         _ptr(bt), _ptr(cl), B, hq, hkv, d, bs, bt.shape[1], nb,
         float(softmax_scale), pp, npairs, _ptr(out))
     _check(rc, "oracle_decode_attention")
+    return out
+
+
+def extend_attention(q_bf16: np.ndarray, k_cache: np.ndarray,
+                     v_cache: np.ndarray, k_scales: np.ndarray,
+                     v_scales: np.ndarray, block_tables: np.ndarray,
+                     context_lens: np.ndarray, q_start: np.ndarray,
+                     softmax_scale: float = 0.0) -> np.ndarray:
+    """fp64 causal extend (prefill) attention over the dequantised cache.
+
+    q_bf16: uint16 [q_start[-1], H_q, D], the new query rows of every
+    sequence packed in order; sequence b's rows are its last
+    q_start[b+1]-q_start[b] cached positions.  Returns float64 of q's shape.
+    """
+    lib = _load()
+    q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    qs = np.ascontiguousarray(q_start, dtype=np.int32)
+    for a in (k_cache, v_cache):
+        assert a.dtype == np.int8 and a.flags.c_contiguous
+    for a in (k_scales, v_scales):
+        assert a.dtype == np.float32 and a.flags.c_contiguous
+    nq, hq, d = q.shape
+    nb, hkv, bs, d2 = k_cache.shape
+    B = cl.shape[0]
+    assert d2 == d and qs.shape == (B + 1,) and int(qs[-1]) == nq
+    out = np.zeros((nq, hq, d), dtype=np.float64)
+    rc = lib.oracle_extend_attention(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales),
+        _ptr(bt), _ptr(cl), _ptr(qs), B, hq, hkv, d, bs, bt.shape[1], nb,
+        float(softmax_scale), _ptr(out))
+    _check(rc, "oracle_extend_attention")
     return out
 
 

@@ -117,21 +117,18 @@ int oracle_quantize_append(const uint16_t *x, const int64_t *slot_mapping,
 }
 
 /*
- * Exact decode attention for one (sequence b, query head h), fp64.
- * out_row receives head_dim doubles.
+ * Exact attention of one query row over the first n tokens of sequence b's
+ * paged cache (KV head kvh), fp64.  out_row receives head_dim doubles; n == 0
+ * gives a zero row.
  */
-static int attend_one(const uint16_t *q, const int8_t *k_cache,
+static int attend_row(const uint16_t *qrow, const int8_t *k_cache,
                       const int8_t *v_cache, const float *k_scales,
                       const float *v_scales, const int32_t *block_tables,
-                      const int32_t *context_lens, int32_t num_q_heads,
                       int32_t num_kv_heads, int32_t head_dim,
                       int32_t block_size, int32_t max_blocks_per_seq,
                       int64_t num_blocks, double softmax_scale, int32_t b,
-                      int32_t h, double *out_row)
+                      int32_t kvh, int32_t n, double *out_row)
 {
-    int32_t group = num_q_heads / num_kv_heads;
-    int32_t kvh = h / group;
-    int32_t n = context_lens[b];
     for (int32_t j = 0; j < head_dim; ++j)
         out_row[j] = 0.0;
     if (n == 0)
@@ -139,7 +136,6 @@ static int attend_one(const uint16_t *q, const int8_t *k_cache,
     if (n < 0 || n > max_blocks_per_seq * block_size)
         return ORACLE_BAD_ARG;
 
-    const uint16_t *qrow = q + ((int64_t)b * num_q_heads + h) * head_dim;
     double *score = (double *)malloc(sizeof(double) * (size_t)n);
     if (!score)
         return ORACLE_NOMEM;
@@ -187,6 +183,27 @@ static int attend_one(const uint16_t *q, const int8_t *k_cache,
 }
 
 /*
+ * Exact decode attention for one (sequence b, query head h), fp64: the
+ * sequence's one query row over all context_lens[b] cached tokens.
+ */
+static int attend_one(const uint16_t *q, const int8_t *k_cache,
+                      const int8_t *v_cache, const float *k_scales,
+                      const float *v_scales, const int32_t *block_tables,
+                      const int32_t *context_lens, int32_t num_q_heads,
+                      int32_t num_kv_heads, int32_t head_dim,
+                      int32_t block_size, int32_t max_blocks_per_seq,
+                      int64_t num_blocks, double softmax_scale, int32_t b,
+                      int32_t h, double *out_row)
+{
+    int32_t group = num_q_heads / num_kv_heads;
+    const uint16_t *qrow = q + ((int64_t)b * num_q_heads + h) * head_dim;
+    return attend_row(qrow, k_cache, v_cache, k_scales, v_scales, block_tables,
+                      num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                      num_blocks, softmax_scale, b, h / group, context_lens[b],
+                      out_row);
+}
+
+/*
  * Decode attention for a list of (b, h) pairs (pairs = 2*n_pairs int32, NULL
  * meaning every pair in row-major order).  out holds n_pairs * head_dim
  * doubles (B * H_q * head_dim when pairs == NULL).
@@ -226,6 +243,60 @@ int oracle_decode_attention(const uint16_t *q, const int8_t *k_cache,
                             out + p * head_dim);
         if (rc != ORACLE_OK)
             return rc;
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Extend (prefill) attention over the paged cache, fp64
+ * [KV Cache 优化全景解析, §2.2 Prefill 与 Decode 两阶段: the prompt's tokens
+ * are processed together and fill the cache; §11.2 chunked prefill: a long
+ * prompt enters in chunks, each attending to everything cached before it].
+ * Sequence b has n_new_b = q_start[b+1] - q_start[b] new query tokens, the
+ * last n_new_b of its context_lens[b] cached tokens (appended before the
+ * call, as in decode).  Query row i of sequence b sits at position
+ * p = context_lens[b] - n_new_b + i and attends causally to cached tokens
+ * 0..p, i.e. to the first p + 1 tokens [same page, §2.1: softmax(QK^T /
+ * sqrt(d)) V; causal because generation sees only earlier tokens].
+ *   q   (bf16 bits) [q_start[batch]][H_q][D], rows packed by sequence
+ *   out (fp64)      [q_start[batch]][H_q][D]
+ * Returns ORACLE_BAD_ARG when n_new_b > context_lens[b] or q_start is not
+ * non-decreasing from 0.
+ */
+int oracle_extend_attention(const uint16_t *q, const int8_t *k_cache,
+                            const int8_t *v_cache, const float *k_scales,
+                            const float *v_scales, const int32_t *block_tables,
+                            const int32_t *context_lens, const int32_t *q_start,
+                            int32_t batch, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim,
+                            int32_t block_size, int32_t max_blocks_per_seq,
+                            int64_t num_blocks, double softmax_scale,
+                            double *out)
+{
+    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_q_heads % num_kv_heads != 0 || q_start[0] != 0)
+        return ORACLE_BAD_ARG;
+    if (softmax_scale <= 0.0)
+        softmax_scale = 1.0 / sqrt((double)head_dim);
+    int32_t group = num_q_heads / num_kv_heads;
+    for (int32_t b = 0; b < batch; ++b) {
+        int32_t n_new = q_start[b + 1] - q_start[b];
+        if (n_new < 0 || n_new > context_lens[b])
+            return ORACLE_BAD_ARG;
+        for (int32_t i = 0; i < n_new; ++i) {
+            int64_t row = (int64_t)q_start[b] + i;
+            int32_t keys = context_lens[b] - n_new + i + 1;
+            for (int32_t h = 0; h < num_q_heads; ++h) {
+                const uint16_t *qrow = q + (row * num_q_heads + h) * head_dim;
+                double *orow = out + (row * num_q_heads + h) * head_dim;
+                int rc = attend_row(qrow, k_cache, v_cache, k_scales, v_scales,
+                                    block_tables, num_kv_heads, head_dim,
+                                    block_size, max_blocks_per_seq, num_blocks,
+                                    softmax_scale, b, h / group, keys, orow);
+                if (rc != ORACLE_OK)
+                    return rc;
+            }
+        }
     }
     return ORACLE_OK;
 }
