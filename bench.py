@@ -315,6 +315,17 @@ class DeviceWorkload:
         self.out = torch.empty(self.q.shape, dtype=torch.bfloat16, device=dev)
         self.ws = self.cache.workspace(w.batch, w.num_q_heads,
                                        w.max_context_len, chunk)
+        # groups sharing a prefix: decoded through the shared-prefix entry
+        # point (the shared pages scored once per group)
+        self.prefix = None
+        if w.prefix_group is not None and w.prefix_len > 0:
+            ng = int(w.prefix_group.max()) + 1
+            self.prefix = (
+                torch.from_numpy(w.prefix_group.astype(np.int32)).to(dev),
+                torch.full((ng,), w.prefix_len, dtype=torch.int32, device=dev),
+                int(np.bincount(w.prefix_group[w.prefix_group >= 0]).max()),
+                w.prefix_len)
+        self.use_prefix = self.prefix is not None
 
     def append(self, k=None, v=None, s=None):
         self.cache.append(self.k_new if k is None else k,
@@ -324,6 +335,15 @@ class DeviceWorkload:
     def decode(self, form, q=None, bt=None, cl=None):
         import paged_int8_kv_b200 as pk
         c = self.cache
+        if self.use_prefix and form == 0:
+            pg, pl, gmax, plen = self.prefix
+            pk.kv8_paged_decode_attention_prefix(
+                self.q if q is None else q, c.k_cache, c.v_cache, c.k_scales,
+                c.v_scales, self.bt if bt is None else bt,
+                self.cl if cl is None else cl, self.out,
+                self.w.max_context_len, pg, pl, gmax, plen,
+                chunk_tokens=self.chunk, workspace=self.ws)
+            return
         pk.kv8_paged_decode_attention_form(
             self.q if q is None else q, c.k_cache, c.v_cache, c.k_scales,
             c.v_scales, self.bt if bt is None else bt,
@@ -404,6 +424,12 @@ def run_per_workload(args, dev, peak: float) -> dict:
         rec.update({"workload": w.name, "chunk_tokens": dw.chunk,
                     "calls": len(ms), "l2": "flushed before each call",
                     "stat": "median"})
+        if dw.use_prefix:
+            # the same batch through the plain entry point, for comparison
+            rec["entry_point"] = "kv8_paged_decode_attention_prefix"
+            dw.use_prefix = False
+            plain = time_decode_calls(dw, args.kernel, args.calls, 10, flush)
+            rec["plain_decode_us"] = statistics.median(plain) * 1e3
         res[name] = rec
         del dw
         torch.cuda.empty_cache()

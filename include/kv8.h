@@ -173,6 +173,48 @@ KV8_API int32_t kv8_paged_decode_attention(
     size_t workspace_bytes, void *out, int32_t out_dtype, void *stream);
 
 /*
+ * kv8_paged_decode_attention_prefix -- kv8_paged_decode_attention for a
+ * batch in which groups of sequences share the first tokens of their
+ * context, stored once: the same physical blocks open every member's block
+ * table [KV Cache 优化全景解析, §4.2 PagedAttention: several sequences map
+ * one physical block].  The shared pages are read, converted and scored once
+ * for the whole group instead of once per member, the way serving systems
+ * group the requests that share a prefix [garden.houmin.site
+ * infra/kv-cache-optimize, §4.3.1 Prefix-aware Scheduling (BatchLLM)].
+ * The results are those of kv8_paged_decode_attention on the same inputs
+ * (up to rounding order, within the same accuracy).
+ *
+ * Arguments as kv8_paged_decode_attention (form KV8_FORM_AUTO), plus
+ *   prefix_group    int32 [batch] device: the group of sequence b, or -1
+ *   prefix_lens     int32 [num_groups] device: tokens group g's members
+ *                   share at the start of their contexts.  The whole chunks
+ *                   of that prefix (prefix_lens[g] / chunk_tokens of them)
+ *                   are computed once for the group; the rest of each
+ *                   member's context as usual.  Every member's
+ *                   context_lens must be >= prefix_lens[g], and its block
+ *                   table must list the group's blocks for those tokens (a
+ *                   member found shorter sets bit 1 of the device status
+ *                   word and its row is left incomplete).
+ *   num_groups      number of groups (0: a plain decode call)
+ *   max_group_size  host bound on the members of any group (any size;
+ *                   members are served 8 at a time)
+ *   max_prefix_len  host bound on prefix_lens (<= max_context_len)
+ *   chunk_tokens    must be > 0
+ * A sequence belongs to at most one group.  The call enqueues a memset of
+ * the merge tickets, the shared-prefix kernel and the decode kernel.
+ */
+KV8_API int32_t kv8_paged_decode_attention_prefix(
+    const void *q, const int8_t *k_cache, const int8_t *v_cache,
+    const float *k_scales, const float *v_scales, const int32_t *block_tables,
+    const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    const int32_t *prefix_group, const int32_t *prefix_lens,
+    int32_t num_groups, int32_t max_group_size, int32_t max_prefix_len,
+    float softmax_scale, int32_t chunk_tokens, void *workspace,
+    size_t workspace_bytes, void *out, int32_t out_dtype, void *stream);
+
+/*
  * kv8_split_reduce -- merge the per-chunk partials of a split decode launch.
  *
  * For each (b, h) whose context spans C = ceil(n / chunk_tokens) > 1 chunks,
@@ -243,7 +285,9 @@ KV8_API int32_t kv8_paged_decode_attention_form(
  * kv8_read_device_status -- synchronise the current device, then read the
  * library's sticky device status word (0 = clean; bit 0 = a kernel gave up
  * waiting for one of its own shared-memory copies and skipped that work
- * instead of hanging).  clear != 0 resets the word to 0 afterwards.
+ * instead of hanging; bit 1 = a shared-prefix group listed a member whose
+ * context is shorter than the group's prefix).  clear != 0 resets the word
+ * to 0 afterwards.
  */
 KV8_API int32_t kv8_read_device_status(uint32_t *status, int32_t clear);
 

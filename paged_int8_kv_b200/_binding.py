@@ -38,6 +38,7 @@ EXPORTED = (
     "kv8_paged_decode_attention",
     "kv8_split_reduce",
     "kv8_paged_decode_attention_form",
+    "kv8_paged_decode_attention_prefix",
     "kv8_read_device_status",
     "kv8_paged_decode_attention_noalloc",
 )
@@ -69,6 +70,10 @@ def _load() -> ctypes.CDLL:
     lib.kv8_paged_decode_attention.argtypes = [
         P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
         P, sz, P, i32, P]
+    lib.kv8_paged_decode_attention_prefix.restype = i32
+    lib.kv8_paged_decode_attention_prefix.argtypes = [
+        P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, P, P,
+        i32, i32, i32, f32, i32, P, sz, P, i32, P]
     lib.kv8_split_reduce.restype = i32
     lib.kv8_split_reduce.argtypes = [P, sz, P, i32, i32, i32, i32, i32, P, i32, P]
     lib.kv8_paged_decode_attention_form.restype = i32
@@ -183,6 +188,33 @@ def kv8_paged_decode_attention_form(q: torch.Tensor, k_cache: torch.Tensor,
                              block_tables, context_lens, out, max_context_len,
                              chunk_tokens, workspace, softmax_scale),
                int(form), _stream(stream)))
+    return out
+
+
+def kv8_paged_decode_attention_prefix(q: torch.Tensor, k_cache: torch.Tensor,
+                                      v_cache: torch.Tensor,
+                                      k_scales: torch.Tensor,
+                                      v_scales: torch.Tensor,
+                                      block_tables: torch.Tensor,
+                                      context_lens: torch.Tensor,
+                                      out: torch.Tensor, max_context_len: int,
+                                      prefix_group: torch.Tensor,
+                                      prefix_lens: torch.Tensor,
+                                      max_group_size: int, max_prefix_len: int,
+                                      chunk_tokens: int = 512,
+                                      workspace: torch.Tensor | None = None,
+                                      softmax_scale: float = 0.0,
+                                      stream=None) -> torch.Tensor:
+    """Decode with shared prefixes: prefix_group int32 [B] (-1 = none),
+    prefix_lens int32 [num_groups] (both on the GPU)."""
+    a = _decode_args(q, k_cache, v_cache, k_scales, v_scales, block_tables,
+                     context_lens, out, max_context_len, chunk_tokens,
+                     workspace, softmax_scale)
+    _check("kv8_paged_decode_attention_prefix",
+           lib.kv8_paged_decode_attention_prefix(
+               *a[:15], _p(prefix_group), _p(prefix_lens),
+               int(prefix_lens.shape[0]), int(max_group_size),
+               int(max_prefix_len), *a[15:], _stream(stream)))
     return out
 
 

@@ -75,6 +75,112 @@ void split_shape(int32_t max_context_len, int32_t chunk_tokens,
   }
 }
 
+// Everything a decode launch needs, from the arguments of an entry point.
+struct DecodeSetup {
+  kv8::DecodeParams p;
+  CUtensorMap tmk, tmv;
+  bool nothing = false;  // batch == 0: checked, nothing to launch
+};
+
+// The argument checks and parameter set-up shared by the decode entry
+// points.  Returns a KV8 status; launches nothing.
+int32_t prepare_decode(
+    const void* q, const int8_t* k_cache, const int8_t* v_cache,
+    const float* k_scales, const float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void* workspace,
+    size_t workspace_bytes, void* out, int32_t out_dtype, DecodeSetup* d) {
+  // ---- shape checks
+  if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+      max_context_len < 0 || chunk_tokens < 0)
+    return KV8_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return KV8_ERR_INVALID_ARG;
+  if (out_dtype != KV8_OUT_BF16 && out_dtype != KV8_OUT_F32)
+    return KV8_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || block_size != kBlockSize)
+    return KV8_ERR_UNSUPPORTED;
+  if (!group_supported(num_q_heads / num_kv_heads)) return KV8_ERR_UNSUPPORTED;
+  if (chunk_tokens % block_size != 0) return KV8_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_context_len) >
+      static_cast<int64_t>(max_blocks_per_seq) * block_size)
+    return KV8_ERR_INVALID_ARG;
+  if (batch > 65535 || num_kv_heads > 65535) return KV8_ERR_UNSUPPORTED;
+  if (num_blocks > INT32_MAX / num_kv_heads) return KV8_ERR_UNSUPPORTED;
+  if (batch == 0) {
+    d->nothing = true;
+    return KV8_OK;
+  }
+  // ---- pointer checks
+  if (!q || !k_cache || !v_cache || !k_scales || !v_scales || !block_tables ||
+      !context_lens || !out)
+    return KV8_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(k_scales) || !aligned16(v_scales) || !aligned4(block_tables) ||
+      !aligned4(context_lens) || !aligned16(out))
+    return KV8_ERR_INVALID_ARG;
+
+  int32_t chunk_eff, max_chunks;
+  split_shape(max_context_len, chunk_tokens, &chunk_eff, &max_chunks);
+  if (static_cast<int64_t>(max_chunks) * num_kv_heads * batch > INT32_MAX)
+    return KV8_ERR_UNSUPPORTED;
+  float* ws_ml = nullptr;
+  float* ws_o = nullptr;
+  uint32_t* ws_ctr = nullptr;
+  if (max_chunks > 1) {
+    const size_t need = kv8::workspace_total_bytes(batch, num_q_heads, max_chunks);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace))
+      return KV8_ERR_WORKSPACE;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    const size_t ml_bytes = kv8::workspace_ml_bytes(batch, num_q_heads, max_chunks);
+    const size_t o_bytes = kv8::workspace_o_bytes(batch, num_q_heads, max_chunks);
+    ws_ml = reinterpret_cast<float*>(base);
+    ws_o = reinterpret_cast<float*>(base + ml_bytes);
+    ws_ctr = reinterpret_cast<uint32_t*>(base + ml_bytes + o_bytes);
+  }
+
+  const int64_t pages = num_blocks * num_kv_heads;
+  if (!encode_page_map(&d->tmk, k_cache, pages) ||
+      !encode_page_map(&d->tmv, v_cache, pages))
+    return KV8_ERR_CUDA;
+
+  if (!(softmax_scale > 0.0f))
+    softmax_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)));
+  kv8::DecodeParams& p = d->p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.ws_ml = ws_ml;
+  p.ws_o = ws_o;
+  p.ws_ctr = ws_ctr;
+  p.out = out;
+  p.batch = batch;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.chunk_tokens = chunk_eff;
+  p.max_chunks = max_chunks;
+  p.out_f32 = out_dtype == KV8_OUT_F32 ? 1 : 0;
+  p.q_scale = static_cast<float>(static_cast<double>(softmax_scale) *
+                                 1.4426950408889634074);  // log2(e)
+  p.prefix_group = nullptr;
+  p.prefix_lens = nullptr;
+  return KV8_OK;
+}
+
+// Zero the merge tickets of a split launch on `st` (nothing when unsplit).
+bool clear_tickets(const DecodeSetup& d, int32_t batch, int32_t num_q_heads,
+                   cudaStream_t st) {
+  return !d.p.ws_ctr ||
+         cudaMemsetAsync(d.p.ws_ctr, 0,
+                         kv8::workspace_ctr_bytes(batch, num_q_heads),
+                         st) == cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -183,86 +289,60 @@ int32_t kv8_paged_decode_attention_form(
     size_t workspace_bytes, void* out, int32_t out_dtype, int32_t form,
     void* stream) {
   if (form < KV8_FORM_AUTO || form > KV8_FORM_MMA_I8) return KV8_ERR_INVALID_ARG;
-  // ---- shape checks
-  if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
-      block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
-      max_context_len < 0 || chunk_tokens < 0)
-    return KV8_ERR_INVALID_ARG;
-  if (num_q_heads % num_kv_heads != 0) return KV8_ERR_INVALID_ARG;
-  if (out_dtype != KV8_OUT_BF16 && out_dtype != KV8_OUT_F32)
-    return KV8_ERR_INVALID_ARG;
-  if (head_dim != kHeadDim || block_size != kBlockSize)
-    return KV8_ERR_UNSUPPORTED;
-  if (!group_supported(num_q_heads / num_kv_heads)) return KV8_ERR_UNSUPPORTED;
-  if (chunk_tokens % block_size != 0) return KV8_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(max_context_len) >
-      static_cast<int64_t>(max_blocks_per_seq) * block_size)
-    return KV8_ERR_INVALID_ARG;
-  if (batch > 65535 || num_kv_heads > 65535) return KV8_ERR_UNSUPPORTED;
-  if (num_blocks > INT32_MAX / num_kv_heads) return KV8_ERR_UNSUPPORTED;
-  if (batch == 0) return KV8_OK;
-  // ---- pointer checks
-  if (!q || !k_cache || !v_cache || !k_scales || !v_scales || !block_tables ||
-      !context_lens || !out)
-    return KV8_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
-      !aligned16(k_scales) || !aligned16(v_scales) || !aligned4(block_tables) ||
-      !aligned4(context_lens) || !aligned16(out))
-    return KV8_ERR_INVALID_ARG;
-
-  int32_t chunk_eff, max_chunks;
-  split_shape(max_context_len, chunk_tokens, &chunk_eff, &max_chunks);
-  float* ws_ml = nullptr;
-  float* ws_o = nullptr;
-  uint32_t* ws_ctr = nullptr;
-  if (max_chunks > 1) {
-    const size_t need = kv8::workspace_total_bytes(batch, num_q_heads, max_chunks);
-    if (!workspace || workspace_bytes < need || !aligned16(workspace))
-      return KV8_ERR_WORKSPACE;
-    uint8_t* base = static_cast<uint8_t*>(workspace);
-    const size_t ml_bytes = kv8::workspace_ml_bytes(batch, num_q_heads, max_chunks);
-    const size_t o_bytes = kv8::workspace_o_bytes(batch, num_q_heads, max_chunks);
-    ws_ml = reinterpret_cast<float*>(base);
-    ws_o = reinterpret_cast<float*>(base + ml_bytes);
-    ws_ctr = reinterpret_cast<uint32_t*>(base + ml_bytes + o_bytes);
-  }
-
-  CUtensorMap tmk, tmv;
-  const int64_t pages = num_blocks * num_kv_heads;
-  if (!encode_page_map(&tmk, k_cache, pages) ||
-      !encode_page_map(&tmv, v_cache, pages))
-    return KV8_ERR_CUDA;
-
-  if (!(softmax_scale > 0.0f))
-    softmax_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)));
-  kv8::DecodeParams p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k_scales = k_scales;
-  p.v_scales = v_scales;
-  p.block_tables = block_tables;
-  p.context_lens = context_lens;
-  p.ws_ml = ws_ml;
-  p.ws_o = ws_o;
-  p.ws_ctr = ws_ctr;
-  p.out = out;
-  p.batch = batch;
-  p.num_q_heads = num_q_heads;
-  p.num_kv_heads = num_kv_heads;
-  p.max_blocks_per_seq = max_blocks_per_seq;
-  p.chunk_tokens = chunk_eff;
-  p.max_chunks = max_chunks;
-  p.out_f32 = out_dtype == KV8_OUT_F32 ? 1 : 0;
-  p.q_scale = static_cast<float>(static_cast<double>(softmax_scale) *
-                                 1.4426950408889634074);  // log2(e)
-
+  DecodeSetup d;
+  const int32_t rc0 = prepare_decode(
+      q, k_cache, v_cache, k_scales, v_scales, block_tables, context_lens,
+      batch, num_q_heads, num_kv_heads, head_dim, block_size,
+      max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+      chunk_tokens, workspace, workspace_bytes, out, out_dtype, &d);
+  if (rc0 != KV8_OK || d.nothing) return rc0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (ws_ctr &&
-      cudaMemsetAsync(ws_ctr, 0, kv8::workspace_ctr_bytes(batch, num_q_heads),
-                      st) != cudaSuccess)
-    return KV8_ERR_CUDA;
+  if (!clear_tickets(d, batch, num_q_heads, st)) return KV8_ERR_CUDA;
   int rc = form == KV8_FORM_TCGEN05
-               ? kv8::launch_decode_tc(p, tmk, tmv, st)
-               : kv8::launch_decode(p, tmk, tmv, form, st);
+               ? kv8::launch_decode_tc(d.p, d.tmk, d.tmv, st)
+               : kv8::launch_decode(d.p, d.tmk, d.tmv, form, st);
+  if (rc == -2) return KV8_ERR_UNSUPPORTED;
+  if (rc != 0) return KV8_ERR_CUDA;
+  return KV8_OK;
+}
+
+int32_t kv8_paged_decode_attention_prefix(
+    const void* q, const int8_t* k_cache, const int8_t* v_cache,
+    const float* k_scales, const float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    const int32_t* prefix_group, const int32_t* prefix_lens,
+    int32_t num_groups, int32_t max_group_size, int32_t max_prefix_len,
+    float softmax_scale, int32_t chunk_tokens, void* workspace,
+    size_t workspace_bytes, void* out, int32_t out_dtype, void* stream) {
+  if (num_groups < 0 || max_group_size < 0 || max_prefix_len < 0 ||
+      chunk_tokens <= 0 || max_prefix_len > max_context_len)
+    return KV8_ERR_INVALID_ARG;
+  if (num_groups > 0 && (!prefix_group || !prefix_lens ||
+                         !aligned4(prefix_group) || !aligned4(prefix_lens)))
+    return KV8_ERR_INVALID_ARG;
+  DecodeSetup d;
+  const int32_t rc0 = prepare_decode(
+      q, k_cache, v_cache, k_scales, v_scales, block_tables, context_lens,
+      batch, num_q_heads, num_kv_heads, head_dim, block_size,
+      max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+      chunk_tokens, workspace, workspace_bytes, out, out_dtype, &d);
+  if (rc0 != KV8_OK || d.nothing) return rc0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!clear_tickets(d, batch, num_q_heads, st)) return KV8_ERR_CUDA;
+  kv8::PrefixShape ps;
+  ps.num_groups = num_groups;
+  ps.rounds = (max_group_size + 7) / 8;
+  ps.prefix_chunks = max_prefix_len / d.p.chunk_tokens;
+  if (num_groups > 0 && ps.rounds > 0 && ps.prefix_chunks > 0) {
+    d.p.prefix_group = prefix_group;
+    d.p.prefix_lens = prefix_lens;
+    const int rc = kv8::launch_prefix(d.p, ps, d.tmk, d.tmv, st);
+    if (rc == -2) return KV8_ERR_UNSUPPORTED;
+    if (rc != 0) return KV8_ERR_CUDA;
+  }
+  const int rc = kv8::launch_decode(d.p, d.tmk, d.tmv, KV8_FORM_AUTO, st);
   if (rc == -2) return KV8_ERR_UNSUPPORTED;
   if (rc != 0) return KV8_ERR_CUDA;
   return KV8_OK;

@@ -17,6 +17,9 @@ namespace kv8 {
 // of its work instead of hanging.
 enum : uint32_t {
   KV8_DEV_WAIT_TIMEOUT = 1u,
+  // a shared-prefix group listed a member whose context is shorter than the
+  // group's prefix; that member's shared chunks were skipped
+  KV8_DEV_BAD_PREFIX = 2u,
 };
 
 // Upper bound on mbarrier polls before a wait gives up (each poll may also

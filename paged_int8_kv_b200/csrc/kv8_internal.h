@@ -55,6 +55,19 @@ struct DecodeParams {
   int32_t max_chunks;    // ceil(max_context_len / chunk_tokens)
   int32_t out_f32;       // 1 = fp32 output, 0 = bf16
   float q_scale;         // softmax_scale * log2(e)
+  // shared prefixes (nullptr when the batch has none): sequence b belongs to
+  // group prefix_group[b] (or none, -1), whose first
+  // prefix_lens[g] / chunk_tokens whole chunks a prefix launch computes; a
+  // decode launch then skips those chunks of b
+  const int32_t* prefix_group;  // [B]
+  const int32_t* prefix_lens;   // [num_groups]
+};
+
+// Extra launch facts of the shared-prefix kernel.
+struct PrefixShape {
+  int32_t num_groups;
+  int32_t rounds;         // ceil(max members per group / 8)
+  int32_t prefix_chunks;  // max over groups of prefix_lens / chunk_tokens
 };
 
 // Workspace carve-up shared by the decode and reduce launchers.
@@ -83,6 +96,16 @@ int launch_split_reduce(const float* ws_ml, const float* ws_o,
                         int32_t num_q_heads, int32_t chunk_tokens,
                         int32_t max_chunks, void* out, int32_t out_f32,
                         cudaStream_t stream);
+
+// The shared-prefix chunks of a batch (kv8_prefix.cu): one CTA of 8 warps
+// per (chunk, KV head, group, round of 8 members).  Same return codes as
+// launch_decode.
+int launch_prefix(const DecodeParams& p, const PrefixShape& ps,
+                  const CUtensorMap& tmk, const CUtensorMap& tmv,
+                  cudaStream_t stream);
+
+// Sticky status word of the shared-prefix kernel (no synchronize).
+int read_prefix_status(uint32_t* value, int clear);
 
 // Decode on the tcgen05 tensor cores (kv8_decode_tc.cu); same contract as
 // launch_decode.
