@@ -215,6 +215,41 @@ KV8_API int32_t kv8_paged_decode_attention_prefix(
     size_t workspace_bytes, void *out, int32_t out_dtype, void *stream);
 
 /*
+ * kv8_paged_extend_attention -- extend (prefill) attention over the paged
+ * INT8 cache: every sequence's new query rows attend causally to its cache.
+ *
+ * A prompt's tokens are processed together and fill the cache; a long prompt
+ * may enter in chunks, each attending to everything cached before it
+ * [KV Cache 优化全景解析——从基础原理到工程实践, §2.2 Prefill 与 Decode 两阶段,
+ * §11.2 chunked prefill].  The new K/V rows are appended first
+ * (kv8_quantize_append), as in decode.  Sequence b has n_b = q_start[b+1] -
+ * q_start[b] new rows, its last n_b cached positions; row i sits at position
+ * p = context_lens[b] - n_b + i and attends to tokens 0..p:
+ *     out = softmax(q K_hat^T / sqrt(d)) V_hat     [same page, §2.1]
+ * with K_hat = code * ks, V_hat = code * vs and fp32 accumulation.  Both
+ * products run on the 5th-generation tensor cores (fp16 operands: the INT8
+ * codes exactly, q scaled per row by a power of two, the probabilities
+ * rounded to fp16).
+ *
+ *   q            bf16 [q_start[batch]][num_q_heads][head_dim], rows packed
+ *                by sequence
+ *   q_start      int32 [batch + 1] device, non-decreasing from 0;
+ *                n_b <= context_lens[b]
+ *   max_q_len    host bound on n_b (sizes the grid)
+ *   out          [q_start[batch]][num_q_heads][head_dim], bf16 or fp32
+ * Other arguments as kv8_paged_decode_attention; no workspace.  The call
+ * enqueues one kernel.
+ */
+KV8_API int32_t kv8_paged_extend_attention(
+    const void *q, const int8_t *k_cache, const int8_t *v_cache,
+    const float *k_scales, const float *v_scales, const int32_t *block_tables,
+    const int32_t *context_lens, const int32_t *q_start, int32_t batch,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_q_len, float softmax_scale, void *out, int32_t out_dtype,
+    void *stream);
+
+/*
  * kv8_split_reduce -- merge the per-chunk partials of a split decode launch.
  *
  * For each (b, h) whose context spans C = ceil(n / chunk_tokens) > 1 chunks,

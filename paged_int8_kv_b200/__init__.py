@@ -20,7 +20,7 @@ _BINDING_NAMES = {
     "Kv8Error", "default_softmax_scale", "kv8_decode_chunk_tokens",
     "kv8_decode_workspace_bytes",
     "kv8_paged_decode_attention", "kv8_paged_decode_attention_form",
-    "kv8_paged_decode_attention_prefix",
+    "kv8_paged_decode_attention_prefix", "kv8_paged_extend_attention",
     "kv8_paged_decode_attention_noalloc",
     "kv8_quantize_append",
     "kv8_read_device_status", "kv8_split_reduce",

@@ -39,6 +39,7 @@ EXPORTED = (
     "kv8_split_reduce",
     "kv8_paged_decode_attention_form",
     "kv8_paged_decode_attention_prefix",
+    "kv8_paged_extend_attention",
     "kv8_read_device_status",
     "kv8_paged_decode_attention_noalloc",
 )
@@ -74,6 +75,10 @@ def _load() -> ctypes.CDLL:
     lib.kv8_paged_decode_attention_prefix.argtypes = [
         P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, P, P,
         i32, i32, i32, f32, i32, P, sz, P, i32, P]
+    lib.kv8_paged_extend_attention.restype = i32
+    lib.kv8_paged_extend_attention.argtypes = [
+        P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32,
+        P, i32, P]
     lib.kv8_split_reduce.restype = i32
     lib.kv8_split_reduce.argtypes = [P, sz, P, i32, i32, i32, i32, i32, P, i32, P]
     lib.kv8_paged_decode_attention_form.restype = i32
@@ -215,6 +220,28 @@ def kv8_paged_decode_attention_prefix(q: torch.Tensor, k_cache: torch.Tensor,
                *a[:15], _p(prefix_group), _p(prefix_lens),
                int(prefix_lens.shape[0]), int(max_group_size),
                int(max_prefix_len), *a[15:], _stream(stream)))
+    return out
+
+
+def kv8_paged_extend_attention(q: torch.Tensor, k_cache: torch.Tensor,
+                               v_cache: torch.Tensor, k_scales: torch.Tensor,
+                               v_scales: torch.Tensor,
+                               block_tables: torch.Tensor,
+                               context_lens: torch.Tensor,
+                               q_start: torch.Tensor, out: torch.Tensor,
+                               max_q_len: int, softmax_scale: float = 0.0,
+                               stream=None) -> torch.Tensor:
+    """q bf16 [rows, H_q, D] (new rows of every sequence, packed);
+    q_start int32 [B+1]; out bf16 or fp32 like q (written in place)."""
+    nq, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    out_dtype = KV8_OUT_F32 if out.dtype == torch.float32 else KV8_OUT_BF16
+    _check("kv8_paged_extend_attention", lib.kv8_paged_extend_attention(
+        _p(q), _p(k_cache), _p(v_cache), _p(k_scales), _p(v_scales),
+        _p(block_tables), _p(context_lens), _p(q_start),
+        int(context_lens.shape[0]), hq, hkv, d, bs, block_tables.shape[1], nb,
+        int(max_q_len), float(softmax_scale), _p(out), out_dtype,
+        _stream(stream)))
     return out
 
 

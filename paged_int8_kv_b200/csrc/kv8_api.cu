@@ -348,6 +348,50 @@ int32_t kv8_paged_decode_attention_prefix(
   return KV8_OK;
 }
 
+int32_t kv8_paged_extend_attention(
+    const void* q, const int8_t* k_cache, const int8_t* v_cache,
+    const float* k_scales, const float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, const int32_t* q_start, int32_t batch,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_q_len, float softmax_scale, void* out, int32_t out_dtype,
+    void* stream) {
+  if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
+      max_q_len < 0)
+    return KV8_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return KV8_ERR_INVALID_ARG;
+  if (out_dtype != KV8_OUT_BF16 && out_dtype != KV8_OUT_F32)
+    return KV8_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || block_size != kBlockSize)
+    return KV8_ERR_UNSUPPORTED;
+  if (!group_supported(num_q_heads / num_kv_heads)) return KV8_ERR_UNSUPPORTED;
+  if (batch > 65535 || num_kv_heads > 65535) return KV8_ERR_UNSUPPORTED;
+  if (num_blocks > INT32_MAX / num_kv_heads) return KV8_ERR_UNSUPPORTED;
+  if (batch == 0 || max_q_len == 0) return KV8_OK;
+  if (!q || !k_cache || !v_cache || !k_scales || !v_scales || !block_tables ||
+      !context_lens || !q_start || !out)
+    return KV8_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(k_scales) || !aligned16(v_scales) || !aligned4(block_tables) ||
+      !aligned4(context_lens) || !aligned4(q_start) || !aligned16(out))
+    return KV8_ERR_INVALID_ARG;
+  CUtensorMap tmk, tmv;
+  const int64_t pages = num_blocks * num_kv_heads;
+  if (!encode_page_map(&tmk, k_cache, pages) ||
+      !encode_page_map(&tmv, v_cache, pages))
+    return KV8_ERR_CUDA;
+  if (!(softmax_scale > 0.0f))
+    softmax_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(head_dim)));
+  const int rc = kv8::launch_extend(
+      q, k_scales, v_scales, block_tables, context_lens, q_start, batch,
+      num_q_heads, num_kv_heads, max_blocks_per_seq, max_q_len, softmax_scale,
+      out, out_dtype == KV8_OUT_F32 ? 1 : 0, tmk, tmv,
+      static_cast<cudaStream_t>(stream));
+  if (rc == -2) return KV8_ERR_UNSUPPORTED;
+  return rc == 0 ? KV8_OK : KV8_ERR_CUDA;
+}
+
 int32_t kv8_split_reduce(const void* workspace, size_t workspace_bytes,
                          const int32_t* context_lens, int32_t batch,
                          int32_t num_q_heads, int32_t head_dim,

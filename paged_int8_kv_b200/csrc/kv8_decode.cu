@@ -385,10 +385,11 @@ int read_device_status(uint32_t* value, int clear) {
         cudaSuccess)
       return -1;
   }
-  uint32_t tc = 0, pf = 0;
+  uint32_t tc = 0, pf = 0, ex = 0;
   if (read_tc_status(&tc, clear) != 0) return -1;
   if (read_prefix_status(&pf, clear) != 0) return -1;
-  *value |= tc | pf;
+  if (read_ext_status(&ex, clear) != 0) return -1;
+  *value |= tc | pf | ex;
   return 0;
 }
 

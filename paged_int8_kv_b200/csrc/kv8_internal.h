@@ -107,6 +107,19 @@ int launch_prefix(const DecodeParams& p, const PrefixShape& ps,
 // Sticky status word of the shared-prefix kernel (no synchronize).
 int read_prefix_status(uint32_t* value, int clear);
 
+// Extend (prefill) attention on tcgen05 (kv8_extend.cu).  Same return codes
+// as launch_decode.
+int launch_extend(const void* q, const float* k_scales, const float* v_scales,
+                  const int32_t* block_tables, const int32_t* context_lens,
+                  const int32_t* q_start, int32_t batch, int32_t num_q_heads,
+                  int32_t num_kv_heads, int32_t max_blocks_per_seq,
+                  int32_t max_q_len, float softmax_scale, void* out,
+                  int32_t out_f32, const CUtensorMap& tmk,
+                  const CUtensorMap& tmv, cudaStream_t stream);
+
+// Sticky status word of the extend kernel (no synchronize).
+int read_ext_status(uint32_t* value, int clear);
+
 // Decode on the tcgen05 tensor cores (kv8_decode_tc.cu); same contract as
 // launch_decode.
 int launch_decode_tc(const DecodeParams& p, const CUtensorMap& tmk,
