@@ -250,6 +250,58 @@ KV8_API int32_t kv8_paged_extend_attention(
     void *stream);
 
 /*
+ * Context-parallel decode: one long context spread over several GPUs.
+ *
+ * Context partitioning splits a sequence's context across devices that each
+ * process their own part [garden.houmin.site infra/kv-cache-optimize,
+ * §4.1.2 KV-Runahead]; for decode, each rank holds the blocks of its part of
+ * every sequence (its own cache, block tables and context lengths for that
+ * part), computes the chunk partials (m, l, o) of its part, the ranks
+ * exchange the partials (an all-gather of (2 + head_dim) floats per chunk and
+ * query head), and the log-sum-exp merge over every rank's chunks gives the
+ * attention over the whole context, the merge kv8_split_reduce performs for
+ * one rank.
+ *
+ * kv8_decode_partials_bytes -- bytes of one rank's partials: per (sequence,
+ * query head, chunk slot) (m, l) then o, for C = ceil(max_context_len /
+ * chunk_tokens) slots (at least 1).  0 for invalid arguments.
+ *
+ * kv8_paged_decode_attention_partials -- the decode call of one rank: the
+ * same arguments as kv8_paged_decode_attention (its local cache, tables and
+ * context lengths), chunk_tokens > 0, every chunk slot of every (sequence,
+ * query head) written to `partials` (empty slots as m = -inf, l = 0, o = 0),
+ * nothing merged, no output.  Every rank must use the same batch,
+ * num_q_heads, max_context_len (a bound on every rank's local lengths) and
+ * chunk_tokens, so that the layouts match.
+ *
+ * kv8_merge_partials -- the log-sum-exp merge over `ranks` partial buffers,
+ * rank r's at partials + r * rank_stride bytes (each written by
+ * kv8_paged_decode_attention_partials with the same batch, num_q_heads,
+ * max_context_len and chunk_tokens), into out [batch][num_q_heads][head_dim]
+ * (bf16 or fp32).
+ */
+KV8_API size_t kv8_decode_partials_bytes(int32_t batch, int32_t num_q_heads,
+                                         int32_t head_dim,
+                                         int32_t max_context_len,
+                                         int32_t chunk_tokens);
+
+KV8_API int32_t kv8_paged_decode_attention_partials(
+    const void *q, const int8_t *k_cache, const int8_t *v_cache,
+    const float *k_scales, const float *v_scales, const int32_t *block_tables,
+    const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void *partials,
+    size_t partials_bytes, void *stream);
+
+KV8_API int32_t kv8_merge_partials(const void *partials, size_t rank_stride,
+                                   int32_t ranks, int32_t batch,
+                                   int32_t num_q_heads, int32_t head_dim,
+                                   int32_t max_context_len,
+                                   int32_t chunk_tokens, void *out,
+                                   int32_t out_dtype, void *stream);
+
+/*
  * kv8_split_reduce -- merge the per-chunk partials of a split decode launch.
  *
  * For each (b, h) whose context spans C = ceil(n / chunk_tokens) > 1 chunks,

@@ -40,6 +40,9 @@ EXPORTED = (
     "kv8_paged_decode_attention_form",
     "kv8_paged_decode_attention_prefix",
     "kv8_paged_extend_attention",
+    "kv8_decode_partials_bytes",
+    "kv8_paged_decode_attention_partials",
+    "kv8_merge_partials",
     "kv8_read_device_status",
     "kv8_paged_decode_attention_noalloc",
 )
@@ -79,6 +82,15 @@ def _load() -> ctypes.CDLL:
     lib.kv8_paged_extend_attention.argtypes = [
         P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32,
         P, i32, P]
+    lib.kv8_decode_partials_bytes.restype = sz
+    lib.kv8_decode_partials_bytes.argtypes = [i32, i32, i32, i32, i32]
+    lib.kv8_paged_decode_attention_partials.restype = i32
+    lib.kv8_paged_decode_attention_partials.argtypes = [
+        P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
+        P, sz, P]
+    lib.kv8_merge_partials.restype = i32
+    lib.kv8_merge_partials.argtypes = [P, sz, i32, i32, i32, i32, i32, i32,
+                                       P, i32, P]
     lib.kv8_split_reduce.restype = i32
     lib.kv8_split_reduce.argtypes = [P, sz, P, i32, i32, i32, i32, i32, P, i32, P]
     lib.kv8_paged_decode_attention_form.restype = i32
@@ -267,6 +279,51 @@ def kv8_paged_decode_attention_noalloc(q: torch.Tensor, k_cache: torch.Tensor,
                block_tables.shape[1], nb, int(max_context_len),
                float(softmax_scale), int(chunk_tokens), _p(out), out_dtype,
                _stream(stream)))
+    return out
+
+
+def kv8_decode_partials_bytes(batch: int, num_q_heads: int, head_dim: int,
+                              max_context_len: int, chunk_tokens: int) -> int:
+    return int(lib.kv8_decode_partials_bytes(batch, num_q_heads, head_dim,
+                                             max_context_len, chunk_tokens))
+
+
+def kv8_paged_decode_attention_partials(q: torch.Tensor, k_cache: torch.Tensor,
+                                        v_cache: torch.Tensor,
+                                        k_scales: torch.Tensor,
+                                        v_scales: torch.Tensor,
+                                        block_tables: torch.Tensor,
+                                        context_lens: torch.Tensor,
+                                        partials: torch.Tensor,
+                                        max_context_len: int,
+                                        chunk_tokens: int,
+                                        softmax_scale: float = 0.0,
+                                        stream=None) -> torch.Tensor:
+    """One rank's chunk partials of a context-parallel decode (uint8 buffer
+    of kv8_decode_partials_bytes bytes, written in place)."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    _check("kv8_paged_decode_attention_partials",
+           lib.kv8_paged_decode_attention_partials(
+               _p(q), _p(k_cache), _p(v_cache), _p(k_scales), _p(v_scales),
+               _p(block_tables), _p(context_lens), B, hq, hkv, d, bs,
+               block_tables.shape[1], nb, int(max_context_len),
+               float(softmax_scale), int(chunk_tokens), _p(partials),
+               partials.numel() * partials.element_size(), _stream(stream)))
+    return partials
+
+
+def kv8_merge_partials(partials: torch.Tensor, rank_stride: int, ranks: int,
+                       out: torch.Tensor, max_context_len: int,
+                       chunk_tokens: int, stream=None) -> torch.Tensor:
+    """Merge `ranks` partial buffers (rank r at byte r * rank_stride of
+    `partials`) into out [B, H_q, D] (bf16 or fp32, written in place)."""
+    B, hq, d = out.shape
+    out_dtype = KV8_OUT_F32 if out.dtype == torch.float32 else KV8_OUT_BF16
+    _check("kv8_merge_partials", lib.kv8_merge_partials(
+        _p(partials), int(rank_stride), int(ranks), B, hq, d,
+        int(max_context_len), int(chunk_tokens), _p(out), out_dtype,
+        _stream(stream)))
     return out
 
 

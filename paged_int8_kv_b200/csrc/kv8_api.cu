@@ -91,7 +91,8 @@ int32_t prepare_decode(
     int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
     int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
     float softmax_scale, int32_t chunk_tokens, void* workspace,
-    size_t workspace_bytes, void* out, int32_t out_dtype, DecodeSetup* d) {
+    size_t workspace_bytes, void* out, int32_t out_dtype, DecodeSetup* d,
+    bool partials_only = false) {
   // ---- shape checks
   if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
@@ -129,16 +130,19 @@ int32_t prepare_decode(
   float* ws_ml = nullptr;
   float* ws_o = nullptr;
   uint32_t* ws_ctr = nullptr;
-  if (max_chunks > 1) {
-    const size_t need = kv8::workspace_total_bytes(batch, num_q_heads, max_chunks);
+  if (max_chunks > 1 || partials_only) {
+    const size_t ml_bytes = kv8::workspace_ml_bytes(batch, num_q_heads, max_chunks);
+    const size_t o_bytes = kv8::workspace_o_bytes(batch, num_q_heads, max_chunks);
+    const size_t need =
+        partials_only ? ml_bytes + o_bytes
+                      : kv8::workspace_total_bytes(batch, num_q_heads, max_chunks);
     if (!workspace || workspace_bytes < need || !aligned16(workspace))
       return KV8_ERR_WORKSPACE;
     uint8_t* base = static_cast<uint8_t*>(workspace);
-    const size_t ml_bytes = kv8::workspace_ml_bytes(batch, num_q_heads, max_chunks);
-    const size_t o_bytes = kv8::workspace_o_bytes(batch, num_q_heads, max_chunks);
     ws_ml = reinterpret_cast<float*>(base);
     ws_o = reinterpret_cast<float*>(base + ml_bytes);
-    ws_ctr = reinterpret_cast<uint32_t*>(base + ml_bytes + o_bytes);
+    if (!partials_only)
+      ws_ctr = reinterpret_cast<uint32_t*>(base + ml_bytes + o_bytes);
   }
 
   const int64_t pages = num_blocks * num_kv_heads;
@@ -169,6 +173,7 @@ int32_t prepare_decode(
                                  1.4426950408889634074);  // log2(e)
   p.prefix_group = nullptr;
   p.prefix_lens = nullptr;
+  p.partials_only = partials_only ? 1 : 0;
   return KV8_OK;
 }
 
@@ -389,6 +394,69 @@ int32_t kv8_paged_extend_attention(
       out, out_dtype == KV8_OUT_F32 ? 1 : 0, tmk, tmv,
       static_cast<cudaStream_t>(stream));
   if (rc == -2) return KV8_ERR_UNSUPPORTED;
+  return rc == 0 ? KV8_OK : KV8_ERR_CUDA;
+}
+
+size_t kv8_decode_partials_bytes(int32_t batch, int32_t num_q_heads,
+                                 int32_t head_dim, int32_t max_context_len,
+                                 int32_t chunk_tokens) {
+  if (batch <= 0 || num_q_heads <= 0 || head_dim != kHeadDim ||
+      max_context_len < 0 || chunk_tokens <= 0 || chunk_tokens % kBlockSize)
+    return 0;
+  int32_t chunk_eff, max_chunks;
+  split_shape(max_context_len, chunk_tokens, &chunk_eff, &max_chunks);
+  return kv8::workspace_ml_bytes(batch, num_q_heads, max_chunks) +
+         kv8::workspace_o_bytes(batch, num_q_heads, max_chunks);
+}
+
+int32_t kv8_paged_decode_attention_partials(
+    const void* q, const int8_t* k_cache, const int8_t* v_cache,
+    const float* k_scales, const float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void* partials,
+    size_t partials_bytes, void* stream) {
+  if (chunk_tokens <= 0) return KV8_ERR_INVALID_ARG;
+  DecodeSetup d;
+  const int32_t rc0 = prepare_decode(
+      q, k_cache, v_cache, k_scales, v_scales, block_tables, context_lens,
+      batch, num_q_heads, num_kv_heads, head_dim, block_size,
+      max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+      chunk_tokens, partials, partials_bytes, partials /* unused out */,
+      KV8_OUT_F32, &d, true);
+  if (rc0 != KV8_OK || d.nothing) return rc0;
+  const int rc = kv8::launch_decode(d.p, d.tmk, d.tmv, KV8_FORM_AUTO,
+                                    static_cast<cudaStream_t>(stream));
+  if (rc == -2) return KV8_ERR_UNSUPPORTED;
+  return rc == 0 ? KV8_OK : KV8_ERR_CUDA;
+}
+
+int32_t kv8_merge_partials(const void* partials, size_t rank_stride,
+                           int32_t ranks, int32_t batch, int32_t num_q_heads,
+                           int32_t head_dim, int32_t max_context_len,
+                           int32_t chunk_tokens, void* out, int32_t out_dtype,
+                           void* stream) {
+  if (ranks <= 0 || batch < 0 || num_q_heads <= 0 || max_context_len < 0 ||
+      chunk_tokens <= 0)
+    return KV8_ERR_INVALID_ARG;
+  if (out_dtype != KV8_OUT_BF16 && out_dtype != KV8_OUT_F32)
+    return KV8_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim) return KV8_ERR_UNSUPPORTED;
+  if (chunk_tokens % kBlockSize != 0) return KV8_ERR_INVALID_ARG;
+  if (batch == 0) return KV8_OK;
+  const size_t one = kv8_decode_partials_bytes(batch, num_q_heads, head_dim,
+                                               max_context_len, chunk_tokens);
+  if (!partials || !out || !aligned16(partials) || !aligned16(out) ||
+      (rank_stride & 15u))
+    return KV8_ERR_INVALID_ARG;
+  if (ranks > 1 && rank_stride < one) return KV8_ERR_INVALID_ARG;
+  int32_t chunk_eff, max_chunks;
+  split_shape(max_context_len, chunk_tokens, &chunk_eff, &max_chunks);
+  const int rc = kv8::launch_merge_ranks(
+      static_cast<const uint8_t*>(partials), rank_stride, ranks, batch,
+      num_q_heads, max_chunks, out, out_dtype == KV8_OUT_F32 ? 1 : 0,
+      static_cast<cudaStream_t>(stream));
   return rc == 0 ? KV8_OK : KV8_ERR_CUDA;
 }
 

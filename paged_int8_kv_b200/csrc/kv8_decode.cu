@@ -108,6 +108,11 @@ __device__ __forceinline__ bool item_done(const DecodeParams& p,
 __device__ __forceinline__ bool item_fill(const DecodeParams& p, Item& it) {
   it.n = p.context_lens[it.b];
   it.tok0 = it.chunk * p.chunk_tokens;
+  if (p.partials_only && it.tok0 >= it.n) {  // an empty slot: (-inf, 0, 0)
+    it.tok1 = it.tok0;
+    it.npages = 0;
+    return true;
+  }
   if (it.tok0 >= it.n && !(it.n == 0 && it.chunk == 0)) return false;
   if (p.prefix_group) {  // whole chunks of a shared prefix: a prefix launch's
     const int g = p.prefix_group[it.b];
@@ -260,11 +265,11 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     sk.ci0 = row0 * p.max_chunks + cmp.chunk;
     sk.max_chunks = p.max_chunks;
     const int nchunks = (cmp.n + p.chunk_tokens - 1) / p.chunk_tokens;
-    sk.single = nchunks <= 1;
+    sk.single = nchunks <= 1 && !p.partials_only;
     sk.out_f32 = p.out_f32;
     math.finish(sk);
 
-    if (!sk.single) {
+    if (!sk.single && !p.partials_only) {
       // the last chunk of this (sequence, KV group) to finish merges them
       __threadfence();
       __syncwarp();
@@ -307,6 +312,57 @@ split_reduce_kernel(const float* __restrict__ ws_ml,
   merge_head_warp(ws_ml + static_cast<int64_t>(bh) * max_chunks * 2,
                   ws_o + static_cast<int64_t>(bh) * max_chunks * kD, nchunks,
                   out, bh, out_f32);
+}
+
+// --------------------------------------------------------------------------
+// Merge across ranks: one warp per (b, hq) over ranks x max_chunks partials
+// (empty ones carry m = -inf and weigh nothing).
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(32)
+merge_ranks_kernel(const uint8_t* __restrict__ partials, size_t rank_stride,
+                   size_t o_offset, int32_t ranks, int32_t max_chunks,
+                   void* out, int32_t out_f32) {
+  const int64_t bh = blockIdx.x;
+  const int lane = threadIdx.x;
+  const int total = ranks * max_chunks;
+  auto ml_at = [&](int k) {
+    const int r = k / max_chunks, c = k - r * max_chunks;
+    return reinterpret_cast<const float*>(partials + r * rank_stride) +
+           (bh * max_chunks + c) * 2;
+  };
+  auto o_at = [&](int k) {
+    const int r = k / max_chunks, c = k - r * max_chunks;
+    return reinterpret_cast<const float*>(partials + r * rank_stride + o_offset) +
+           (bh * max_chunks + c) * kD;
+  };
+  float mx = -INFINITY;
+  for (int k = lane; k < total; k += 32) mx = fmaxf(mx, ml_at(k)[0]);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+  float ls = 0.0f;
+  for (int k = lane; k < total; k += 32) {
+    const float* ml = ml_at(k);
+    ls += ml[0] == -INFINITY ? 0.0f : ml[1] * ex2(ml[0] - mx);
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) ls += __shfl_xor_sync(kFull, ls, m);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < total; ++k) {
+    const float mc = ml_at(k)[0];
+    if (mc == -INFINITY) continue;
+    const float w = ex2(mc - mx);
+    const float4 v = reinterpret_cast<const float4*>(o_at(k))[lane];
+    acc.x += w * v.x;
+    acc.y += w * v.y;
+    acc.z += w * v.z;
+    acc.w += w * v.w;
+  }
+  const float inv = ls > 0.0f ? 1.0f / ls : 0.0f;
+  const int64_t base = bh * kD + 4 * lane;
+  store_out(out, base + 0, acc.x * inv, out_f32);
+  store_out(out, base + 1, acc.y * inv, out_f32);
+  store_out(out, base + 2, acc.z * inv, out_f32);
+  store_out(out, base + 3, acc.w * inv, out_f32);
 }
 
 template <int G, int WPC, int SPW, class Math>
@@ -428,6 +484,18 @@ int launch_decode(const DecodeParams& p, const CUtensorMap& tmk,
     case 8: return launch_group<8>(p, tmk, tmv, variant, stream);
     default: return -2;
   }
+}
+
+int launch_merge_ranks(const uint8_t* partials, size_t rank_stride,
+                       int32_t ranks, int32_t batch, int32_t num_q_heads,
+                       int32_t max_chunks, void* out, int32_t out_f32,
+                       cudaStream_t stream) {
+  const int64_t nbh = static_cast<int64_t>(batch) * num_q_heads;
+  if (nbh == 0) return 0;
+  merge_ranks_kernel<<<static_cast<unsigned>(nbh), 32, 0, stream>>>(
+      partials, rank_stride, workspace_ml_bytes(batch, num_q_heads, max_chunks),
+      ranks, max_chunks, out, out_f32);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 int launch_split_reduce(const float* ws_ml, const float* ws_o,

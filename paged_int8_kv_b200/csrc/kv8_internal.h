@@ -61,6 +61,10 @@ struct DecodeParams {
   // decode launch then skips those chunks of b
   const int32_t* prefix_group;  // [B]
   const int32_t* prefix_lens;   // [num_groups]
+  // 1: write the (m, l, o) partial of every chunk slot c < max_chunks of
+  // every (sequence, query head), empty chunks as (-inf, 0, 0), and merge
+  // nothing (the partials of several launches are merged afterwards)
+  int32_t partials_only;
 };
 
 // Extra launch facts of the shared-prefix kernel.
@@ -78,6 +82,14 @@ size_t workspace_o_bytes(int32_t batch, int32_t num_q_heads,
 size_t workspace_ctr_bytes(int32_t batch, int32_t num_q_heads);
 size_t workspace_total_bytes(int32_t batch, int32_t num_q_heads,
                              int32_t max_chunks);
+
+// Merge of the chunk partials of several launches (one per rank of a
+// context-parallel decode): rank r's partials, laid out as a workspace's
+// (m, l) and o regions, start `rank_stride` bytes after rank r-1's.
+int launch_merge_ranks(const uint8_t* partials, size_t rank_stride,
+                       int32_t ranks, int32_t batch, int32_t num_q_heads,
+                       int32_t max_chunks, void* out, int32_t out_f32,
+                       cudaStream_t stream);
 
 int launch_quantize_append(const void* k_new, const void* v_new,
                            const int64_t* slot_mapping, int64_t n_tokens,
