@@ -335,7 +335,7 @@ class DeviceWorkload:
     def decode(self, form, q=None, bt=None, cl=None):
         import paged_int8_kv_b200 as pk
         c = self.cache
-        if self.use_prefix and form == 0:
+        if self.use_prefix:
             pg, pl, gmax, plen = self.prefix
             pk.kv8_paged_decode_attention_prefix(
                 self.q if q is None else q, c.k_cache, c.v_cache, c.k_scales,
@@ -379,12 +379,19 @@ def time_decode_calls(dw: DeviceWorkload, form: int, calls: int, warmup: int,
           for _ in range(calls)]
     for i in range(calls):
         if flush is not None:
-            flush.fill_(i & 0xFF)
+            flush_l2(flush)
         ev[i][0].record(stream)
         dw.decode(form)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     return [a.elapsed_time(b) for a, b in ev]
+
+
+def flush_l2(buf) -> None:
+    """Evict L2 by reading a buffer larger than it (a read leaves no dirty
+    lines behind, so the timed call pays no write-back of the flush)."""
+    import torch
+    buf.view(torch.int64).amax()
 
 
 def rate_record(w: W.Workload, dec_ms: float, peak: float) -> dict:
@@ -413,7 +420,7 @@ def run_per_workload(args, dev, peak: float) -> dict:
     timed one decode call at a time (median of ``--calls`` calls, L2
     flushed before each call: these caches fit in or near L2)."""
     import torch
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
     res = {}
     for name in PER_WORKLOAD:
         w = W.NAMED[name]()
@@ -450,7 +457,7 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     flush = None
     ab = algorithmic_bytes(w)
     if ab["total"] <= 4 * 126e6:
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
     # per step: the quantize-append kernel and the decode kernel (a split
     # launch also enqueues a small memset of its merge tickets)
     launches_per_step = 2
@@ -492,7 +499,7 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     t_start.record(stream)
     for i in range(args.steps):
         if flush is not None:
-            flush.fill_(i & 0xFF)
+            flush_l2(flush)
         ev[i][0].record(stream)
         dw.append()
         dec[i][0].record(stream)
@@ -548,7 +555,7 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     e0.record(stream)
     for _ in range(args.steps):
         if flush is not None:
-            flush.fill_(1)
+            flush_l2(flush)
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
@@ -623,6 +630,81 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     return 0
 
 
+def extend_flops(lens, new, num_q_heads: int, head_dim: int = 128) -> int:
+    """Algorithmic flops of a causal extend: every new row of every query
+    head against every token it sees, 2*d for q.k and 2*d for p.v."""
+    total = 0
+    for t, n in zip(lens, new):
+        keys = sum(t - n + i + 1 for i in range(n))
+        total += 4 * head_dim * keys * num_q_heads
+    return total
+
+
+def run_extend(args, rank: int, world: int, dist):
+    """Extend (chunked-prefill) attention: batch 4 sequences of the
+    Llama-3.1-8B head shape, 32768 cached tokens each, of which the last
+    2048 are the new query rows; one kv8_paged_extend_attention call per
+    step, inputs resident (1.1 GB of cache, larger than L2)."""
+    import torch
+    import paged_int8_kv_b200 as pk
+    dev = torch.device("cuda", _env_int("LOCAL_RANK", 0))
+    torch.cuda.set_device(dev)
+    B, T, NEW = 4, 32768, 2048
+    w = W.make_workload("llama8b_extend_b4_ctx32k_new2k", 1006, [T] * B, 32, 8,
+                        description="batch 4, context 32768, 2048 new rows each")
+    dw = DeviceWorkload(w, dev, 0)
+    qs = np.arange(0, (B + 1) * NEW, NEW, dtype=np.int32)
+    rng = np.random.default_rng([1006, 9])
+    qh = W.f32_to_bf16_bits(rng.standard_normal((B * NEW, 32, 128), dtype=np.float32))
+    q = torch.from_numpy(qh).view(torch.bfloat16).to(dev)
+    qsd = torch.from_numpy(qs).to(dev)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    c = dw.cache
+
+    def call():
+        pk.kv8_paged_extend_attention(q, c.k_cache, c.v_cache, c.k_scales,
+                                      c.v_scales, dw.bt, dw.cl, qsd, out, NEW)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    stream = torch.cuda.current_stream()
+    for a, b in ev:
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.median([a.elapsed_time(b) for a, b in ev])
+    ms = max_over_ranks([ms], dist, dev)[0]
+    status = pk.kv8_read_device_status(clear=True)
+    fl = extend_flops([T] * B, [NEW] * B, 32)
+    peak = None
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        peak = 1590.0
+    tflops = fl / (ms * 1e-3) / 1e12
+    if rank == 0:
+        print(json.dumps({
+            "metric": "paged KV8 extend attention new tokens/s and tensor TFLOP/s",
+            "value": whole_job_rate(B * NEW, world, ms), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16 operands, f32 accumulation",
+            "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": w.name, "batch": B, "context": T,
+                       "new_rows": NEW, "q_heads": 32, "kv_heads": 8},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": tflops / peak,
+                         "algorithmic_flops": fl,
+                         "peak_source": "MEASURED_PEAKS.json bf16_tflops (fp16 "
+                                        "runs at the bf16 rate)"},
+            "device_status": status}), flush=True)
+    return 0
+
+
 def run_dry_cpu(args, rank: int, world: int, dist):
     """The launch and rank logic alone, on CPU ranks over gloo: every rank
     times a trivial host step, the max over ranks is taken, rank 0 prints a
@@ -681,6 +763,8 @@ def main():
     ap.add_argument("--ref-seqs", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true")
+    ap.add_argument("--extend", action="store_true",
+                    help="time extend (chunked-prefill) attention instead")
     ap.add_argument("--dry-run-cpu", action="store_true",
                     help="rank/launch logic only, on CPU over gloo (no GPU work, "
                          "no measurement)")
@@ -710,6 +794,8 @@ def main():
     try:
         if args.dry_run_cpu:
             return run_dry_cpu(args, rank, world, dist)
+        if args.extend:
+            return run_extend(args, rank, world, dist)
         return run_kv8(args, W.NAMED[args.workload](), rank, world, dist)
     finally:
         if dist is not None:

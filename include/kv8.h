@@ -327,7 +327,8 @@ KV8_API int32_t kv8_split_reduce(const void *workspace, size_t workspace_bytes,
                          void *out, int32_t out_dtype, void *stream);
 
 /* Decode forms for kv8_paged_decode_attention_form. */
-#define KV8_FORM_AUTO 0      /* what kv8_paged_decode_attention uses */
+#define KV8_FORM_AUTO 0      /* KV8_FORM_MMA_I8 for groups of <= 4 heads,
+                                KV8_FORM_MMA_F16PV for groups of 8 */
 #define KV8_FORM_CUDA_CORE 1 /* codes converted to fp32, fp32 FMA */
 #define KV8_FORM_MMA_F16PV 2 /* warp mma: int8 q.k, fp16 p.v */
 #define KV8_FORM_TCGEN05 3   /* 5th-generation tensor cores, TMEM accumulators */
@@ -336,7 +337,9 @@ KV8_API int32_t kv8_split_reduce(const void *workspace, size_t workspace_bytes,
 /*
  * kv8_paged_decode_attention_form -- kv8_paged_decode_attention with the
  * decode form chosen by the caller, for every call separately:
- *   KV8_FORM_AUTO       the form kv8_paged_decode_attention uses,
+ *   KV8_FORM_AUTO       the form kv8_paged_decode_attention uses:
+ *                       KV8_FORM_MMA_I8 for groups of 1, 2 or 4 query
+ *                       heads per KV head, KV8_FORM_MMA_F16PV for 8,
  *   KV8_FORM_CUDA_CORE  codes converted to fp32 in registers, fp32 FMA,
  *   KV8_FORM_MMA_F16PV  warp tensor cores (mma.sync): q.k as int8 products
  *                       of the K codes with exact int8 digit planes of q;

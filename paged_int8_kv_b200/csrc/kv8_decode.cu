@@ -412,8 +412,10 @@ int launch_group(const DecodeParams& p, const CUtensorMap& tmk,
                  const CUtensorMap& tmv, int32_t variant, cudaStream_t stream) {
   if (variant == KV8_FORM_CUDA_CORE)
     return launch_decode_kernel<G, 4, 4, SimtMath<G>>(p, tmk, tmv, stream);
+  // automatic: both products on int8 mma for groups of up to 4 heads
+  // (their accumulators fit a warp), the fp16 p.v form for groups of 8
   if constexpr (G <= 4) {
-    if (variant == KV8_FORM_MMA_I8)
+    if (variant == KV8_FORM_MMA_I8 || variant == KV8_FORM_AUTO)
       return launch_decode_kernel<G, 4, 3, I8Math<G>>(p, tmk, tmv, stream);
   }
   return launch_decode_kernel<G, 4, 3, MmaMath<G>>(p, tmk, tmv, stream);
