@@ -174,6 +174,7 @@ int32_t prepare_decode(
   p.prefix_group = nullptr;
   p.prefix_lens = nullptr;
   p.partials_only = partials_only ? 1 : 0;
+  p.work_ctr = ws_ctr ? ws_ctr + static_cast<size_t>(batch) * num_q_heads : nullptr;
   return KV8_OK;
 }
 

@@ -61,9 +61,9 @@ struct SmemPlan {
   static constexpr int kTileBytes = WPC * SPW * 2 * kPageBytes;
   static constexpr int kScaleBytes = WPC * SPW * 2 * kBS * 4;
   static constexpr int kScratchBytes = WPC * ScratchBytes;
-  static constexpr int kBarBytes = WPC * SPW * 8;
+  static constexpr int kBarBytes = WPC * (SPW * 8 + 32);  // + work queue
   static constexpr int kBytes =
-      kTileBytes + kScaleBytes + kScratchBytes + kBarBytes + 1024;
+      kTileBytes + kScaleBytes + kScratchBytes + kBarBytes + 16 + 1024;
 };
 
 // --------------------------------------------------------------------------
@@ -81,25 +81,16 @@ struct Item {
   int b, kvh, chunk, n, tok0, tok1, npages;
 };
 
-// The warp stride W = (dc * H_kv + dk) * B + db as mixed-radix digits, so
-// that stepping an item is a pair of compare-and-carry steps, no division.
-struct Stride {
-  int dc, dk, db;
-};
-
-__device__ __forceinline__ void item_set(const DecodeParams& p, int64_t idx,
+// Item idx < max_chunks * H_kv * B (< 2^31), numbered chunk-major:
+// idx = (chunk * H_kv + kvh) * B + b.
+__device__ __forceinline__ void item_set(const DecodeParams& p, uint32_t idx,
                                          Item& it) {
-  const int64_t per_chunk = static_cast<int64_t>(p.num_kv_heads) * p.batch;
-  const int64_t c = idx / per_chunk;
-  const int64_t rem = idx - c * per_chunk;
-  it.chunk = c > p.max_chunks ? p.max_chunks : static_cast<int>(c);
-  it.kvh = static_cast<int>(rem / p.batch);
-  it.b = static_cast<int>(rem - static_cast<int64_t>(it.kvh) * p.batch);
-}
-
-__device__ __forceinline__ bool item_done(const DecodeParams& p,
-                                          const Item& it) {
-  return it.chunk >= p.max_chunks;
+  const uint32_t per_chunk = static_cast<uint32_t>(p.num_kv_heads) * p.batch;
+  const uint32_t c = idx / per_chunk;
+  const uint32_t rem = idx - c * per_chunk;
+  it.chunk = static_cast<int>(c);
+  it.kvh = static_cast<int>(rem / static_cast<uint32_t>(p.batch));
+  it.b = static_cast<int>(rem - static_cast<uint32_t>(it.kvh) * p.batch);
 }
 
 // Fill in the item's extent; false if the chunk lies past its sequence (a
@@ -123,23 +114,6 @@ __device__ __forceinline__ bool item_fill(const DecodeParams& p, Item& it) {
   return true;
 }
 
-__device__ __forceinline__ void item_next(const DecodeParams& p, Item& it,
-                                          const Stride& st) {
-  do {
-    it.b += st.db;
-    it.kvh += st.dk;
-    it.chunk += st.dc;
-    if (it.b >= p.batch) {
-      it.b -= p.batch;
-      ++it.kvh;
-    }
-    if (it.kvh >= p.num_kv_heads) {
-      it.kvh -= p.num_kv_heads;
-      ++it.chunk;
-    }
-  } while (!item_done(p, it) && !item_fill(p, it));
-}
-
 template <int G, int WPC, int SPW, class Math>
 __global__ void __launch_bounds__(WPC * 32,
                                   Math::kWarpsPerSM / WPC > 0 ? Math::kWarpsPerSM / WPC : 1)
@@ -156,10 +130,9 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                warp * SPW * 2 * kBS;
   uint8_t* scratch =
       smem + Plan::kTileBytes + Plan::kScaleBytes + warp * Math::kScratchBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kTileBytes +
-                                               Plan::kScaleBytes +
-                                               Plan::kScratchBytes) +
-                   warp * SPW;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      smem + Plan::kTileBytes + Plan::kScaleBytes + Plan::kScratchBytes +
+      warp * (SPW * 8 + 32));
   if (lane == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
@@ -168,31 +141,89 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     fence_mbar_init();
   }
   __syncwarp();
-
-  Stride st;
-  {
-    Item w;
-    item_set(p, static_cast<int64_t>(gridDim.x) * WPC, w);
-    st.dc = w.chunk;
-    st.dk = w.kvh;
-    st.db = w.b;
+  // tensor memory for the page math, if it keeps state there: warp w uses
+  // lanes 32w..32w+31 of the CTA's columns
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(
+      smem + Plan::kTileBytes + Plan::kScaleBytes + Plan::kScratchBytes +
+      Plan::kBarBytes);
+  if constexpr (Math::kTmemCols > 0) {
+    if (warp == 0) {
+      asm volatile(
+          "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+              smem_u32(tslot)),
+          "r"(Math::kTmemCols)
+          : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::
+                       : "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   }
-  Item cmp;
-  item_set(p, static_cast<int64_t>(blockIdx.x) * WPC + warp, cmp);
-  if (!item_done(p, cmp) && !item_fill(p, cmp)) item_next(p, cmp, st);
+
+  // ---- work items.  A warp's first item is gw = CTA * WPC + warp; its
+  // next ones are gw + W, gw + 2W, ... (W = warps in the grid) or, when the
+  // launch has a work counter, W + (counter++): a warp that finishes early
+  // takes more, so uneven items do not leave a slow tail.  The issue cursor
+  // takes items and queues their indices in shared memory; the compute
+  // cursor, up to SPW pages behind, pops them in the same order.
+  int* wq = reinterpret_cast<int*>(bars + SPW);  // 8 entries per warp
+  uint32_t q_tail = 0, q_head = 0;
+  // item indices fit 31 bits (the host checks max_chunks * H_kv * B)
+  const uint32_t n_items = static_cast<uint32_t>(p.max_chunks) *
+                           p.num_kv_heads * p.batch;
+  const uint32_t W = gridDim.x * WPC;
+  uint32_t next_idx = blockIdx.x * WPC + warp;
+  bool first_take = true;
+  // issue side: the next item that has work (or none); queues its index
+  auto take = [&](Item& it) -> bool {
+    for (;;) {
+      uint32_t idx = next_idx;
+      if (!first_take) {
+        if (p.work_ctr) {
+          uint32_t t = 0;
+          if (lane == 0) t = atomicAdd(p.work_ctr, 1u);
+          idx = W + __shfl_sync(kFull, t, 0);
+        } else {
+          idx = next_idx + W;
+        }
+      }
+      first_take = false;
+      next_idx = idx;
+      const bool live = idx < n_items;  // (no wrap: W + counter < 2^32)
+      if (live) item_set(p, idx, it);
+      if (!live || item_fill(p, it)) {
+        if (lane == 0) wq[q_tail & 7] = live ? static_cast<int>(idx) : -1;
+        ++q_tail;
+        __syncwarp();
+        return live;
+      }
+    }
+  };
+  // compute side: the next queued item (false: no more)
+  auto pop = [&](Item& it) -> bool {
+    __syncwarp();
+    const int idx = wq[q_head & 7];
+    ++q_head;
+    if (idx < 0) return false;
+    item_set(p, static_cast<uint32_t>(idx), it);
+    item_fill(p, it);
+    return true;
+  };
 
   // ---- issue cursor: SPW pages ahead of the compute cursor
-  Item iss = cmp;
+  Item iss;
+  bool iss_live = take(iss);
   int iss_page = 0;
   int bt_reg = 0;
   uint32_t k_iss = 0;
   int slot_iss = 0;
   auto issue_one = [&]() {
-    while (!item_done(p, iss) && iss_page >= iss.npages) {
-      item_next(p, iss, st);
+    while (iss_live && iss_page >= iss.npages) {
+      iss_live = take(iss);
       iss_page = 0;
     }
-    if (item_done(p, iss)) return;
+    if (!iss_live) return;
     if ((iss_page & 31) == 0) {
       const int j = iss_page + lane;
       bt_reg = j < iss.npages
@@ -228,11 +259,15 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
 
   Math math;
   math.attach(scratch);
+  if constexpr (Math::kTmemCols > 0)
+    math.attach_tmem(*tslot + (static_cast<uint32_t>(32 * warp) << 16));
   uint32_t k_cmp = 0;
   int slot = 0;
   uint32_t phase = 0;
   bool ok = true;
-  while (!item_done(p, cmp)) {
+  Item cmp;
+  bool cmp_live = pop(cmp);
+  while (cmp_live) {
     const int64_t row0 = static_cast<int64_t>(cmp.b) * p.num_q_heads + cmp.kvh * G;
     math.init(p.q + row0 * kD, p.q_scale, lane);
     for (int j = 0; j < cmp.npages; ++j) {
@@ -284,13 +319,22 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
                           p.out, row0 + h, p.out_f32);
       }
     }
-    item_next(p, cmp, st);
+    cmp_live = pop(cmp);
   }
   if (!ok) {
     // A copy never landed: drain the other copies in flight (bounded) and
     // stop.  The sticky status word reports it.
     for (uint32_t k = k_cmp + 1; k < k_iss; ++k)
       mbar_wait(&bars[k % SPW], (k / SPW) & 1, &g_device_status);
+  }
+  if constexpr (Math::kTmemCols > 0) {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(
+                       *tslot),
+                   "r"(Math::kTmemCols)
+                   : "memory");
   }
 }
 
@@ -415,8 +459,9 @@ int launch_group(const DecodeParams& p, const CUtensorMap& tmk,
   // automatic: both products on int8 mma for groups of up to 4 heads
   // (their accumulators fit a warp), the fp16 p.v form for groups of 8
   if constexpr (G <= 4) {
+    // partials in tensor memory leave room for a fourth page slot per warp
     if (variant == KV8_FORM_MMA_I8 || variant == KV8_FORM_AUTO)
-      return launch_decode_kernel<G, 4, 3, I8Math<G>>(p, tmk, tmv, stream);
+      return launch_decode_kernel<G, 4, 4, I8Math<G, true>>(p, tmk, tmv, stream);
   }
   return launch_decode_kernel<G, 4, 3, MmaMath<G>>(p, tmk, tmv, stream);
 }
@@ -465,7 +510,8 @@ size_t workspace_o_bytes(int32_t batch, int32_t num_q_heads,
 }
 
 size_t workspace_ctr_bytes(int32_t batch, int32_t num_q_heads) {
-  return static_cast<size_t>(batch) * num_q_heads * sizeof(uint32_t);
+  // merge tickets, then the work counter (padded to 16 bytes)
+  return static_cast<size_t>(batch) * num_q_heads * sizeof(uint32_t) + 16;
 }
 
 size_t workspace_total_bytes(int32_t batch, int32_t num_q_heads,

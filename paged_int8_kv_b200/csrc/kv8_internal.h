@@ -46,6 +46,8 @@ struct DecodeParams {
   float* ws_o;                  // [B][Hq][max_chunks][128]
   uint32_t* ws_ctr;             // [B][Hq] tickets (index b*Hq + first head
                                 // of the KV group), zero at launch
+  uint32_t* work_ctr;           // items taken past the first wave, zero at
+                                // launch (nullptr: static item order)
   void* out;                    // [B][Hq][128] bf16 or f32
   int32_t batch;
   int32_t num_q_heads;

@@ -95,6 +95,7 @@ template <int G>
 struct SimtMath {
   static constexpr int kWarpsPerSM = 0;  // no register cap
   static constexpr int kScratchBytes = 0;
+  static constexpr int kTmemCols = 0;
   static constexpr int DPL = (G <= 4) ? 16 : 8;  // dims per lane
   static constexpr int LPT = kD / DPL;           // lanes per token
   static constexpr int TPP = 32 / LPT;           // tokens per pass
@@ -105,6 +106,7 @@ struct SimtMath {
   float2 q2[G][DPL / 2];
 
   __device__ __forceinline__ void attach(uint8_t*) {}
+  __device__ __forceinline__ void attach_tmem(uint32_t) {}
   float2 o2[G][DPL / 2];
   float m_run, l_run;
 
@@ -355,6 +357,7 @@ template <int G, bool SharedV = false>
 struct MmaMath {
   static constexpr int kWarpsPerSM = 12;  // cap registers at 168 per thread
   static constexpr int kScratchBytes = 0;
+  static constexpr int kTmemCols = 0;
   static constexpr float kSlack = 8.0f;   // log2 units
   static constexpr int kVSlack = 4;
   int lane, r, c;
@@ -368,6 +371,7 @@ struct MmaMath {
   float fs;         // 2^-e_run
 
   __device__ __forceinline__ void attach(uint8_t*) {}
+  __device__ __forceinline__ void attach_tmem(uint32_t) {}
 
   __device__ __forceinline__ void init(const __nv_bfloat16* qg, float q_scale,
                                        int lane_) {
@@ -651,6 +655,42 @@ struct MmaMath {
   }
 };
 
+// 32 consecutive 32-bit columns of this thread's tensor-memory lane (the
+// warp's lane quarter), loaded / stored and waited for.
+__device__ __forceinline__ void tm_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,"
+      "%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,"
+      "%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
+        "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
+        "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tm_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,"
+      "%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,"
+      "%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]),
+      "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]),
+      "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]), "f"(v[17]),
+      "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]),
+      "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]),
+      "f"(v[30]), "f"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // s8 x u8 integer mma: D[16x8] (s32) += A[16x16] (s8, row) . B[16x8] (u8, col).
 __device__ __forceinline__ void mma16816_s8u8(int (&d)[4], uint32_t a0,
                                               uint32_t a1, uint32_t b0) {
@@ -703,11 +743,15 @@ __device__ __forceinline__ void ldsm_x2_trans_b8(uint32_t addr, uint32_t& r0,
 //   when the references move and at the end of an item.  The two lanes
 //   c and c^2 hold complementary planes of the same outputs and are summed
 //   at the end.
-template <int G>
+// InTmem: the drained fp32 partials live in 32 tensor-memory columns of the
+// warp's lane quarter instead of 4 KB of the warp's shared memory (which is
+// then free for page slots).
+template <int G, bool InTmem = false>
 struct I8Math {
   static_assert(G == 1 || G == 2 || G == 4, "groups of 1, 2 or 4 heads");
   static constexpr int kWarpsPerSM = 12;  // cap registers at 168 per thread
-  static constexpr int kScratchBytes = 32 * 32 * 4;  // fp32 [32][lane]
+  static constexpr int kScratchBytes = InTmem ? 0 : 32 * 32 * 4;  // fp32 [32][lane]
+  static constexpr int kTmemCols = InTmem ? 32 : 0;
   static constexpr float kSlack = 6.0f;   // log2 units
   static constexpr int kVSlack = 2;
   static constexpr int kF = 23;  // P'' < 2^(kSlack + kVSlack): P < 2^31
@@ -720,6 +764,7 @@ struct I8Math {
   float qf;           // score factor of head hr: 2^-sh * softmax_scale * log2(e)
   int acc[8][2][4];   // p.v int32 accumulators: m-tile, n-tile, fragment
   float* of;          // this warp's drained fp32 partials, [32][lane]
+  uint32_t otm;       // ... or their tensor-memory address (InTmem)
   float m_run, l_run;
   int e_run;
   float vlim;         // 2^(e_run + kVSlack)
@@ -731,6 +776,7 @@ struct I8Math {
   __device__ __forceinline__ void attach(uint8_t* scratch) {
     of = reinterpret_cast<float*>(scratch);
   }
+  __device__ __forceinline__ void attach_tmem(uint32_t taddr) { otm = taddr; }
 
   __device__ __forceinline__ void init(const __nv_bfloat16* qg, float q_scale,
                                        int lane_) {
@@ -813,16 +859,36 @@ struct I8Math {
   __device__ __forceinline__ void drain(float aA, float aB) {
     const float w0 = pow2i(8 * (c >> 1) - kF);
     const float w1 = pow2i(16 + 8 * (c >> 1) - kF);
+    if constexpr (InTmem) {
+      float o[32];
+      if (of_live) {
+        tm_ld32(otm, o);
+      } else {
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int k = m * 4 + e;
-        const float v = __int2float_rn(acc[m][0][e]) * w0 +
-                         __int2float_rn(acc[m][1][e]) * w1;
-        const float old = of_live ? of[k * 32 + lane] : 0.0f;
-        of[k * 32 + lane] = (old + v) * ((e & 1) ? aB : aA);
+        for (int k = 0; k < 32; ++k) o[k] = 0.0f;
       }
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int k = m * 4 + e;
+          const float v = __int2float_rn(acc[m][0][e]) * w0 +
+                           __int2float_rn(acc[m][1][e]) * w1;
+          o[k] = (o[k] + v) * ((e & 1) ? aB : aA);
+        }
+      tm_st32(otm, o);
+    } else {
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int k = m * 4 + e;
+          const float v = __int2float_rn(acc[m][0][e]) * w0 +
+                           __int2float_rn(acc[m][1][e]) * w1;
+          const float old = of_live ? of[k * 32 + lane] : 0.0f;
+          of[k * 32 + lane] = (old + v) * ((e & 1) ? aB : aA);
+        }
+    }
     of_live = true;
     zero_acc();
   }
@@ -949,12 +1015,24 @@ struct I8Math {
     const float mB = __shfl_sync(kFull, m_run, 4 * hB);
     const float f = pow2i(e_run);
     const bool wA = c < 2 && nA < G, wB = c < 2 && nB < G;
+    float o[32];
+    if constexpr (InTmem) {
+      if (of_live) {
+        tm_ld32(otm, o);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = 0.0f;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) o[k] = of_live ? of[k * 32 + lane] : 0.0f;
+    }
 #pragma unroll
     for (int m = 0; m < 8; ++m)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int k = m * 4 + e;
-        float v = of_live ? of[k * 32 + lane] : 0.0f;
+        float v = o[k];
         v += __shfl_xor_sync(kFull, v, 2);  // the complementary planes
         const int d = 16 * m + r + ((e & 2) ? 8 : 0);
         if (e & 1) {

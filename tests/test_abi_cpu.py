@@ -54,7 +54,8 @@ def test_workspace_bytes_closed_form():
     ml = 64 * 32 * 64 * 2 * 4          # (m, l) per (sequence, head, chunk)
     o = 64 * 32 * 64 * 128 * 4         # unnormalised output per chunk
     tickets = 64 * 32 * 4              # one merge ticket per (sequence, head)
-    assert ws == ((ml + 255) // 256) * 256 + o + tickets
+    counter = 16                       # the work counter, padded
+    assert ws == ((ml + 255) // 256) * 256 + o + tickets + counter
     assert pk.kv8_decode_workspace_bytes(64, 32, 128, 512, 512) == 0
     assert pk.kv8_decode_workspace_bytes(64, 32, 128, 32768, 0) == 0
     assert pk.kv8_decode_workspace_bytes(64, 32, 64, 32768, 512) == 0
