@@ -35,24 +35,35 @@ def shard_bounds(context_len: int, world: int, rank: int,
     return min(c0 * chunk_tokens, context_len), min(c1 * chunk_tokens, context_len)
 
 
+def max_local_len(context_lens, world: int, chunk_tokens: int) -> int:
+    """The longest part any rank holds of any context: the bound every rank
+    passes as max_context_len, so that their partial layouts match."""
+    return max([e - s for n in context_lens for s, e in
+                (shard_bounds(int(n), world, r, chunk_tokens)
+                 for r in range(world))] + [0])
+
+
 def local_tables(block_tables, context_lens, world: int, rank: int,
                  chunk_tokens: int, block_size: int = 16):
     """A rank's block tables and lengths for its part of every sequence,
     sliced from global (host) tables: row b lists the blocks of tokens
-    [begin_b, end_b).  Returns (tables [B, max_local_blocks], lens [B],
-    max_local_len); works on numpy arrays or CPU tensors."""
+    [begin_b, end_b).  Returns (tables [B, width], lens [B], bound) where
+    bound = max_local_len(...) is the same on every rank and the tables are
+    width = ceil(bound / block_size) wide on every rank (padding entries
+    are never read); works on numpy arrays or CPU tensors."""
     import numpy as np
     bt = np.asarray(block_tables)
     lens = np.asarray(context_lens)
     spans = [shard_bounds(int(n), world, rank, chunk_tokens) for n in lens]
     nblk = [math.ceil((e - s) / block_size) for s, e in spans]
-    width = max(nblk + [1])
+    bound = max_local_len(lens, world, chunk_tokens)
+    width = max(math.ceil(bound / block_size), 1)
     out = np.zeros((bt.shape[0], width), dtype=np.int32)
     for b, (s, e) in enumerate(spans):
         j0 = s // block_size
         out[b, :nblk[b]] = bt[b, j0:j0 + nblk[b]]
     local = np.asarray([e - s for s, e in spans], dtype=np.int32)
-    return out, local, int(local.max()) if local.size else 0
+    return out, local, bound
 
 
 def context_parallel_decode(q: torch.Tensor, k_cache: torch.Tensor,

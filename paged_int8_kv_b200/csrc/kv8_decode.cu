@@ -69,28 +69,33 @@ struct SmemPlan {
 // --------------------------------------------------------------------------
 // The decode kernel.  Persistent: a grid of (SMs x resident CTAs) CTAs of
 // WPC independent warps.  A work item is one (sequence, KV head, context
-// chunk); items are numbered chunk-major, i = (chunk * H_kv + kvh) * B + b,
-// and warp gw of W takes items gw, gw + W, ... (skipping chunks past a
-// sequence's end), so every warp sees a mix of chunk positions.  A warp
-// streams its items' pages through its own SPW-slot ring back to back: the
-// issue cursor runs SPW pages ahead of the compute cursor, across item
-// boundaries, so the ring never drains between chunks.  There are no CTA
-// barriers: each warp writes its chunk's result straight from registers.
+// chunk); items are numbered chunk-major with the KV head fastest (see
+// item_set).  A warp's first item is fixed by its index; after that it takes
+// the next untaken item from a counter (split launches) or steps by the
+// grid's warp count.  A warp streams its items' pages through its own
+// SPW-slot ring back to back: the issue cursor runs SPW pages ahead of the
+// compute cursor, across item boundaries, so the ring never drains between
+// chunks.  There are no CTA barriers in the loop: each warp writes its
+// chunk's result straight from registers.
 // --------------------------------------------------------------------------
 struct Item {
   int b, kvh, chunk, n, tok0, tok1, npages;
 };
 
-// Item idx < max_chunks * H_kv * B (< 2^31), numbered chunk-major:
-// idx = (chunk * H_kv + kvh) * B + b.
+// Item idx < max_chunks * B * H_kv (< 2^31), numbered chunk-major with the
+// KV head fastest: idx = (chunk * B + b) * H_kv + kvh.  Neighbouring warps
+// then stream the same blocks for different KV heads at about the same
+// time, and a block's KV-head pages are contiguous in the cache (H_kv x 2 KB
+// of codes, H_kv x 64 B of scales), so DRAM sees long runs instead of
+// scattered 2 KB pages.
 __device__ __forceinline__ void item_set(const DecodeParams& p, uint32_t idx,
                                          Item& it) {
   const uint32_t per_chunk = static_cast<uint32_t>(p.num_kv_heads) * p.batch;
   const uint32_t c = idx / per_chunk;
   const uint32_t rem = idx - c * per_chunk;
   it.chunk = static_cast<int>(c);
-  it.kvh = static_cast<int>(rem / static_cast<uint32_t>(p.batch));
-  it.b = static_cast<int>(rem - static_cast<uint32_t>(it.kvh) * p.batch);
+  it.b = static_cast<int>(rem / static_cast<uint32_t>(p.num_kv_heads));
+  it.kvh = static_cast<int>(rem - static_cast<uint32_t>(it.b) * p.num_kv_heads);
 }
 
 // Fill in the item's extent; false if the chunk lies past its sequence (a

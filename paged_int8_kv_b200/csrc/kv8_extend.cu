@@ -541,13 +541,18 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
         // P16 is free and O is up to date once the previous O product is done
         if (t >= 1) ewait(&bars[B_O_DONE], (t - 1) & 1, failed);
         tc_fence_after();
-        if (moved && j > 0) {  // rescale this row of O in tensor memory
+        // rescale O in tensor memory where the row's references moved; the
+        // tensor-memory loads and stores are warp-collective, so the whole
+        // warp takes the branch (rows that did not move multiply by 1)
+        const bool rescale = moved && j > 0;
+        if (__any_sync(kFull, rescale)) {
+          const float f = rescale ? a_o : 1.0f;
 #pragma unroll 1
           for (int c = 0; c < kD / 32; ++c) {
             float o[32];
             tmem_ld32(trow + kColO + 32 * c, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= a_o;
+            for (int i = 0; i < 32; ++i) o[i] *= f;
             tmem_st32(trow + kColO + 32 * c, o);
           }
         }

@@ -40,8 +40,7 @@ def test_context_parallel_matches_oracle(pk, oracle_mod, ranks, chunk):
     w = W.make_workload("cp", 8000 + ranks, lens, 32, 8, extra_blocks=3,
                         outliers=(3, 10.0))
     cache, q, bt, cl = U.device_inputs(w)
-    maxl = max(CP.local_tables(w.block_tables, w.context_lens, ranks, r, chunk)[2]
-               for r in range(ranks))
+    maxl = CP.max_local_len(w.context_lens, ranks, chunk)
     nbytes = pk.kv8_decode_partials_bytes(w.batch, w.num_q_heads, 128, maxl, chunk)
     stride = (nbytes + 255) // 256 * 256
     allp = torch.full((ranks * stride,), 0xFF, dtype=torch.uint8, device="cuda")
