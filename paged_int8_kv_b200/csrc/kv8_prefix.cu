@@ -35,19 +35,23 @@ __device__ uint32_t g_prefix_status = 0;
 
 namespace {
 
-constexpr int kPW = 8;    // warps per CTA = members per round
-constexpr int kPNB = 4;   // page slots in the CTA's ring
+constexpr int kPW = 8;     // warps per CTA = members per round
+constexpr int kPNB = 12;   // page slots in the CTA's ring (one CTA per SM:
+                           // 11 pages in flight)
 constexpr uint32_t kPTx = 2 * kPageBytes + 2 * kBS * sizeof(float);
 
 // Shared memory (base aligned to 1024 bytes for the 128-byte swizzle):
 //   [kPNB][K page 2048 | V page 2048]   TMA-staged int8 pages
-//   [kPNB][4096]                        V page as fp16 [16 tok][128 dims]
+//   [2][4096]                           V page as fp16 [16 tok][128 dims], by
+//                                       page parity (page k's copy is free
+//                                       once every warp is past page k+1's
+//                                       barrier)
 //   [kPNB][ks 64 | vs 64]               scales
 //   [kPNB] mbarriers; two ints: a wait gave up, the first page not waited for
 struct PrefixPlan {
   static constexpr int kTiles = 0;
   static constexpr int kVh = kTiles + kPNB * 2 * kPageBytes;
-  static constexpr int kScl = kVh + kPNB * 4096;
+  static constexpr int kScl = kVh + 2 * 4096;
   static constexpr int kBar = kScl + kPNB * 2 * kBS * 4;
   static constexpr int kFail = kBar + kPNB * 8;
   static constexpr int kBytes = kFail + 16 + 1024;
@@ -233,7 +237,7 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
         o.z = hsub2_u32(prmt(x1, 0x64646464u, 0x4140u), kBias1152);
         o.w = hsub2_u32(prmt(x1, 0x64646464u, 0x4342u), kBias1152);
         const int ch = 2 * cj + hf;  // fp16 chunk: dims 8ch .. 8ch+7
-        *reinterpret_cast<uint4*>(vh + s * 4096 + t * 256 + ((ch ^ (t & 7)) << 4)) = o;
+        *reinterpret_cast<uint4*>(vh + (k & 1) * 4096 + t * 256 + ((ch ^ (t & 7)) << 4)) = o;
       }
       __syncthreads();
       // every warp is past page k-1: its slot is free for page k-1+kPNB
@@ -243,7 +247,7 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
         const float* ks = scl + s * 2 * kBS;
         uint32_t h0, h2, g0, g2;
         math.template qk_softmax<true>(tk, ks, ks + kBS, kBS, h0, h2, g0, g2);
-        math.pv_f16(smem_u32(vh + s * 4096), h0, h2, g0, g2);
+        math.pv_f16(smem_u32(vh + (k & 1) * 4096), h0, h2, g0, g2);
       }
     }
     if (b_w < 0) continue;
