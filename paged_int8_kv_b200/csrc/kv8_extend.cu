@@ -538,6 +538,19 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
           moved = true;
         }
         const float mu = m_run == -INFINITY ? 0.0f : m_run;
+        // probabilities first (packed fp16 in registers), so that the
+        // exponentials overlap the previous O product on the tensor cores
+        uint32_t ph[kKT / 2];
+        float lsum = 0.0f;
+#pragma unroll
+        for (int c = 0; c < kKT / 2; ++c) {
+          const float p0 = ex2(sv[2 * c] - mu), p1 = ex2(sv[2 * c + 1] - mu);
+          lsum += p0 + p1;
+          const float v0 = sv[2 * c] == -INFINITY ? 0.0f : vs[2 * c];
+          const float v1 = sv[2 * c + 1] == -INFINITY ? 0.0f : vs[2 * c + 1];
+          const __half2 hv = __floats2half2_rn(p0 * (v0 * fs), p1 * (v1 * fs));
+          ph[c] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
         // P16 is free and O is up to date once the previous O product is done
         if (t >= 1) ewait(&bars[B_O_DONE], (t - 1) & 1, failed);
         tc_fence_after();
@@ -556,22 +569,10 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
             tmem_st32(trow + kColO + 32 * c, o);
           }
         }
-        float lsum = 0.0f;
 #pragma unroll
-        for (int c = 0; c < kKT / 8; ++c) {
-          uint32_t h[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int c0 = 8 * c + 2 * k;
-            const float p0 = ex2(sv[c0] - mu), p1 = ex2(sv[c0 + 1] - mu);
-            lsum += p0 + p1;
-            const float v0 = sv[c0] == -INFINITY ? 0.0f : vs[c0];
-            const float v1 = sv[c0 + 1] == -INFINITY ? 0.0f : vs[c0 + 1];
-            const __half2 hv = __floats2half2_rn(p0 * (v0 * fs), p1 * (v1 * fs));
-            h[k] = *reinterpret_cast<const uint32_t*>(&hv);
-          }
-          *reinterpret_cast<uint4*>(p16 + op_off(r, c)) = make_uint4(h[0], h[1], h[2], h[3]);
-        }
+        for (int c = 0; c < kKT / 8; ++c)
+          *reinterpret_cast<uint4*>(p16 + op_off(r, c)) =
+              make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
         l_run += lsum;
         fence_proxy_async_smem();
         tc_fence_before();
