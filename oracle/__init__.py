@@ -58,6 +58,11 @@ def _load():
     lib.oracle_extend_attention.restype = ctypes.c_int
     lib.oracle_extend_attention.argtypes = [
         P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, f64, P]
+    lib.oracle_quantize_append_int4.restype = ctypes.c_int
+    lib.oracle_quantize_append_int4.argtypes = [P, P, i64, i32, i32, i32, i64, P, P]
+    lib.oracle_decode_attention_int4.restype = ctypes.c_int
+    lib.oracle_decode_attention_int4.argtypes = [
+        P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, f64, P]
     lib.oracle_kv_cache_bytes.restype = f64
     lib.oracle_kv_cache_bytes.argtypes = [i64] * 7
     lib.oracle_kv8_scale_bytes.restype = f64
@@ -163,6 +168,45 @@ def extend_attention(q_bf16: np.ndarray, k_cache: np.ndarray,
         _ptr(bt), _ptr(cl), _ptr(qs), B, hq, hkv, d, bs, bt.shape[1], nb,
         float(softmax_scale), _ptr(out))
     _check(rc, "oracle_extend_attention")
+    return out
+
+
+def quantize_append_int4(x_bf16: np.ndarray, slot_mapping: np.ndarray,
+                         cache: np.ndarray, scales: np.ndarray) -> None:
+    """INT4 variant: quantise x (uint16 bf16 bits, [n, H_kv, D]) into cache
+    (uint8 [NB, H_kv, BS, D/2], excess-8 nibbles) and scales (float32
+    [NB, H_kv, BS]) in place."""
+    lib = _load()
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    assert cache.dtype == np.uint8 and cache.flags.c_contiguous
+    assert scales.dtype == np.float32 and scales.flags.c_contiguous
+    nb, hkv, bs, dh = cache.shape
+    assert x.shape[1:] == (hkv, 2 * dh) and sm.shape == (x.shape[0],)
+    rc = lib.oracle_quantize_append_int4(_ptr(x), _ptr(sm), x.shape[0], hkv,
+                                         2 * dh, bs, nb, _ptr(cache), _ptr(scales))
+    _check(rc, "oracle_quantize_append_int4")
+
+
+def decode_attention_int4(q_bf16: np.ndarray, k_cache: np.ndarray,
+                          v_cache: np.ndarray, k_scales: np.ndarray,
+                          v_scales: np.ndarray, block_tables: np.ndarray,
+                          context_lens: np.ndarray,
+                          softmax_scale: float = 0.0) -> np.ndarray:
+    """fp64 decode attention over the dequantised INT4 cache; [B, H_q, D]."""
+    lib = _load()
+    q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    B, hq, d = q.shape
+    nb, hkv, bs, dh = k_cache.shape
+    assert 2 * dh == d and v_cache.shape == k_cache.shape
+    out = np.zeros((B, hq, d), dtype=np.float64)
+    rc = lib.oracle_decode_attention_int4(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales),
+        _ptr(bt), _ptr(cl), B, hq, hkv, d, bs, bt.shape[1], nb,
+        float(softmax_scale), _ptr(out))
+    _check(rc, "oracle_decode_attention_int4")
     return out
 
 

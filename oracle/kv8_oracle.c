@@ -121,13 +121,30 @@ int oracle_quantize_append(const uint16_t *x, const int64_t *slot_mapping,
  * paged cache (KV head kvh), fp64.  out_row receives head_dim doubles; n == 0
  * gives a zero row.
  */
-static int attend_row(const uint16_t *qrow, const int8_t *k_cache,
-                      const int8_t *v_cache, const float *k_scales,
-                      const float *v_scales, const int32_t *block_tables,
-                      int32_t num_kv_heads, int32_t head_dim,
-                      int32_t block_size, int32_t max_blocks_per_seq,
-                      int64_t num_blocks, double softmax_scale, int32_t b,
-                      int32_t kvh, int32_t n, double *out_row)
+/*
+ * Code j of the cache row starting at row index `base` (row = one token of
+ * one KV head): an int8 code (bits == 8), or the nibble of an INT4 row
+ * (bits == 4; head_dim / 2 bytes per row, dims 2i / 2i+1 in the low / high
+ * nibble of byte i, stored as code + 8).
+ */
+static int code_at(const void *cache, int64_t base, int32_t head_dim,
+                   int32_t bits, int32_t j)
+{
+    if (bits == 8)
+        return ((const int8_t *)cache)[base * head_dim + j];
+    uint8_t byte = ((const uint8_t *)cache)[base * (head_dim / 2) + j / 2];
+    int nib = (j & 1) ? (byte >> 4) : (byte & 15);
+    return nib - 8;
+}
+
+static int attend_row_bits(const uint16_t *qrow, const void *k_cache,
+                           const void *v_cache, const float *k_scales,
+                           const float *v_scales, const int32_t *block_tables,
+                           int32_t num_kv_heads, int32_t head_dim,
+                           int32_t block_size, int32_t max_blocks_per_seq,
+                           int64_t num_blocks, double softmax_scale, int32_t b,
+                           int32_t kvh, int32_t n, int32_t bits,
+                           double *out_row)
 {
     for (int32_t j = 0; j < head_dim; ++j)
         out_row[j] = 0.0;
@@ -151,10 +168,10 @@ static int attend_row(const uint16_t *qrow, const int8_t *k_cache,
         }
         int64_t base = (phys * num_kv_heads + kvh) * (int64_t)block_size + off;
         double ks = (double)k_scales[base];
-        const int8_t *kc = k_cache + base * head_dim;
         double dot = 0.0;
         for (int32_t j = 0; j < head_dim; ++j)
-            dot += (double)bf16_bits_to_float(qrow[j]) * ((double)kc[j] * ks);
+            dot += (double)bf16_bits_to_float(qrow[j]) *
+                   ((double)code_at(k_cache, base, head_dim, bits, j) * ks);
         score[t] = softmax_scale * dot;
         if (score[t] > smax)
             smax = score[t];
@@ -170,16 +187,29 @@ static int attend_row(const uint16_t *qrow, const int8_t *k_cache,
         int64_t off = t % block_size;
         int64_t base = (phys * num_kv_heads + kvh) * (int64_t)block_size + off;
         double vs = (double)v_scales[base];
-        const int8_t *vc = v_cache + base * head_dim;
         double w = score[t] / denom;
         for (int32_t j = 0; j < head_dim; ++j)
-            out_row[j] += w * ((double)vc[j] * vs);
+            out_row[j] += w * ((double)code_at(v_cache, base, head_dim, bits, j) * vs);
     }
     free(score);
     for (int32_t j = 0; j < head_dim; ++j)
         if (!isfinite(out_row[j]))
             return ORACLE_NONFINITE;
     return ORACLE_OK;
+}
+
+static int attend_row(const uint16_t *qrow, const int8_t *k_cache,
+                      const int8_t *v_cache, const float *k_scales,
+                      const float *v_scales, const int32_t *block_tables,
+                      int32_t num_kv_heads, int32_t head_dim,
+                      int32_t block_size, int32_t max_blocks_per_seq,
+                      int64_t num_blocks, double softmax_scale, int32_t b,
+                      int32_t kvh, int32_t n, double *out_row)
+{
+    return attend_row_bits(qrow, k_cache, v_cache, k_scales, v_scales,
+                           block_tables, num_kv_heads, head_dim, block_size,
+                           max_blocks_per_seq, num_blocks, softmax_scale, b,
+                           kvh, n, 8, out_row);
 }
 
 /*
@@ -298,6 +328,106 @@ int oracle_extend_attention(const uint16_t *q, const int8_t *k_cache,
             }
         }
     }
+    return ORACLE_OK;
+}
+
+/*
+ * INT4 variant of the cache.  The K/V of historical tokens are quantised to
+ * 4 bits [nano-KvLLM, §2.2 量化感知缓存]; INT4 takes 0.5 byte per element
+ * [KV Cache 优化全景解析, §2.3 table].  Readings (the pages give no formula):
+ * the same symmetric per-(token, KV head) scheme as INT8 with 7 levels each
+ * side, s = fl32(max|x| / 7) (IEEE division; s = 0 for an all-zero row),
+ * c_j = clamp(rint(fl32(x_j / s)), -7, 7) (ties to even; 0 when s == 0).
+ * Storage: the nibble c_j + 8 (1..15; 8 for a zero row), dims 2i and 2i+1
+ * in the low and high nibble of byte i; cache [num_blocks][H_kv][BS][D/2]
+ * bytes, scales [num_blocks][H_kv][BS] fp32.
+ */
+int oracle_quantize_append_int4(const uint16_t *x, const int64_t *slot_mapping,
+                                int64_t n_tokens, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t block_size,
+                                int64_t num_blocks, uint8_t *cache,
+                                float *scales)
+{
+    if (n_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || (head_dim & 1))
+        return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < n_tokens; ++i) {
+        int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        int64_t blk = slot / block_size;
+        int64_t off = slot % block_size;
+        if (blk >= num_blocks)
+            return ORACLE_BAD_ARG;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            const uint16_t *row = x + (i * num_kv_heads + h) * (int64_t)head_dim;
+            float a = 0.0f;
+            for (int32_t j = 0; j < head_dim; ++j) {
+                float v = bf16_bits_to_float(row[j]);
+                if (!isfinite(v))
+                    return ORACLE_NONFINITE;
+                float m = fabsf(v);
+                if (m > a)
+                    a = m;
+            }
+            float s = (a == 0.0f) ? 0.0f : a / 7.0f;
+            int64_t base = (blk * num_kv_heads + h) * (int64_t)block_size + off;
+            uint8_t *dst = cache + base * (head_dim / 2);
+            for (int32_t j = 0; j < head_dim; j += 2) {
+                int nib[2];
+                for (int k = 0; k < 2; ++k) {
+                    int code = 0;
+                    if (s != 0.0f) {
+                        float y = bf16_bits_to_float(row[j + k]) / s;
+                        float r = nearbyintf(y);
+                        if (r > 7.0f)
+                            r = 7.0f;
+                        if (r < -7.0f)
+                            r = -7.0f;
+                        code = (int)r;
+                    }
+                    nib[k] = code + 8;
+                }
+                dst[j / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
+            }
+            scales[base] = s;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Decode attention over the INT4 cache, fp64: as oracle_decode_attention,
+ * with k_hat = (nibble - 8) * ks and v_hat = (nibble - 8) * vs.
+ */
+int oracle_decode_attention_int4(const uint16_t *q, const uint8_t *k_cache,
+                                 const uint8_t *v_cache, const float *k_scales,
+                                 const float *v_scales,
+                                 const int32_t *block_tables,
+                                 const int32_t *context_lens, int32_t batch,
+                                 int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t block_size,
+                                 int32_t max_blocks_per_seq, int64_t num_blocks,
+                                 double softmax_scale, double *out)
+{
+    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_q_heads % num_kv_heads != 0 || (head_dim & 1))
+        return ORACLE_BAD_ARG;
+    if (softmax_scale <= 0.0)
+        softmax_scale = 1.0 / sqrt((double)head_dim);
+    int32_t group = num_q_heads / num_kv_heads;
+    for (int32_t b = 0; b < batch; ++b)
+        for (int32_t h = 0; h < num_q_heads; ++h) {
+            const uint16_t *qrow = q + ((int64_t)b * num_q_heads + h) * head_dim;
+            int rc = attend_row_bits(qrow, k_cache, v_cache, k_scales, v_scales,
+                                     block_tables, num_kv_heads, head_dim,
+                                     block_size, max_blocks_per_seq, num_blocks,
+                                     softmax_scale, b, h / group,
+                                     context_lens[b], 4,
+                                     out + ((int64_t)b * num_q_heads + h) * head_dim);
+            if (rc != ORACLE_OK)
+                return rc;
+        }
     return ORACLE_OK;
 }
 
