@@ -423,6 +423,49 @@ KV8_API int32_t kv8_paged_decode_attention_noalloc(
     float softmax_scale, int32_t chunk_tokens, void *out, int32_t out_dtype,
     void *stream);
 
+/*
+ * The INT4 variant of the cache.
+ *
+ * Historical tokens' K and V may be kept in 4 bits [nano-KvLLM, §2.2
+ * 量化感知缓存], half a byte per element [KV Cache 优化全景解析, §2.3
+ * table]; the pages give no formula, so the INT8 scheme carries over with 7
+ * levels each side of zero, per (token, KV head):
+ *     s = fl32(max_j |x_j| / 7) (IEEE division; s = 0 for an all-zero row)
+ *     c_j = clamp(rint(fl32(x_j / s)), -7, 7), ties to even; 0 when s == 0
+ * stored as the nibble c_j + 8, dims 2i and 2i+1 in the low and high nibble
+ * of byte i.  Layout: k_cache / v_cache uint8 [num_blocks][num_kv_heads]
+ * [block_size][head_dim / 2] (64 bytes a token, 1 KB a page), k_scales /
+ * v_scales fp32 [num_blocks][num_kv_heads][block_size].
+ *
+ * kv8_int4_quantize_append -- kv8_quantize_append into the INT4 cache (same
+ * arguments, same rules on slots and padding).
+ */
+KV8_API int32_t kv8_int4_quantize_append(const void *k_new, const void *v_new,
+                                         const int64_t *slot_mapping,
+                                         int64_t n_tokens, int32_t num_kv_heads,
+                                         int32_t head_dim, int32_t block_size,
+                                         int64_t num_blocks, uint8_t *k_cache,
+                                         uint8_t *v_cache, float *k_scales,
+                                         float *v_scales, void *stream);
+
+/*
+ * kv8_int4_paged_decode_attention -- kv8_paged_decode_attention over the
+ * INT4 cache: k_hat = c * ks, v_hat = c * vs with c = nibble - 8.  Same
+ * arguments, workspace (kv8_decode_workspace_bytes), split and status codes;
+ * groups of 1, 2 or 4 query heads per KV head (a larger group returns
+ * KV8_ERR_UNSUPPORTED).  Both products run on the warp tensor cores with
+ * the nibbles as unsigned 8-bit operands; the +8 bias is removed exactly in
+ * integer arithmetic.
+ */
+KV8_API int32_t kv8_int4_paged_decode_attention(
+    const void *q, const uint8_t *k_cache, const uint8_t *v_cache,
+    const float *k_scales, const float *v_scales, const int32_t *block_tables,
+    const int32_t *context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void *workspace,
+    size_t workspace_bytes, void *out, int32_t out_dtype, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -45,6 +45,8 @@ EXPORTED = (
     "kv8_merge_partials",
     "kv8_read_device_status",
     "kv8_paged_decode_attention_noalloc",
+    "kv8_int4_quantize_append",
+    "kv8_int4_paged_decode_attention",
 )
 
 
@@ -101,6 +103,12 @@ def _load() -> ctypes.CDLL:
     lib.kv8_paged_decode_attention_noalloc.argtypes = [
         P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
         P, i32, P]
+    lib.kv8_int4_quantize_append.restype = i32
+    lib.kv8_int4_quantize_append.argtypes = [P, P, P, i64, i32, i32, i32, i64, P, P, P, P, P]
+    lib.kv8_int4_paged_decode_attention.restype = i32
+    lib.kv8_int4_paged_decode_attention.argtypes = [
+        P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
+        P, sz, P, i32, P]
     lib.kv8_read_device_status.restype = i32
     lib.kv8_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
     return lib
@@ -140,6 +148,19 @@ def kv8_quantize_append(k_new: torch.Tensor, v_new: torch.Tensor,
     _check("kv8_quantize_append", lib.kv8_quantize_append(
         _p(k_new), _p(v_new), _p(slot_mapping), slot_mapping.shape[0], hkv, d,
         bs, nb, _p(k_cache), _p(v_cache), _p(k_scales), _p(v_scales),
+        _stream(stream)))
+
+
+def kv8_int4_quantize_append(k_new: torch.Tensor, v_new: torch.Tensor,
+                             slot_mapping: torch.Tensor, k_cache: torch.Tensor,
+                             v_cache: torch.Tensor, k_scales: torch.Tensor,
+                             v_scales: torch.Tensor, stream=None) -> None:
+    """INT4 cache: k_new/v_new bf16 [n, H_kv, D]; caches uint8
+    [NB, H_kv, 16, D/2] (packed excess-8 nibbles); scales fp32 [NB, H_kv, 16]."""
+    nb, hkv, bs, dh = k_cache.shape
+    _check("kv8_int4_quantize_append", lib.kv8_int4_quantize_append(
+        _p(k_new), _p(v_new), _p(slot_mapping), slot_mapping.shape[0], hkv,
+        2 * dh, bs, nb, _p(k_cache), _p(v_cache), _p(k_scales), _p(v_scales),
         _stream(stream)))
 
 
@@ -205,6 +226,27 @@ def kv8_paged_decode_attention_form(q: torch.Tensor, k_cache: torch.Tensor,
                              block_tables, context_lens, out, max_context_len,
                              chunk_tokens, workspace, softmax_scale),
                int(form), _stream(stream)))
+    return out
+
+
+def kv8_int4_paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor,
+                                    v_cache: torch.Tensor,
+                                    k_scales: torch.Tensor,
+                                    v_scales: torch.Tensor,
+                                    block_tables: torch.Tensor,
+                                    context_lens: torch.Tensor,
+                                    out: torch.Tensor, max_context_len: int,
+                                    chunk_tokens: int = 512,
+                                    workspace: torch.Tensor | None = None,
+                                    softmax_scale: float = 0.0,
+                                    stream=None) -> torch.Tensor:
+    """Decode attention over the INT4 cache (uint8 [NB, H_kv, 16, D/2])."""
+    _check("kv8_int4_paged_decode_attention",
+           lib.kv8_int4_paged_decode_attention(
+               *_decode_args(q, k_cache, v_cache, k_scales, v_scales,
+                             block_tables, context_lens, out, max_context_len,
+                             chunk_tokens, workspace, softmax_scale),
+               _stream(stream)))
     return out
 
 

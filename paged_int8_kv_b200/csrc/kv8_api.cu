@@ -39,22 +39,26 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Tensor map over a code cache viewed as [num_blocks*H_kv pages][16 rows]
+// Tensor map over a code cache viewed as [num_blocks*H_kv pages][rows]
 // [128 bytes]: one box is one page, written to shared memory with the
 // 128-byte swizzle (16-byte chunk j of row r lands at chunk j ^ (r & 7)).
-bool encode_page_map(CUtensorMap* map, const int8_t* cache, int64_t pages) {
+// INT8 codes: 16 rows, one token each.  Packed INT4 codes (64 bytes a
+// token): 8 rows, tokens 2r and 2r+1 in row r.
+bool encode_page_map(CUtensorMap* map, const void* cache, int64_t pages,
+                     int bits = 8) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const int rows = bits == 4 ? kBlockSize / 2 : kBlockSize;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim),
-                        static_cast<cuuint64_t>(kBlockSize),
+                        static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(pages)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim),
-                           static_cast<cuuint64_t>(kHeadDim * kBlockSize)};
+                           static_cast<cuuint64_t>(kHeadDim * rows)};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(kHeadDim),
-                       static_cast<cuuint32_t>(kBlockSize), 1};
+                       static_cast<cuuint32_t>(rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
-                  const_cast<int8_t*>(cache), dims, strides, box, estr,
+                  const_cast<void*>(cache), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -92,7 +96,7 @@ int32_t prepare_decode(
     int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
     float softmax_scale, int32_t chunk_tokens, void* workspace,
     size_t workspace_bytes, void* out, int32_t out_dtype, DecodeSetup* d,
-    bool partials_only = false) {
+    bool partials_only = false, int bits = 8) {
   // ---- shape checks
   if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 ||
@@ -146,8 +150,8 @@ int32_t prepare_decode(
   }
 
   const int64_t pages = num_blocks * num_kv_heads;
-  if (!encode_page_map(&d->tmk, k_cache, pages) ||
-      !encode_page_map(&d->tmv, v_cache, pages))
+  if (!encode_page_map(&d->tmk, k_cache, pages, bits) ||
+      !encode_page_map(&d->tmv, v_cache, pages, bits))
     return KV8_ERR_CUDA;
 
   if (!(softmax_scale > 0.0f))
@@ -501,6 +505,62 @@ int32_t kv8_test_skip_first_copy(int32_t on) {
 int32_t kv8_read_device_status(uint32_t* status, int32_t clear) {
   if (!status) return KV8_ERR_INVALID_ARG;
   return kv8::read_device_status(status, clear) == 0 ? KV8_OK : KV8_ERR_CUDA;
+}
+
+int32_t kv8_int4_quantize_append(const void* k_new, const void* v_new,
+                                 const int64_t* slot_mapping, int64_t n_tokens,
+                                 int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t block_size, int64_t num_blocks,
+                                 uint8_t* k_cache, uint8_t* v_cache,
+                                 float* k_scales, float* v_scales,
+                                 void* stream) {
+  if (n_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      num_blocks <= 0)
+    return KV8_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim || block_size != kBlockSize)
+    return KV8_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return KV8_OK;
+  if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache || !k_scales ||
+      !v_scales)
+    return KV8_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned4(k_scales) || !aligned4(v_scales) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return KV8_ERR_INVALID_ARG;
+  if (n_tokens > (int64_t(1) << 40) / num_kv_heads) return KV8_ERR_UNSUPPORTED;
+  int rc = kv8::launch_quantize_append(
+      k_new, v_new, slot_mapping, n_tokens, num_kv_heads,
+      reinterpret_cast<int8_t*>(k_cache), reinterpret_cast<int8_t*>(v_cache),
+      k_scales, v_scales, static_cast<cudaStream_t>(stream), 4);
+  return rc == 0 ? KV8_OK : KV8_ERR_CUDA;
+}
+
+int32_t kv8_int4_paged_decode_attention(
+    const void* q, const uint8_t* k_cache, const uint8_t* v_cache,
+    const float* k_scales, const float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float softmax_scale, int32_t chunk_tokens, void* workspace,
+    size_t workspace_bytes, void* out, int32_t out_dtype, void* stream) {
+  if (num_kv_heads > 0 && num_q_heads > 0 && num_q_heads % num_kv_heads == 0 &&
+      num_q_heads / num_kv_heads > 4)
+    return KV8_ERR_UNSUPPORTED;
+  DecodeSetup d;
+  const int32_t rc0 = prepare_decode(
+      q, reinterpret_cast<const int8_t*>(k_cache),
+      reinterpret_cast<const int8_t*>(v_cache), k_scales, v_scales,
+      block_tables, context_lens, batch, num_q_heads, num_kv_heads, head_dim,
+      block_size, max_blocks_per_seq, num_blocks, max_context_len,
+      softmax_scale, chunk_tokens, workspace, workspace_bytes, out, out_dtype,
+      &d, false, 4);
+  if (rc0 != KV8_OK || d.nothing) return rc0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!clear_tickets(d, batch, num_q_heads, st)) return KV8_ERR_CUDA;
+  const int rc = kv8::launch_decode_int4(d.p, d.tmk, d.tmv, st);
+  if (rc == -2) return KV8_ERR_UNSUPPORTED;
+  if (rc != 0) return KV8_ERR_CUDA;
+  return KV8_OK;
 }
 
 }  // extern "C"

@@ -46,19 +46,18 @@ __device__ int g_test_skip_first_copy = 0;
 
 namespace {
 
-constexpr uint32_t kPageTx = 2 * kPageBytes + 2 * kBS * sizeof(float);
-
 // --------------------------------------------------------------------------
 // Shared-memory plan of a decode CTA of WPC independent warps (base aligned
 // to 1024 bytes):
-//   per warp w: SPW slots of [K page 2048 B | V page 2048 B]   (tiles)
+//   per warp w: SPW slots of [K page | V page]   (tiles; CodeBytes each:
+//               2048 for INT8 codes, 1024 for packed INT4 codes)
 //   per warp w: SPW slots of [ks 64 B | vs 64 B]              (scales)
 //   per warp w: the page math's scratch (ScratchBytes, may be 0)
 //   per warp w: SPW mbarriers
 // --------------------------------------------------------------------------
-template <int WPC, int SPW, int ScratchBytes = 0>
+template <int WPC, int SPW, int ScratchBytes = 0, int CodeBytes = kPageBytes>
 struct SmemPlan {
-  static constexpr int kTileBytes = WPC * SPW * 2 * kPageBytes;
+  static constexpr int kTileBytes = WPC * SPW * 2 * CodeBytes;
   static constexpr int kScaleBytes = WPC * SPW * 2 * kBS * 4;
   static constexpr int kScratchBytes = WPC * ScratchBytes;
   static constexpr int kBarBytes = WPC * (SPW * 8 + 32);  // + work queue
@@ -124,13 +123,15 @@ __global__ void __launch_bounds__(WPC * 32,
                                   Math::kWarpsPerSM / WPC > 0 ? Math::kWarpsPerSM / WPC : 1)
 decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
               const __grid_constant__ CUtensorMap tmv) {
-  using Plan = SmemPlan<WPC, SPW, Math::kScratchBytes>;
+  using Plan = SmemPlan<WPC, SPW, Math::kScratchBytes, Math::kCodeBytes>;
+  constexpr int kCB = Math::kCodeBytes;
+  constexpr uint32_t kPageTx = 2 * kCB + 2 * kBS * sizeof(float);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  uint8_t* tiles = smem + warp * SPW * 2 * kPageBytes;
+  uint8_t* tiles = smem + warp * SPW * 2 * kCB;
   float* scl = reinterpret_cast<float*>(smem + Plan::kTileBytes) +
                warp * SPW * 2 * kBS;
   uint8_t* scratch =
@@ -246,9 +247,9 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     if (lane == 0 && issue_copies) {
       const int s = slot_iss;
       const int page = blk * p.num_kv_heads + iss.kvh;
-      uint8_t* tk = tiles + s * 2 * kPageBytes;
+      uint8_t* tk = tiles + s * 2 * kCB;
       tma_load_3d(tk, &tmk, 0, 0, page, &bars[s]);
-      tma_load_3d(tk + kPageBytes, &tmv, 0, 0, page, &bars[s]);
+      tma_load_3d(tk + kCB, &tmv, 0, 0, page, &bars[s]);
       float* sc = scl + s * 2 * kBS;
       bulk_g2s(sc, p.k_scales + static_cast<int64_t>(page) * kBS,
                kBS * sizeof(float), &bars[s]);
@@ -280,13 +281,13 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
         ok = false;
         break;
       }
-      const uint8_t* tk = tiles + slot * 2 * kPageBytes;
+      const uint8_t* tk = tiles + slot * 2 * kCB;
       const float* ks = scl + slot * 2 * kBS;
       const int nv = cmp.tok1 - (cmp.tok0 + j * kBS);
       if (nv >= kBS)
-        math.template page<true>(tk, tk + kPageBytes, ks, ks + kBS, kBS);
+        math.template page<true>(tk, tk + kCB, ks, ks + kBS, kBS);
       else
-        math.template page<false>(tk, tk + kPageBytes, ks, ks + kBS, nv);
+        math.template page<false>(tk, tk + kCB, ks, ks + kBS, nv);
       __syncwarp();
       issue_one();
       ++k_cmp;
@@ -418,7 +419,8 @@ template <int G, int WPC, int SPW, class Math>
 int launch_decode_kernel(const DecodeParams& p, const CUtensorMap& tmk,
                          const CUtensorMap& tmv, cudaStream_t stream) {
   auto kern = decode_kernel<G, WPC, SPW, Math>;
-  constexpr int smem = SmemPlan<WPC, SPW, Math::kScratchBytes>::kBytes;
+  constexpr int smem =
+      SmemPlan<WPC, SPW, Math::kScratchBytes, Math::kCodeBytes>::kBytes;
   static LaunchFacts table[kMaxDevices];  // per device, this instantiation
   LaunchFacts* f = facts_for_current_device(table);
   if (!f) return -1;
@@ -469,6 +471,14 @@ int launch_group(const DecodeParams& p, const CUtensorMap& tmk,
       return launch_decode_kernel<G, 4, 4, I8Math<G, true>>(p, tmk, tmv, stream);
   }
   return launch_decode_kernel<G, 4, 3, MmaMath<G>>(p, tmk, tmv, stream);
+}
+
+// INT4 cache: 1 KB pages, so twice the slots of the INT8 form for the same
+// bytes in flight per warp
+template <int G>
+int launch_group_int4(const DecodeParams& p, const CUtensorMap& tmk,
+                      const CUtensorMap& tmv, cudaStream_t stream) {
+  return launch_decode_kernel<G, 4, 8, I4Math<G>>(p, tmk, tmv, stream);
 }
 
 }  // namespace
@@ -535,6 +545,17 @@ int launch_decode(const DecodeParams& p, const CUtensorMap& tmk,
     case 2: return launch_group<2>(p, tmk, tmv, variant, stream);
     case 4: return launch_group<4>(p, tmk, tmv, variant, stream);
     case 8: return launch_group<8>(p, tmk, tmv, variant, stream);
+    default: return -2;
+  }
+}
+
+int launch_decode_int4(const DecodeParams& p, const CUtensorMap& tmk,
+                       const CUtensorMap& tmv, cudaStream_t stream) {
+  const int g = p.num_q_heads / p.num_kv_heads;
+  switch (g) {
+    case 1: return launch_group_int4<1>(p, tmk, tmv, stream);
+    case 2: return launch_group_int4<2>(p, tmk, tmv, stream);
+    case 4: return launch_group_int4<4>(p, tmk, tmv, stream);
     default: return -2;
   }
 }

@@ -93,17 +93,23 @@ int launch_merge_ranks(const uint8_t* partials, size_t rank_stride,
                        int32_t max_chunks, void* out, int32_t out_f32,
                        cudaStream_t stream);
 
+// bits = 8: int8 codes; bits = 4: the INT4 variant (excess-8 nibbles).
 int launch_quantize_append(const void* k_new, const void* v_new,
                            const int64_t* slot_mapping, int64_t n_tokens,
                            int32_t num_kv_heads, int8_t* k_cache,
                            int8_t* v_cache, float* k_scales, float* v_scales,
-                           cudaStream_t stream);
+                           cudaStream_t stream, int32_t bits = 8);
 
 // Returns 0 on success, -1 on a CUDA error, -2 if the group size has no
 // compiled kernel.
 int launch_decode(const DecodeParams& p, const CUtensorMap& tmk,
                   const CUtensorMap& tmv, int32_t variant,
                   cudaStream_t stream);
+
+// The INT4 cache (packed excess-8 nibbles, 1 KB pages): groups of 1, 2, 4.
+// Same return codes as launch_decode.
+int launch_decode_int4(const DecodeParams& p, const CUtensorMap& tmk,
+                       const CUtensorMap& tmv, cudaStream_t stream);
 
 int launch_split_reduce(const float* ws_ml, const float* ws_o,
                         const int32_t* context_lens, int32_t batch,

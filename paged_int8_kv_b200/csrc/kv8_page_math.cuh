@@ -96,6 +96,7 @@ struct SimtMath {
   static constexpr int kWarpsPerSM = 0;  // no register cap
   static constexpr int kScratchBytes = 0;
   static constexpr int kTmemCols = 0;
+  static constexpr int kCodeBytes = 2048;  // one page of K (or V) codes
   static constexpr int DPL = (G <= 4) ? 16 : 8;  // dims per lane
   static constexpr int LPT = kD / DPL;           // lanes per token
   static constexpr int TPP = 32 / LPT;           // tokens per pass
@@ -358,6 +359,7 @@ struct MmaMath {
   static constexpr int kWarpsPerSM = 12;  // cap registers at 168 per thread
   static constexpr int kScratchBytes = 0;
   static constexpr int kTmemCols = 0;
+  static constexpr int kCodeBytes = 2048;  // one page of K (or V) codes
   static constexpr float kSlack = 8.0f;   // log2 units
   static constexpr int kVSlack = 4;
   int lane, r, c;
@@ -752,6 +754,7 @@ struct I8Math {
   static constexpr int kWarpsPerSM = 12;  // cap registers at 168 per thread
   static constexpr int kScratchBytes = InTmem ? 0 : 32 * 32 * 4;  // fp32 [32][lane]
   static constexpr int kTmemCols = InTmem ? 32 : 0;
+  static constexpr int kCodeBytes = 2048;  // one page of K (or V) codes
   static constexpr float kSlack = 6.0f;   // log2 units
   static constexpr int kVSlack = 2;
   static constexpr int kF = 23;  // P'' < 2^(kSlack + kVSlack): P < 2^31
@@ -1048,5 +1051,357 @@ struct I8Math {
   }
 };
 
+// s8 x u8 integer mma, K = 32: D[16x8] (s32) += A[16x32] (s8) . B[32x8] (u8).
+__device__ __forceinline__ void mma16832_s8u8(int (&d)[4], uint32_t a0,
+                                              uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0,
+                                              uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, "
+      "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// u8 x u8 integer mma, K = 16: D[16x8] (s32) += A[16x16] (u8) . B[16x8] (u8).
+__device__ __forceinline__ void mma16816_u8u8(int (&d)[4], uint32_t a0,
+                                              uint32_t a1, uint32_t b0) {
+  asm("mma.sync.aligned.m16n8k16.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, "
+      "{%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+// The INT4 form (groups of G <= 4 heads) over the INT4 cache: K and V codes
+// are excess-8 nibbles u = c + 8, two per byte (dims 2i / 2i+1 in the low /
+// high nibble of byte i); a page is 16 tokens x 64 bytes, staged by TMA as
+// 8 rows of 128 bytes (tokens 2R and 2R+1 in row R) with the 128-byte
+// swizzle.  The arithmetic is I8Math's, with the nibbles fed to the tensor
+// cores as unsigned bytes and the bias removed exactly in integers:
+// * q.k: sum_j d_j u_j = sum_j d_j c_j + 8 sum_j d_j, so every plane's
+//   accumulator starts at -8 sum_j d_j (the plane's digit sum over the 128
+//   dims).  A thread's 16 bytes of a token (dims 32c..32c+31) unpack into
+//   even-dim words (mask) and odd-dim words (shift + mask); k-step s pairs
+//   the even and odd words of dims 32c + 8s .. + 7, and q's digit planes
+//   are laid out the same way.
+// * p.v: one transposing ldmatrix of the packed V page gives, per 16-byte
+//   column chunk q (dims 32q..32q+31), the even-dim m-tile (low nibbles)
+//   and the odd-dim m-tile (high nibbles); sum_t P_t u_t - 8 sum_t P_t is
+//   taken per digit plane, the planes' digit sums tracked with dp4a and
+//   subtracted (times 8) from the int32 accumulators when they are drained.
+template <int G>
+struct I4Math {
+  static_assert(G == 1 || G == 2 || G == 4, "groups of 1, 2 or 4 heads");
+  static constexpr int kWarpsPerSM = 12;
+  static constexpr int kScratchBytes = 0;
+  static constexpr int kTmemCols = 32;
+  static constexpr int kCodeBytes = 1024;  // one page of K (or V) nibbles
+  static constexpr float kSlack = 6.0f;
+  static constexpr int kVSlack = 2;
+  static constexpr int kF = 23;
+  static constexpr int kMinE = kF - 127;
+  int lane, r, c, up;
+  uint32_t qa[4][4];
+  int dsa, dsb;       // digit sums of planes (rows r, r+8) over the head's dims
+  float qf;
+  int acc[8][2][4];
+  int psum[2];        // this thread's P digit sums (n-tiles 0, 1) since the last drain
+  uint32_t otm;
+  float m_run, l_run;
+  int e_run;
+  float vlim, fsF;
+  uint32_t psel;
+  bool started, of_live;
+
+  __device__ __forceinline__ void attach(uint8_t*) {}
+  __device__ __forceinline__ void attach_tmem(uint32_t taddr) { otm = taddr; }
+
+  __device__ __forceinline__ void init(const __nv_bfloat16* qg, float q_scale,
+                                       int lane_) {
+    lane = lane_;
+    r = lane >> 2;
+    c = lane & 3;
+    up = r >> 2;
+    const int h = (r & 3) % G;
+    float qv[32];
+    const uint4* src = reinterpret_cast<const uint4*>(qg + h * kD + 32 * c);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 raw = src[i];
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        qv[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+        qv[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(qv[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+    const int sh = amax > 0.0f ? 30 - exp_frexp(amax) : 0;
+    const float f1 = pow2i(sh / 2), f2 = pow2i(sh - sh / 2);
+    const uint32_t pa = up ? 2u : 3u, pb = up ? 0u : 1u;
+    const uint32_t sel = pa | ((4u + pa) << 4) | (pb << 8) | ((4u + pb) << 12);
+    int sa = 0, sb = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // k-step s = i / 2; i even: dims 32c + 8s + {0,2,4,6}, odd: + {1,3,5,7}
+      const int s = i >> 1, odd = i & 1;
+      uint32_t u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        u[j] = static_cast<uint32_t>(
+                   __float2int_rn(qv[8 * s + 2 * j + odd] * f1 * f2)) +
+               0x80808080u;
+      const uint32_t x = prmt(u[0], u[1], sel);
+      const uint32_t y = prmt(u[2], u[3], sel);
+      const uint32_t wa = prmt(x, y, 0x5410u) ^ 0x80808080u;
+      const uint32_t wb = prmt(x, y, 0x7632u) ^ 0x80808080u;
+      sa = __dp4a(static_cast<int>(wa), 0x01010101, sa);
+      sb = __dp4a(static_cast<int>(wb), 0x01010101, sb);
+      if (odd) {
+        qa[s][2] = wa;
+        qa[s][3] = wb;
+      } else {
+        qa[s][0] = wa;
+        qa[s][1] = wb;
+      }
+    }
+    sa += __shfl_xor_sync(kFull, sa, 1);
+    sa += __shfl_xor_sync(kFull, sa, 2);
+    sb += __shfl_xor_sync(kFull, sb, 1);
+    sb += __shfl_xor_sync(kFull, sb, 2);
+    dsa = sa;
+    dsb = sb;
+    qf = q_scale * pow2i(-(sh / 2)) * pow2i(-(sh - sh / 2));
+    psel = static_cast<uint32_t>(up) | ((4u + up) << 4) | ((2u + up) << 8) |
+           ((6u + up) << 12);
+    reset();
+  }
+
+  __device__ __forceinline__ void zero_acc() {
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[m][t][e] = 0;
+    psum[0] = psum[1] = 0;
+  }
+
+  __device__ __forceinline__ void reset() {
+    m_run = -INFINITY;
+    l_run = 0.0f;
+    e_run = kMinE;
+    vlim = 0.0f;
+    fsF = pow2i(kF - kMinE);
+    started = false;
+    of_live = false;
+    zero_acc();
+  }
+
+  // remove the V bias (8 x the column's digit sum) from the accumulators
+  __device__ __forceinline__ void unbias() {
+    int s0 = psum[0], s1 = psum[1];
+    s0 += __shfl_xor_sync(kFull, s0, 1);
+    s0 += __shfl_xor_sync(kFull, s0, 2);
+    s1 += __shfl_xor_sync(kFull, s1, 1);
+    s1 += __shfl_xor_sync(kFull, s1, 2);
+    // column n of n-tile t is thread row n's plane: columns 2c, 2c+1 here
+    const int a0 = __shfl_sync(kFull, s0, 4 * (2 * c)), a1 = __shfl_sync(kFull, s0, 4 * (2 * c + 1));
+    const int b0 = __shfl_sync(kFull, s1, 4 * (2 * c)), b1 = __shfl_sync(kFull, s1, 4 * (2 * c + 1));
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[m][0][e] -= 8 * ((e & 1) ? a1 : a0);
+        acc[m][1][e] -= 8 * ((e & 1) ? b1 : b0);
+      }
+  }
+
+  __device__ __forceinline__ void drain(float aA, float aB) {
+    unbias();
+    const float w0 = pow2i(8 * (c >> 1) - kF);
+    const float w1 = pow2i(16 + 8 * (c >> 1) - kF);
+    float o[32];
+    if (of_live) {
+      tm_ld32(otm, o);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) o[k] = 0.0f;
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = m * 4 + e;
+        const float v = __int2float_rn(acc[m][0][e]) * w0 +
+                         __int2float_rn(acc[m][1][e]) * w1;
+        o[k] = (o[k] + v) * ((e & 1) ? aB : aA);
+      }
+    tm_st32(otm, o);
+    of_live = true;
+    zero_acc();
+  }
+
+  template <bool Full>
+  __device__ __forceinline__ void page(const uint8_t* tk, const uint8_t* tv,
+                                       const float* ks, const float* vs,
+                                       int nv) {
+    // ---- S = Qd K^T: n-tile j, column n = r: token 4(r/2) + 2j + r%2;
+    //      this thread's 16 bytes of a token t: row t/2, chunk 4(t%2) + c
+    const int ta = 4 * (r >> 1) + (r & 1), tb = ta + 2;
+    const uint4 pka = *reinterpret_cast<const uint4*>(
+        tk + (ta >> 1) * 128 + (((4 * (ta & 1) + c) ^ ((ta >> 1) & 7)) << 4));
+    const uint4 pkb = *reinterpret_cast<const uint4*>(
+        tk + (tb >> 1) * 128 + (((4 * (tb & 1) + c) ^ ((tb >> 1) & 7)) << 4));
+    int sacc[2][4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      sacc[j][0] = sacc[j][1] = -8 * dsa;
+      sacc[j][2] = sacc[j][3] = -8 * dsb;
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const uint32_t wa = word_of(pka, s), wb = word_of(pkb, s);
+      mma16832_s8u8(sacc[0], qa[s][0], qa[s][1], qa[s][2], qa[s][3],
+                    wa & 0x0F0F0F0Fu, (wa >> 4) & 0x0F0F0F0Fu);
+      mma16832_s8u8(sacc[1], qa[s][0], qa[s][1], qa[s][2], qa[s][3],
+                    wb & 0x0F0F0F0Fu, (wb >> 4) & 0x0F0F0F0Fu);
+    }
+    const float wa = up ? 65536.0f : 16777216.0f;
+    const float wb = up ? 1.0f : 256.0f;
+    float st[4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float part = __fmaf_rn(__int2float_rn(sacc[j][e]), wa,
+                                     __int2float_rn(sacc[j][2 + e]) * wb);
+        st[2 * j + e] = part + __shfl_xor_sync(kFull, part, 16);
+      }
+    const float4 ks4 = *reinterpret_cast<const float4*>(ks + 4 * c);
+    const float4 vs4 = *reinterpret_cast<const float4*>(vs + 4 * c);
+    const float ksv[4] = {ks4.x, ks4.y, ks4.z, ks4.w};
+    const float vsr[4] = {vs4.x, vs4.y, vs4.z, vs4.w};
+    float sc[4], vsv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (Full) {
+        sc[i] = st[i] * qf * ksv[i];
+        vsv[i] = vsr[i];
+      } else {
+        const bool ok = 4 * c + i < nv;
+        sc[i] = ok ? st[i] * qf * ksv[i] : -INFINITY;
+        vsv[i] = ok ? vsr[i] : 0.0f;
+      }
+    }
+    const float lm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    const float lv = fmaxf(fmaxf(vsv[0], vsv[1]), fmaxf(vsv[2], vsv[3]));
+    if (__any_sync(kFull, lm > m_run + kSlack || lv > vlim)) {
+      float x = fmaxf(lm, __shfl_xor_sync(kFull, lm, 1));
+      x = fmaxf(x, __shfl_xor_sync(kFull, x, 2));
+      float vx = fmaxf(lv, __shfl_xor_sync(kFull, lv, 1));
+      vx = fmaxf(vx, __shfl_xor_sync(kFull, vx, 2));
+      const float n = fmaxf(m_run, x);
+      const int e_new = vx > vlim ? max(exp_frexp(vx), kMinE) : e_run;
+      const float a = (n == m_run) ? 1.0f : ex2(m_run - n);
+      const float a_o = a * pow2i(max(e_run - e_new, -126));
+      if (started) {
+        const int hA = ((2 * c) & 3) % G, hB = ((2 * c + 1) & 3) % G;
+        const float aA = __shfl_sync(kFull, a_o, 4 * hA);
+        const float aB = __shfl_sync(kFull, a_o, 4 * hB);
+        drain(aA, aB);
+      }
+      l_run *= a;
+      m_run = n;
+      e_run = e_new;
+      vlim = pow2i(min(e_new + kVSlack, 127));
+      fsF = pow2i(kF - e_new);
+    }
+    const float mu = m_run == -INFINITY ? 0.0f : m_run;
+    float pr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pr[i] = ex2(sc[i] - mu);
+    l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+    uint32_t pi[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pi[i] = __float2uint_rn(pr[i] * (vsv[i] * fsF));
+    const uint32_t x = prmt(pi[0], pi[1], psel);
+    const uint32_t y = prmt(pi[2], pi[3], psel);
+    const uint32_t b0 = prmt(x, y, 0x5410u);
+    const uint32_t b1 = prmt(x, y, 0x7632u);
+    psum[0] = static_cast<int>(__dp4a(b0, 0x01010101u, static_cast<unsigned>(psum[0])));
+    psum[1] = static_cast<int>(__dp4a(b1, 0x01010101u, static_cast<unsigned>(psum[1])));
+
+    // ---- O^T += V^T Pd^T: ldmatrix rows = tokens 0..15; lanes 0..15 take
+    //      column chunk 2w, lanes 16..31 chunk 2w+1 (dims 32q..32q+31)
+    const int vt = lane & 15, vq = lane >> 4;
+    const uint32_t vrow = smem_u32(tv) + (vt >> 1) * 128;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const int q = 2 * w + vq;
+      uint32_t r0, r1, r2, r3;
+      ldsm_x2_trans_b8(vrow + (((4 * (vt & 1) + q) ^ ((vt >> 1) & 7)) << 4), r0, r1, r2, r3);
+      // chunk 2w: m-tiles 4w (even dims) and 4w+1 (odd); chunk 2w+1: 4w+2, 4w+3
+      const uint32_t e0 = r0 & 0x0F0F0F0Fu, e1 = r1 & 0x0F0F0F0Fu;
+      const uint32_t o0 = (r0 >> 4) & 0x0F0F0F0Fu, o1 = (r1 >> 4) & 0x0F0F0F0Fu;
+      const uint32_t e2 = r2 & 0x0F0F0F0Fu, e3 = r3 & 0x0F0F0F0Fu;
+      const uint32_t o2 = (r2 >> 4) & 0x0F0F0F0Fu, o3 = (r3 >> 4) & 0x0F0F0F0Fu;
+      mma16816_u8u8(acc[4 * w][0], e0, e1, b0);
+      mma16816_u8u8(acc[4 * w][1], e0, e1, b1);
+      mma16816_u8u8(acc[4 * w + 1][0], o0, o1, b0);
+      mma16816_u8u8(acc[4 * w + 1][1], o0, o1, b1);
+      mma16816_u8u8(acc[4 * w + 2][0], e2, e3, b0);
+      mma16816_u8u8(acc[4 * w + 2][1], e2, e3, b1);
+      mma16816_u8u8(acc[4 * w + 3][0], o2, o3, b0);
+      mma16816_u8u8(acc[4 * w + 3][1], o2, o3, b1);
+    }
+    started = true;
+  }
+
+  __device__ __forceinline__ void finish(const ChunkSink& sk) {
+    if (started) drain(1.0f, 1.0f);
+    float l = l_run;
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+    const int nA = 2 * c, nB = 2 * c + 1;
+    const int hA = (nA & 3) % G, hB = (nB & 3) % G;
+    const float sA = __shfl_sync(kFull, l, 4 * hA);
+    const float sB = __shfl_sync(kFull, l, 4 * hB);
+    const float mA = __shfl_sync(kFull, m_run, 4 * hA);
+    const float mB = __shfl_sync(kFull, m_run, 4 * hB);
+    const float f = pow2i(e_run);
+    const bool wA = c < 2 && nA < G, wB = c < 2 && nB < G;
+    float o[32];
+    if (of_live) {
+      tm_ld32(otm, o);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) o[k] = 0.0f;
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = m * 4 + e;
+        float v = o[k];
+        v += __shfl_xor_sync(kFull, v, 2);
+        // m-tile m: chunk q = m / 2 (dims 32q..), odd dims when m is odd;
+        // rows r / r+8 are bytes r / r+8 of the chunk
+        const int d = 32 * (m >> 1) + 2 * r + ((e & 2) ? 16 : 0) + (m & 1);
+        if (e & 1) {
+          if (wB) sk.put_o(nB, d, v * f, sB);
+        } else {
+          if (wA) sk.put_o(nA, d, v * f, sA);
+        }
+      }
+    if (r == 0) {
+      if (wA) sk.put_ml(nA, mA, sA);
+      if (wB) sk.put_ml(nB, mB, sB);
+    }
+  }
+};
 }  // namespace
 }  // namespace kv8

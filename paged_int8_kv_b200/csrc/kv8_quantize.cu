@@ -23,13 +23,22 @@ namespace {
 constexpr int kD = 128;
 constexpr int kBS = 16;
 
+// Levels each side of zero: 127 for INT8 codes, 7 for INT4 codes.
+template <int Bits>
 __device__ __forceinline__ int quant_one(float x, float s) {
+  constexpr float kL = Bits == 8 ? 127.0f : 7.0f;
   if (s == 0.0f) return 0;
   float r = rintf(__fdiv_rn(x, s));
-  r = fminf(fmaxf(r, -127.0f), 127.0f);
+  r = fminf(fmaxf(r, -kL), kL);
   return static_cast<int>(r);
 }
 
+// Bits == 8: int8 codes, one 128-byte row per (token, KV head).
+// Bits == 4: the INT4 variant [nano-KvLLM, §2.2: historical tokens' K/V in
+// 4 bits]: s = fl32(max|x|/7), codes clamped to +-7 and stored as the
+// nibble code + 8, dims 2i / 2i+1 in the low / high nibble of byte i; one
+// 64-byte row per (token, KV head).
+template <int Bits>
 __global__ void __launch_bounds__(256)
 quantize_append_kernel(const __nv_bfloat16* __restrict__ k_new,
                        const __nv_bfloat16* __restrict__ v_new,
@@ -39,6 +48,8 @@ quantize_append_kernel(const __nv_bfloat16* __restrict__ k_new,
                        int8_t* __restrict__ v_cache,
                        float* __restrict__ k_scales,
                        float* __restrict__ v_scales) {
+  constexpr float kL = Bits == 8 ? 127.0f : 7.0f;
+  constexpr int kRowBytes = kD * Bits / 8;
   const int lane = threadIdx.x & 31;
   const int64_t warps_total =
       static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -63,16 +74,24 @@ quantize_append_kernel(const __nv_bfloat16* __restrict__ k_new,
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1)
       a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
-    const float s = (a == 0.0f) ? 0.0f : __fdiv_rn(a, 127.0f);
-    uint32_t packed = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      packed |= (static_cast<uint32_t>(quant_one(x[i], s)) & 0xFFu) << (8 * i);
+    const float s = (a == 0.0f) ? 0.0f : __fdiv_rn(a, kL);
     const int64_t blk = slot / kBS;
     const int64_t off = slot - blk * kBS;
     const int64_t base = (blk * num_kv_heads + h) * kBS + off;
-    int8_t* dst = (which ? v_cache : k_cache) + base * kD;
-    reinterpret_cast<uint32_t*>(dst)[lane] = packed;
+    int8_t* dst = (which ? v_cache : k_cache) + base * kRowBytes;
+    if constexpr (Bits == 8) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        packed |= (static_cast<uint32_t>(quant_one<8>(x[i], s)) & 0xFFu) << (8 * i);
+      reinterpret_cast<uint32_t*>(dst)[lane] = packed;
+    } else {
+      uint32_t packed = 0;  // dims 4 lane .. 4 lane + 3 -> two bytes
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        packed |= static_cast<uint32_t>(quant_one<4>(x[i], s) + 8) << (4 * i);
+      reinterpret_cast<uint16_t*>(dst)[lane] = static_cast<uint16_t>(packed);
+    }
     if (lane == 0) (which ? v_scales : k_scales)[base] = s;
   }
 }
@@ -83,13 +102,14 @@ int launch_quantize_append(const void* k_new, const void* v_new,
                            const int64_t* slot_mapping, int64_t n_tokens,
                            int32_t num_kv_heads, int8_t* k_cache,
                            int8_t* v_cache, float* k_scales, float* v_scales,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, int32_t bits) {
   const int64_t n_rows = n_tokens * num_kv_heads * 2;
   const int threads = 256;
   const int64_t warps_per_block = threads / 32;
   int64_t blocks = (n_rows + warps_per_block - 1) / warps_per_block;
   if (blocks > 148 * 64) blocks = 148 * 64;  // grid-stride beyond this
-  quantize_append_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+  auto kern = bits == 4 ? quantize_append_kernel<4> : quantize_append_kernel<8>;
+  kern<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(k_new),
       static_cast<const __nv_bfloat16*>(v_new), slot_mapping, n_rows,
       num_kv_heads, k_cache, v_cache, k_scales, v_scales);
