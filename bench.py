@@ -705,6 +705,97 @@ def run_extend(args, rank: int, world: int, dist):
     return 0
 
 
+INT4_BYTES_PER_TOKEN_HEAD = 2 * 64 + 2 * 4  # packed K+V nibbles, fp32 scales
+
+
+def run_int4(args, w: W.Workload, rank: int, world: int, dist):
+    """The INT4 cache variant on the timed workload: one step = the step's
+    INT4 quantise-append plus one kv8_int4_paged_decode_attention call,
+    inputs resident (the 32K workload's INT4 cache, 2.2 GB, is larger than
+    L2)."""
+    import torch
+    import paged_int8_kv_b200 as pk
+    dev = torch.device("cuda", _env_int("LOCAL_RANK", 0))
+    torch.cuda.set_device(dev)
+    shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim // 2)
+    kc = torch.zeros(shape, dtype=torch.uint8, device=dev)
+    vc = torch.zeros(shape, dtype=torch.uint8, device=dev)
+    ks = torch.zeros(shape[:3], dtype=torch.float32, device=dev)
+    vs = torch.zeros(shape[:3], dtype=torch.float32, device=dev)
+
+    def to_dev(a, bf16=True):
+        t = torch.from_numpy(a).pin_memory().to(dev, non_blocking=True)
+        return t.view(torch.bfloat16) if bf16 else t
+    for k, v, sl in w.fill_segments():
+        if sl.shape[0]:
+            pk.kv8_int4_quantize_append(to_dev(k), to_dev(v), to_dev(sl, False),
+                                        kc, vc, ks, vs)
+    kn, vn, sl = w.step_tokens()
+    k_new, v_new, slots = to_dev(kn), to_dev(vn), to_dev(sl, False)
+    q = to_dev(w.q())
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    cl = torch.from_numpy(w.context_lens).to(dev)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    chunk = pick_chunk(w, args.chunk)
+    nbytes = pk.kv8_decode_workspace_bytes(w.batch, w.num_q_heads, w.head_dim,
+                                           w.max_context_len, chunk)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def decode():
+        pk.kv8_int4_paged_decode_attention(q, kc, vc, ks, vs, bt, cl, out,
+                                           w.max_context_len,
+                                           chunk_tokens=chunk, workspace=ws)
+
+    def step():
+        pk.kv8_int4_quantize_append(k_new, v_new, slots, kc, vc, ks, vs)
+        decode()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks([t0.elapsed_time(t1) / args.steps], dist, dev)[0]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:
+        a.record(stream)
+        decode()
+        b.record(stream)
+    torch.cuda.synchronize()
+    dec_ms = statistics.median([a.elapsed_time(b) for a, b in ev])
+    status = pk.kv8_read_device_status(clear=True)
+    ab = algorithmic_bytes(w)
+    kv = w.token_heads() * INT4_BYTES_PER_TOKEN_HEAD
+    total = kv + ab["total"] - ab["kv"]
+    peak, src = measured_peaks()
+    gbs = total / (dec_ms * 1e-3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "paged INT4-KV decode attention tokens/s and achieved HBM GB/s",
+            "value": whole_job_rate(w.batch, world, ms), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u4 codes, s8/u8 integer mma, f32 softmax",
+            "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": w.name + "_int4", "batch": w.batch,
+                       "context_tokens": int(w.context_lens.sum()),
+                       "chunk_tokens": chunk, "l2": "inputs larger than L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak,
+                         "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "peak_source": src,
+                         "algorithmic_bytes": total,
+                         "decode_us": dec_ms * 1e3},
+            "device_status": status}), flush=True)
+    return 0
+
+
 def run_dry_cpu(args, rank: int, world: int, dist):
     """The launch and rank logic alone, on CPU ranks over gloo: every rank
     times a trivial host step, the max over ranks is taken, rank 0 prints a
@@ -765,6 +856,8 @@ def main():
     ap.add_argument("--no-per-workload", action="store_true")
     ap.add_argument("--extend", action="store_true",
                     help="time extend (chunked-prefill) attention instead")
+    ap.add_argument("--int4", action="store_true",
+                    help="time the INT4 cache variant on --workload instead")
     ap.add_argument("--dry-run-cpu", action="store_true",
                     help="rank/launch logic only, on CPU over gloo (no GPU work, "
                          "no measurement)")
@@ -796,6 +889,8 @@ def main():
             return run_dry_cpu(args, rank, world, dist)
         if args.extend:
             return run_extend(args, rank, world, dist)
+        if args.int4:
+            return run_int4(args, W.NAMED[args.workload](), rank, world, dist)
         return run_kv8(args, W.NAMED[args.workload](), rank, world, dist)
     finally:
         if dist is not None:

@@ -53,14 +53,16 @@ namespace {
 //               2048 for INT8 codes, 1024 for packed INT4 codes)
 //   per warp w: SPW slots of [ks 64 B | vs 64 B]              (scales)
 //   per warp w: the page math's scratch (ScratchBytes, may be 0)
-//   per warp w: SPW mbarriers
+//   per warp w: SPW mbarriers, then its work queue (kQueue item indices)
 // --------------------------------------------------------------------------
+constexpr int kQueue = 16;  // > SPW + 1: queued items each hold an issued page
 template <int WPC, int SPW, int ScratchBytes = 0, int CodeBytes = kPageBytes>
 struct SmemPlan {
   static constexpr int kTileBytes = WPC * SPW * 2 * CodeBytes;
   static constexpr int kScaleBytes = WPC * SPW * 2 * kBS * 4;
   static constexpr int kScratchBytes = WPC * ScratchBytes;
-  static constexpr int kBarBytes = WPC * (SPW * 8 + 32);  // + work queue
+  static_assert(SPW + 1 <= kQueue, "work queue too short for the page ring");
+  static constexpr int kBarBytes = WPC * (SPW * 8 + kQueue * 4);
   static constexpr int kBytes =
       kTileBytes + kScaleBytes + kScratchBytes + kBarBytes + 16 + 1024;
 };
@@ -118,6 +120,31 @@ __device__ __forceinline__ bool item_fill(const DecodeParams& p, Item& it) {
   return true;
 }
 
+// The result of an item without pages: a zero output row for an empty
+// context (a single-chunk item), else an empty partial (m = -inf, l = 0,
+// o = 0) that a merge skips.  Warp-cooperative.
+template <int G>
+__device__ __forceinline__ void write_empty(const DecodeParams& p,
+                                            const Item& it, int lane) {
+  const int64_t row0 = static_cast<int64_t>(it.b) * p.num_q_heads + it.kvh * G;
+  const int nchunks = (it.n + p.chunk_tokens - 1) / p.chunk_tokens;
+  for (int h = 0; h < G; ++h) {
+    if (nchunks <= 1 && !p.partials_only) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        store_out(p.out, (row0 + h) * kD + 4 * lane + e, 0.0f, p.out_f32);
+    } else {
+      const int64_t ci = (row0 + h) * p.max_chunks + it.chunk;
+      reinterpret_cast<float4*>(p.ws_o + ci * kD)[lane] =
+          make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (lane == 0) {
+        p.ws_ml[2 * ci] = -INFINITY;
+        p.ws_ml[2 * ci + 1] = 0.0f;
+      }
+    }
+  }
+}
+
 template <int G, int WPC, int SPW, class Math>
 __global__ void __launch_bounds__(WPC * 32,
                                   Math::kWarpsPerSM / WPC > 0 ? Math::kWarpsPerSM / WPC : 1)
@@ -138,7 +165,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       smem + Plan::kTileBytes + Plan::kScaleBytes + warp * Math::kScratchBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       smem + Plan::kTileBytes + Plan::kScaleBytes + Plan::kScratchBytes +
-      warp * (SPW * 8 + 32));
+      warp * (SPW * 8 + kQueue * 4));
   if (lane == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
@@ -172,8 +199,12 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   // launch has a work counter, W + (counter++): a warp that finishes early
   // takes more, so uneven items do not leave a slow tail.  The issue cursor
   // takes items and queues their indices in shared memory; the compute
-  // cursor, up to SPW pages behind, pops them in the same order.
-  int* wq = reinterpret_cast<int*>(bars + SPW);  // 8 entries per warp
+  // cursor, up to SPW pages behind, pops them in the same order.  Items
+  // without pages (an empty context, or a partials slot past a sequence's
+  // end) are finished by the issue side when taken and never queued, so
+  // every queued item holds a page in flight: at most SPW of them, plus the
+  // end marker.
+  int* wq = reinterpret_cast<int*>(bars + SPW);  // kQueue entries per warp
   uint32_t q_tail = 0, q_head = 0;
   // item indices fit 31 bits (the host checks max_chunks * H_kv * B)
   const uint32_t n_items = static_cast<uint32_t>(p.max_chunks) *
@@ -199,7 +230,11 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       const bool live = idx < n_items;  // (no wrap: W + counter < 2^32)
       if (live) item_set(p, idx, it);
       if (!live || item_fill(p, it)) {
-        if (lane == 0) wq[q_tail & 7] = live ? static_cast<int>(idx) : -1;
+        if (live && it.npages == 0) {
+          write_empty<G>(p, it, lane);
+          continue;
+        }
+        if (lane == 0) wq[q_tail % kQueue] = live ? static_cast<int>(idx) : -1;
         ++q_tail;
         __syncwarp();
         return live;
@@ -209,7 +244,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   // compute side: the next queued item (false: no more)
   auto pop = [&](Item& it) -> bool {
     __syncwarp();
-    const int idx = wq[q_head & 7];
+    const int idx = wq[q_head % kQueue];
     ++q_head;
     if (idx < 0) return false;
     item_set(p, static_cast<uint32_t>(idx), it);
@@ -437,14 +472,14 @@ int launch_decode_kernel(const DecodeParams& p, const CUtensorMap& tmk,
     if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return -1;
-    int nsm = 0, occ = 0;
+    int nsm = 0;
     if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, WPC * 32,
-                                                      smem) != cudaSuccess)
+        cudaSuccess)
       return -1;
+    const int occ = resident_ctas(kern, WPC * 32, smem, Math::kTmemCols);
+    if (occ == 0) return -1;
     sms = nsm;
-    resident = occ > 0 ? occ : 1;
+    resident = occ;
     f->sms.store(sms, std::memory_order_release);
     f->resident.store(resident, std::memory_order_release);
   }

@@ -895,28 +895,13 @@ int launch_tc(const DecodeParams& p, const CUtensorMap& tmk,
     if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return -1;
-    // CTAs per SM from the per-SM limits (the runtime's occupancy query
-    // reports one CTA per SM for this kernel whatever its shared memory)
-    cudaFuncAttributes fa;
-    int nsm = 0, smem_sm = 0, smem_rsv = 0, thr_sm = 0, regs_sm = 0;
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
-        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
-            cudaSuccess ||
-        cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
-            cudaSuccess ||
-        cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) !=
-            cudaSuccess ||
-        cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) !=
-            cudaSuccess)
+    int nsm = 0;
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) !=
+        cudaSuccess)
       return -1;
     sms = nsm;
-    const int warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;
-    int r = smem_sm / (smem + static_cast<int>(fa.sharedSizeBytes) + smem_rsv);
-    r = min(r, thr_sm / kThreads);
-    r = min(r, regs_sm / (warp_regs * (kThreads / 32)));
-    r = min(r, 512 / kTmemCols);  // tensor-memory columns of the SM
-    resident = r < 1 ? 1 : r;
+    resident = resident_ctas(kern, kThreads, smem, kTmemCols);
+    if (resident == 0) return -1;
     f->sms.store(sms, std::memory_order_release);
     f->resident.store(resident, std::memory_order_release);
   }

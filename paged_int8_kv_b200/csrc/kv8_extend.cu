@@ -503,6 +503,7 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
       for (int j = 0; j < it.nkt; ++j) {
         const uint32_t t = u + j;
         ewait(&bars[B_S_FULL + (t & 1)], (t >> 1) & 1, failed);
+        __syncwarp();  // converged for the warp-collective tensor-memory loads
         tc_fence_after();
         const float* ks = reinterpret_cast<const float*>(smem + ExtPlan::kScl +
                                                          (t & 3) * 2 * kKT * 4);
@@ -553,6 +554,7 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
         }
         // P16 is free and O is up to date once the previous O product is done
         if (t >= 1) ewait(&bars[B_O_DONE], (t - 1) & 1, failed);
+        __syncwarp();
         tc_fence_after();
         // rescale O in tensor memory where the row's references moved; the
         // tensor-memory loads and stores are warp-collective, so the whole
@@ -582,6 +584,7 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
       u += it.nkt;
       // ---- output: wait for the last O product, normalise, store
       ewait(&bars[B_O_DONE], (u - 1) & 1, failed);
+      __syncwarp();
       tc_fence_after();
       const float f = pow2i(e_run) / (l_run > 0.0f ? l_run : 1.0f);
 #pragma unroll 1

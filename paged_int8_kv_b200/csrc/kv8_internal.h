@@ -31,6 +31,37 @@ inline LaunchFacts* facts_for_current_device(LaunchFacts (&table)[kMaxDevices]) 
   return &table[dev];
 }
 
+// CTAs of a kernel that fit one SM of the current device at once, from
+// the per-SM limits (shared memory, threads, registers, and the SM's 512
+// tensor-memory columns when the kernel allocates tmem_cols of them per
+// CTA).  The runtime's occupancy query is not used: it reports one CTA per
+// SM for any kernel that allocates tensor memory.  Returns 0 on a CUDA
+// error, else >= 1.
+template <class Kernel>
+int resident_ctas(Kernel kern, int threads, int dyn_smem, int tmem_cols) {
+  int dev = 0, smem_sm = 0, smem_rsv = 0, thr_sm = 0, regs_sm = 0;
+  cudaFuncAttributes fa;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
+                             dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock,
+                             dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor,
+                             dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor,
+                             dev) != cudaSuccess)
+    return 0;
+  const int warps = (threads + 31) / 32;
+  const int warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;
+  int r = smem_sm / (dyn_smem + static_cast<int>(fa.sharedSizeBytes) + smem_rsv);
+  if (thr_sm / threads < r) r = thr_sm / threads;
+  if (warp_regs > 0 && regs_sm / (warp_regs * warps) < r)
+    r = regs_sm / (warp_regs * warps);
+  if (tmem_cols > 0 && 512 / tmem_cols < r) r = 512 / tmem_cols;
+  return r < 1 ? 1 : r;
+}
+
 constexpr int kHeadDim = 128;
 constexpr int kBlockSize = 16;
 constexpr int kPageBytes = kHeadDim * kBlockSize;  // 2048 code bytes
