@@ -565,6 +565,7 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
 #pragma unroll 1
           for (int c = 0; c < kD / 32; ++c) {
             float o[32];
+            __syncwarp();
             tmem_ld32(trow + kColO + 32 * c, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= f;
@@ -590,6 +591,7 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         float o[32];
+        __syncwarp();  // the stores below diverge by row; reconverge first
         tmem_ld32(trow + kColO + 32 * c, o);
         if (live) {
           if (p.out_f32) {
