@@ -343,9 +343,10 @@ int32_t kv8_paged_decode_attention_prefix(
   if (!clear_tickets(d, batch, num_q_heads, st)) return KV8_ERR_CUDA;
   kv8::PrefixShape ps;
   ps.num_groups = num_groups;
-  ps.rounds = (max_group_size + 7) / 8;
+  ps.max_group_size = max_group_size;
+  ps.rounds = 0;
   ps.prefix_chunks = max_prefix_len / d.p.chunk_tokens;
-  if (num_groups > 0 && ps.rounds > 0 && ps.prefix_chunks > 0) {
+  if (num_groups > 0 && max_group_size > 0 && ps.prefix_chunks > 0) {
     d.p.prefix_group = prefix_group;
     d.p.prefix_lens = prefix_lens;
     const int rc = kv8::launch_prefix(d.p, ps, d.tmk, d.tmv, st);

@@ -97,6 +97,49 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src,
       : "memory");
 }
 
+// The same operations on 32-bit shared addresses (no address conversion at
+// each call).
+__device__ __forceinline__ void mbar_arrive_expect_tx_s(uint32_t bar,
+                                                        uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   bar),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_wait_s(uint32_t bar, uint32_t parity,
+                                            uint32_t* status) {
+  for (uint32_t i = 0; i < kMaxWaitPolls; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  atomicOr(status, KV8_DEV_WAIT_TIMEOUT);
+  return false;
+}
+__device__ __forceinline__ void bulk_g2s_s(uint32_t dst, const void* src,
+                                           uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_s(uint32_t dst, const CUtensorMap* map,
+                                              int32_t c0, int32_t c1, int32_t c2,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_"
+      "tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
 // 3-D tiled tensor copy global -> shared through a tensor map (no multicast).
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map,
                                             int32_t c0, int32_t c1, int32_t c2,

@@ -166,6 +166,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       smem + Plan::kTileBytes + Plan::kScaleBytes + Plan::kScratchBytes +
       warp * (SPW * 8 + kQueue * 4));
+  const uint32_t tiles_s = smem_u32(tiles), scl_s = smem_u32(scl);
   if (lane == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
@@ -252,25 +253,33 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     return true;
   };
 
-  // ---- issue cursor: SPW pages ahead of the compute cursor
-  Item iss;
-  bool iss_live = take(iss);
-  int iss_page = 0;
+  // ---- issue cursor: SPW pages ahead of the compute cursor.  Its state is
+  // kept small (the page math needs the registers): the table offset of the
+  // item's first page, its KV head and page count, and the page reached.
+  const uint32_t bars_s = smem_u32(bars);
+  bool iss_live;
+  int iss_page = 0, iss_np = 0, iss_kvh = 0;
+  int64_t iss_tab = 0;
+  auto take_iss = [&]() {
+    Item it;
+    iss_live = take(it);
+    iss_page = 0;
+    if (iss_live) {
+      iss_np = it.npages;
+      iss_kvh = it.kvh;
+      iss_tab = static_cast<int64_t>(it.b) * p.max_blocks_per_seq + it.tok0 / kBS;
+    }
+  };
+  take_iss();
   int bt_reg = 0;
   uint32_t k_iss = 0;
   int slot_iss = 0;
   auto issue_one = [&]() {
-    while (iss_live && iss_page >= iss.npages) {
-      iss_live = take(iss);
-      iss_page = 0;
-    }
+    while (iss_live && iss_page >= iss_np) take_iss();
     if (!iss_live) return;
     if ((iss_page & 31) == 0) {
       const int j = iss_page + lane;
-      bt_reg = j < iss.npages
-                   ? p.block_tables[static_cast<int64_t>(iss.b) * p.max_blocks_per_seq +
-                                    iss.tok0 / kBS + j]
-                   : 0;
+      bt_reg = j < iss_np ? p.block_tables[iss_tab + j] : 0;
     }
     const int blk = __shfl_sync(kFull, bt_reg, iss_page & 31);
     bool issue_copies = true;
@@ -278,18 +287,20 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     issue_copies = !(g_test_skip_first_copy && blockIdx.x == 0 && warp == 0 &&
                      k_iss == 0);
 #endif
-    if (lane == 0) mbar_arrive_expect_tx(&bars[slot_iss], kPageTx);
-    if (lane == 0 && issue_copies) {
-      const int s = slot_iss;
-      const int page = blk * p.num_kv_heads + iss.kvh;
-      uint8_t* tk = tiles + s * 2 * kCB;
-      tma_load_3d(tk, &tmk, 0, 0, page, &bars[s]);
-      tma_load_3d(tk + kCB, &tmv, 0, 0, page, &bars[s]);
-      float* sc = scl + s * 2 * kBS;
-      bulk_g2s(sc, p.k_scales + static_cast<int64_t>(page) * kBS,
-               kBS * sizeof(float), &bars[s]);
-      bulk_g2s(sc + kBS, p.v_scales + static_cast<int64_t>(page) * kBS,
-               kBS * sizeof(float), &bars[s]);
+    if (lane == 0) {
+      const uint32_t bar = bars_s + slot_iss * 8;
+      mbar_arrive_expect_tx_s(bar, kPageTx);
+      if (issue_copies) {
+        const int page = blk * p.num_kv_heads + iss_kvh;
+        const uint32_t tk = tiles_s + slot_iss * (2 * kCB);
+        const uint32_t sc = scl_s + slot_iss * (2 * kBS * 4);
+        tma_load_3d_s(tk, &tmk, 0, 0, page, bar);
+        tma_load_3d_s(tk + kCB, &tmv, 0, 0, page, bar);
+        bulk_g2s_s(sc, p.k_scales + static_cast<int64_t>(page) * kBS,
+                   kBS * sizeof(float), bar);
+        bulk_g2s_s(sc + kBS * 4, p.v_scales + static_cast<int64_t>(page) * kBS,
+                   kBS * sizeof(float), bar);
+      }
     }
     ++k_iss;
     ++iss_page;
@@ -312,17 +323,26 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
     const int64_t row0 = static_cast<int64_t>(cmp.b) * p.num_q_heads + cmp.kvh * G;
     math.init(p.q + row0 * kD, p.q_scale, lane);
     for (int j = 0; j < cmp.npages; ++j) {
-      if (!mbar_wait(&bars[slot], phase, &g_device_status)) {
+      if (!mbar_wait_s(bars_s + slot * 8, phase, &g_device_status)) {
         ok = false;
         break;
       }
-      const uint8_t* tk = tiles + slot * 2 * kCB;
-      const float* ks = scl + slot * 2 * kBS;
       const int nv = cmp.tok1 - (cmp.tok0 + j * kBS);
-      if (nv >= kBS)
-        math.template page<true>(tk, tk + kCB, ks, ks + kBS, kBS);
-      else
-        math.template page<false>(tk, tk + kCB, ks, ks + kBS, nv);
+      if constexpr (Math::kSharedAddr) {
+        const uint32_t tk = tiles_s + slot * (2 * kCB);
+        const uint32_t ks = scl_s + slot * (2 * kBS * 4);
+        if (nv >= kBS)
+          math.template page_s<true>(tk, tk + kCB, ks, ks + kBS * 4, kBS);
+        else
+          math.template page_s<false>(tk, tk + kCB, ks, ks + kBS * 4, nv);
+      } else {
+        const uint8_t* tk = tiles + slot * 2 * kCB;
+        const float* ks = scl + slot * 2 * kBS;
+        if (nv >= kBS)
+          math.template page<true>(tk, tk + kCB, ks, ks + kBS, kBS);
+        else
+          math.template page<false>(tk, tk + kCB, ks, ks + kBS, nv);
+      }
       __syncwarp();
       issue_one();
       ++k_cmp;

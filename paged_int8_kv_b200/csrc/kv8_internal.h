@@ -100,11 +100,14 @@ struct DecodeParams {
   int32_t partials_only;
 };
 
+
 // Extra launch facts of the shared-prefix kernel.
 struct PrefixShape {
   int32_t num_groups;
-  int32_t rounds;         // ceil(max members per group / 8)
-  int32_t prefix_chunks;  // max over groups of prefix_lens / chunk_tokens
+  int32_t max_group_size;  // host bound on the members of a group
+  int32_t rounds;          // set by launch_prefix: ceil(max_group_size /
+                           // members per round)
+  int32_t prefix_chunks;   // max over groups of prefix_lens / chunk_tokens
 };
 
 // Workspace carve-up shared by the decode and reduce launchers.

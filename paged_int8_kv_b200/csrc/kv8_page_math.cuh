@@ -97,6 +97,7 @@ struct SimtMath {
   static constexpr int kScratchBytes = 0;
   static constexpr int kTmemCols = 0;
   static constexpr int kCodeBytes = 2048;  // one page of K (or V) codes
+  static constexpr bool kSharedAddr = false;
   static constexpr int DPL = (G <= 4) ? 16 : 8;  // dims per lane
   static constexpr int LPT = kD / DPL;           // lanes per token
   static constexpr int TPP = 32 / LPT;           // tokens per pass
@@ -360,6 +361,7 @@ struct MmaMath {
   static constexpr int kScratchBytes = 0;
   static constexpr int kTmemCols = 0;
   static constexpr int kCodeBytes = 2048;  // one page of K (or V) codes
+  static constexpr bool kSharedAddr = false;
   static constexpr float kSlack = 8.0f;   // log2 units
   static constexpr int kVSlack = 4;
   int lane, r, c;
@@ -717,6 +719,25 @@ __device__ __forceinline__ void ldsm_x2_trans_b8(uint32_t addr, uint32_t& r0,
       : "memory");
 }
 
+// 16-byte shared-memory loads by 32-bit shared address (ordered like every
+// other volatile access: never hoisted above the wait for the page).
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 // Integer tensor-core form for groups of G <= 4 query heads: both products
 // on int8 mma, no code is converted on the CUDA cores.
 //   S[16 rows x 16 tok] = Qd[16 x 128] . K_code^T        (m16n8k32 s8, exact)
@@ -896,19 +917,28 @@ struct I8Math {
     zero_acc();
   }
 
+  static constexpr bool kSharedAddr = true;
+
   template <bool Full>
   __device__ __forceinline__ void page(const uint8_t* tk, const uint8_t* tv,
                                        const float* ks, const float* vs,
                                        int nv) {
+    page_s<Full>(smem_u32(tk), smem_u32(tv), smem_u32(ks), smem_u32(vs), nv);
+  }
+
+  // page() on 32-bit shared addresses (tk, tv: the K and V pages; ks, vs:
+  // their 16 scales)
+  template <bool Full>
+  __device__ __forceinline__ void page_s(uint32_t tk, uint32_t tv, uint32_t ks,
+                                         uint32_t vs, int nv) {
     // ---- S = Qd K^T.  n-tile j, column n = r: token 4(r/2) + 2j + r%2
-    const int ta = 4 * (r >> 1) + (r & 1), tb = ta + 2;
-    const uint8_t* ra = tk + ta * 128;
-    const uint8_t* rb = tk + tb * 128;
-    const int sw = ta & 7, swb = tb & 7;
-    const uint4 ka0 = *reinterpret_cast<const uint4*>(ra + (((2 * c) ^ sw) << 4));
-    const uint4 ka1 = *reinterpret_cast<const uint4*>(ra + (((2 * c + 1) ^ sw) << 4));
-    const uint4 kb0 = *reinterpret_cast<const uint4*>(rb + (((2 * c) ^ swb) << 4));
-    const uint4 kb1 = *reinterpret_cast<const uint4*>(rb + (((2 * c + 1) ^ swb) << 4));
+    const uint32_t ta = 4 * (r >> 1) + (r & 1), tb = ta + 2;
+    const uint32_t ra = tk + ta * 128, rb = tk + tb * 128;
+    const uint32_t sw = ta & 7, swb = tb & 7, c2 = 2 * c;
+    const uint4 ka0 = lds_u4(ra + ((c2 ^ sw) << 4));
+    const uint4 ka1 = lds_u4(ra + (((c2 + 1) ^ sw) << 4));
+    const uint4 kb0 = lds_u4(rb + ((c2 ^ swb) << 4));
+    const uint4 kb1 = lds_u4(rb + (((c2 + 1) ^ swb) << 4));
     int sacc[2][4];
 #pragma unroll
     for (int j = 0; j < 2; ++j)
@@ -935,8 +965,8 @@ struct I8Math {
                                      __int2float_rn(sacc[j][2 + e]) * wb);
         st[2 * j + e] = part + __shfl_xor_sync(kFull, part, 16);
       }
-    const float4 ks4 = *reinterpret_cast<const float4*>(ks + 4 * c);
-    const float4 vs4 = *reinterpret_cast<const float4*>(vs + 4 * c);
+    const float4 ks4 = lds_f4(ks + 16 * c);
+    const float4 vs4 = lds_f4(vs + 16 * c);
     const float ksv[4] = {ks4.x, ks4.y, ks4.z, ks4.w};
     const float vsr[4] = {vs4.x, vs4.y, vs4.z, vs4.w};
     float sc[4], vsv[4];
@@ -991,7 +1021,7 @@ struct I8Math {
 
     // ---- O^T += V^T Pd^T: ldmatrix rows = tokens 0..15 (lanes 0..15 and
     //      16..31 address the same tokens in m-tiles 2w and 2w+1)
-    const uint32_t vbase = smem_u32(tv) + (lane & 15) * 128;
+    const uint32_t vbase = tv + (lane & 15) * 128;
     const int vsw = lane & 7, vmt = lane >> 4;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -1245,17 +1275,27 @@ struct I4Math {
     zero_acc();
   }
 
+  static constexpr bool kSharedAddr = true;
+
   template <bool Full>
   __device__ __forceinline__ void page(const uint8_t* tk, const uint8_t* tv,
                                        const float* ks, const float* vs,
                                        int nv) {
+    page_s<Full>(smem_u32(tk), smem_u32(tv), smem_u32(ks), smem_u32(vs), nv);
+  }
+
+  // page() on 32-bit shared addresses (tk, tv: the K and V pages; ks, vs:
+  // their 16 scales)
+  template <bool Full>
+  __device__ __forceinline__ void page_s(uint32_t tk, uint32_t tv, uint32_t ks,
+                                         uint32_t vs, int nv) {
     // ---- S = Qd K^T: n-tile j, column n = r: token 4(r/2) + 2j + r%2;
     //      this thread's 16 bytes of a token t: row t/2, chunk 4(t%2) + c
-    const int ta = 4 * (r >> 1) + (r & 1), tb = ta + 2;
-    const uint4 pka = *reinterpret_cast<const uint4*>(
-        tk + (ta >> 1) * 128 + (((4 * (ta & 1) + c) ^ ((ta >> 1) & 7)) << 4));
-    const uint4 pkb = *reinterpret_cast<const uint4*>(
-        tk + (tb >> 1) * 128 + (((4 * (tb & 1) + c) ^ ((tb >> 1) & 7)) << 4));
+    const uint32_t ta = 4 * (r >> 1) + (r & 1), tb = ta + 2;
+    const uint4 pka =
+        lds_u4(tk + (ta >> 1) * 128 + (((4 * (ta & 1) + c) ^ ((ta >> 1) & 7)) << 4));
+    const uint4 pkb =
+        lds_u4(tk + (tb >> 1) * 128 + (((4 * (tb & 1) + c) ^ ((tb >> 1) & 7)) << 4));
     int sacc[2][4];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -1281,8 +1321,8 @@ struct I4Math {
                                      __int2float_rn(sacc[j][2 + e]) * wb);
         st[2 * j + e] = part + __shfl_xor_sync(kFull, part, 16);
       }
-    const float4 ks4 = *reinterpret_cast<const float4*>(ks + 4 * c);
-    const float4 vs4 = *reinterpret_cast<const float4*>(vs + 4 * c);
+    const float4 ks4 = lds_f4(ks + 16 * c);
+    const float4 vs4 = lds_f4(vs + 16 * c);
     const float ksv[4] = {ks4.x, ks4.y, ks4.z, ks4.w};
     const float vsr[4] = {vs4.x, vs4.y, vs4.z, vs4.w};
     float sc[4], vsv[4];
@@ -1338,7 +1378,7 @@ struct I4Math {
     // ---- O^T += V^T Pd^T: ldmatrix rows = tokens 0..15; lanes 0..15 take
     //      column chunk 2w, lanes 16..31 chunk 2w+1 (dims 32q..32q+31)
     const int vt = lane & 15, vq = lane >> 4;
-    const uint32_t vrow = smem_u32(tv) + (vt >> 1) * 128;
+    const uint32_t vrow = tv + (vt >> 1) * 128;
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       const int q = 2 * w + vq;

@@ -1,6 +1,7 @@
 // kv8_prefix.cu -- decode attention over the shared prefix of groups of
-// sequences: the pages several sequences list at the start of their block
-// tables are read, converted and scored once for the whole group.
+// sequences, on the 5th-generation tensor cores: the pages several sequences
+// list at the start of their block tables are read, converted and scored
+// once for all the group's query rows together.
 //
 // What is computed is unchanged from kv8_decode.cu [KV Cache 优化全景解析——
 // 从基础原理到工程实践, §2.1, §3.3]; what changes is how shared pages are
@@ -9,25 +10,21 @@
 // share a prefix so the shared part is handled once [garden.houmin.site
 // infra/kv-cache-optimize, §4.3.1 Prefix-aware Scheduling (BatchLLM)].
 //
-// Work decomposition: a work item is one (prefix chunk, KV head, group,
-// round of 8 members); a CTA of 8 warps takes items in turn (persistent
-// grid), warp w serving member 8 * round + w of the group:
-//   * warp 0 streams the chunk's pages (found through the block table of the
-//     group's first member) into a ring of 4 slots with TMA, across item
-//     boundaries, like the decode kernel's per-warp rings;
-//   * each page's V codes are converted once to fp16 in shared memory, 2
-//     tokens per warp, then a CTA barrier;
-//   * each active warp runs the warp tensor-core page math (MmaMath) for its
-//     member's G query heads on the shared K page and the converted V page;
-//   * at the end of an item each warp hands its member's chunk result to the
-//     same chunk partial / ticket / log-sum-exp merge as the decode kernel,
-//     so chunks computed here and the member's own chunks computed by the
-//     decode kernel merge into one output row, in either order.
+// For one shared chunk of the prefix and one KV head, the new tokens of the
+// group's members form a block of query rows -- member m, head h -- all
+// attending to the same keys: a dense contraction of up to 128 rows, which
+// is the extend kernel's tile.  A work item is (prefix chunk, KV head,
+// group, round of 128 / G members); the CTA runs the extend kernel's roles
+// (TMA producer, tcgen05 issuer, int8 -> fp16 converters, four softmax
+// warps, one row per thread) with no causal mask, and each row ends as the
+// member's chunk partial (m, l, o) in the split workspace.  It then takes
+// the member's merge ticket: chunks computed here and the member's own
+// chunks computed by the decode kernel merge into one output row by
+// log-sum-exp, in either order.
 #include "../../include/kv8.h"
 #include "kv8_common.cuh"
 #include "kv8_internal.h"
-#include "kv8_merge.cuh"
-#include "kv8_page_math.cuh"
+#include "kv8_tc.cuh"
 
 namespace kv8 {
 
@@ -35,264 +32,197 @@ __device__ uint32_t g_prefix_status = 0;
 
 namespace {
 
-constexpr int kPW = 8;     // warps per CTA = members per round
-constexpr int kPNB = 12;   // page slots in the CTA's ring (one CTA per SM:
-                           // 11 pages in flight)
-constexpr uint32_t kPTx = 2 * kPageBytes + 2 * kBS * sizeof(float);
+// Warp-wide scan of prefix_group: the sequence of rank `rank` (by sequence
+// index) among the members of group g, each lane with its own rank; -1
+// where the group has no member of that rank.
+__device__ __forceinline__ int member_of(const DecodeParams& p, int g, int rank,
+                                         int lane) {
+  int found = -1, seen = 0;
+  for (int base = 0; base < p.batch; base += 32) {
+    const int b = base + lane;
+    const int v = b < p.batch ? p.prefix_group[b] : -1;
+    const uint32_t m = __ballot_sync(kFull, v == g);
+    const int cnt = __popc(m);
+    if (found < 0 && rank >= seen && rank < seen + cnt)
+      found = base + static_cast<int>(__fns(m, 0, rank - seen + 1));
+    seen += cnt;
+    if (__all_sync(kFull, rank < seen)) break;
+  }
+  return found;
+}
 
-// Shared memory (base aligned to 1024 bytes for the 128-byte swizzle):
-//   [kPNB][K page 2048 | V page 2048]   TMA-staged int8 pages
-//   [2][4096]                           V page as fp16 [16 tok][128 dims], by
-//                                       page parity (page k's copy is free
-//                                       once every warp is past page k+1's
-//                                       barrier)
-//   [kPNB][ks 64 | vs 64]               scales
-//   [kPNB] mbarriers; two ints: a wait gave up, the first page not waited for
-struct PrefixPlan {
-  static constexpr int kTiles = 0;
-  static constexpr int kVh = kTiles + kPNB * 2 * kPageBytes;
-  static constexpr int kScl = kVh + 2 * 4096;
-  static constexpr int kBar = kScl + kPNB * 2 * kBS * 4;
-  static constexpr int kFail = kBar + kPNB * 8;
-  static constexpr int kBytes = kFail + 16 + 1024;
-};
-
+// Item idx = ((chunk * H_kv + kvh) * groups + g) * rounds + rnd.
 struct PrefixItem {
   int chunk, kvh, g, rnd;
-  int tok0, npages;
 };
-
-// Item idx, numbered chunk-major: idx = ((chunk * H_kv + kvh) * groups + g)
-// * rounds + rnd.  False if the chunk is not a whole chunk of the group's
-// prefix.
 __device__ __forceinline__ bool pitem_load(const DecodeParams& p,
-                                           const PrefixShape& ps, int64_t idx,
-                                           PrefixItem& it) {
+                                           const PrefixShape& ps, int members,
+                                           int64_t idx, PrefixItem& it,
+                                           int& first, int lane) {
   it.rnd = static_cast<int>(idx % ps.rounds);
   idx /= ps.rounds;
   it.g = static_cast<int>(idx % ps.num_groups);
   idx /= ps.num_groups;
   it.kvh = static_cast<int>(idx % p.num_kv_heads);
   it.chunk = static_cast<int>(idx / p.num_kv_heads);
-  const int whole = p.prefix_lens[it.g] / p.chunk_tokens;
-  if (it.chunk >= whole) return false;
-  it.tok0 = it.chunk * p.chunk_tokens;
-  it.npages = p.chunk_tokens / kBS;
-  return true;
+  if (it.chunk >= p.prefix_lens[it.g] / p.chunk_tokens) return false;
+  // lane 0: the group's first member (its table lists the prefix blocks);
+  // lane 1: the round's first member (none: the round is empty)
+  const int b = member_of(p, it.g, lane == 1 ? members * it.rnd : 0, lane);
+  first = __shfl_sync(kFull, b, 0);
+  return __shfl_sync(kFull, b, 1) >= 0;
 }
 
-// Warp-wide scan of prefix_group for group g: the first member (by sequence
-// index) and the members of rank `mine` and `lead` (-1 where there is none).
-__device__ __forceinline__ void find_members(const DecodeParams& p, int g,
-                                             int mine, int lead, int lane,
-                                             int& first, int& b_mine,
-                                             int& b_lead) {
-  first = b_mine = b_lead = -1;
-  int seen = 0;
-  for (int base = 0; base < p.batch; base += 32) {
-    const int b = base + lane;
-    const int v = b < p.batch ? p.prefix_group[b] : -1;
-    const uint32_t m = __ballot_sync(kFull, v == g);
-    const int cnt = __popc(m);
-    if (m) {
-      if (first < 0) first = base + __ffs(m) - 1;
-      if (b_mine < 0 && mine < seen + cnt)
-        b_mine = base + static_cast<int>(__fns(m, 0, mine - seen + 1));
-      if (b_lead < 0 && lead < seen + cnt)
-        b_lead = base + static_cast<int>(__fns(m, 0, lead - seen + 1));
-    }
-    seen += cnt;
-    if (b_mine >= 0 && b_lead >= 0) break;
+// The prefix items as the producer, issuer and converter roles see them.
+struct PrefixItems {
+  const DecodeParams& p;
+  const PrefixShape& ps;
+  int members;  // per round: 128 / G
+  __device__ __forceinline__ int64_t size() const {
+    return static_cast<int64_t>(ps.prefix_chunks) * p.num_kv_heads *
+           ps.num_groups * ps.rounds;
   }
-}
-
-// Bounded wait for page k; once any wait of the CTA has given up, later
-// waits are skipped (the launch then only has to finish; the status word
-// reports it) and the first page not waited for is recorded in fail[1].
-__device__ __forceinline__ void pwait(uint64_t* bar, uint32_t parity,
-                                      uint32_t k, volatile int* fail) {
-  if (!fail[0] && mbar_wait(bar, parity, &g_prefix_status)) return;
-  fail[0] = 1;
-  atomicMin(const_cast<int*>(&fail[1]), static_cast<int>(k));
-}
+  __device__ __forceinline__ bool load(int64_t idx, TileItem& t, int lane) const {
+    PrefixItem it;
+    int first;
+    if (!pitem_load(p, ps, members, idx, it, first, lane)) return false;
+    t.tab = static_cast<int64_t>(first) * p.max_blocks_per_seq +
+            it.chunk * (p.chunk_tokens / kBS);
+    t.kvh = it.kvh;
+    t.npages = p.chunk_tokens / kBS;
+    t.nkt = (p.chunk_tokens + kKT - 1) / kKT;
+    return true;
+  }
+};
 
 template <int G>
-__global__ void __launch_bounds__(kPW * 32, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 prefix_kernel(const DecodeParams p, const PrefixShape ps,
               const __grid_constant__ CUtensorMap tmk,
               const __grid_constant__ CUtensorMap tmv) {
+  constexpr int M = kRows / G;  // members per round
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  uint8_t* tiles = smem + PrefixPlan::kTiles;
-  uint8_t* vh = smem + PrefixPlan::kVh;
-  float* scl = reinterpret_cast<float*>(smem + PrefixPlan::kScl);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PrefixPlan::kBar);
-  volatile int* fail = reinterpret_cast<volatile int*>(smem + PrefixPlan::kFail);
-  if (threadIdx.x == 0) {
-    prefetch_tensormap(&tmk);
-    prefetch_tensormap(&tmv);
-    for (int s = 0; s < kPNB; ++s) mbar_init(&bars[s], 1);
-    fail[0] = 0;
-    fail[1] = 0x7fffffff;
-    fence_mbar_init();
-  }
-  __syncthreads();
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ExtPlan::kBar);
+  const uint32_t tmem = tc_setup(smem, &tmk, &tmv, warp);
+  bool failed = false;
 
-  const int64_t n_items = static_cast<int64_t>(ps.prefix_chunks) *
-                          p.num_kv_heads * ps.num_groups * ps.rounds;
-  const int64_t stride = gridDim.x;
-
-  // ---- issue cursor (warp 0): kPNB pages ahead, across items
-  int64_t iss_idx = blockIdx.x;
-  PrefixItem iss;
-  int iss_page = 0, iss_first = -1, bt_reg = 0;
-  bool iss_live = false;
-  uint32_t k_iss = 0;
-  auto iss_seek = [&]() {  // warp 0: the next item with pages, or none
-    for (; iss_idx < n_items; iss_idx += stride) {
-      if (!pitem_load(p, ps, iss_idx, iss)) continue;
-      int b_mine, b_lead;
-      find_members(p, iss.g, 0, 8 * iss.rnd, lane, iss_first, b_mine, b_lead);
-      if (b_lead >= 0) {
-        iss_live = true;
-        iss_page = 0;
-        return;
-      }
-    }
-    iss_live = false;
-  };
-  auto issue_one = [&]() {  // warp 0
-    if (!iss_live || __any_sync(kFull, fail[0] != 0)) return;
-    if ((iss_page & 31) == 0) {
-      const int j = iss_page + lane;
-      bt_reg = j < iss.npages
-                   ? p.block_tables[static_cast<int64_t>(iss_first) * p.max_blocks_per_seq +
-                                    iss.tok0 / kBS + j]
-                   : 0;
-    }
-    const int blk = __shfl_sync(kFull, bt_reg, iss_page & 31);
-    if (lane == 0) {
-      const int s = k_iss % kPNB;
-      const int page = blk * p.num_kv_heads + iss.kvh;
-      mbar_arrive_expect_tx(&bars[s], kPTx);
-      uint8_t* tk = tiles + s * 2 * kPageBytes;
-      tma_load_3d(tk, &tmk, 0, 0, page, &bars[s]);
-      tma_load_3d(tk + kPageBytes, &tmv, 0, 0, page, &bars[s]);
-      float* sc = scl + s * 2 * kBS;
-      bulk_g2s(sc, p.k_scales + static_cast<int64_t>(page) * kBS,
-               kBS * sizeof(float), &bars[s]);
-      bulk_g2s(sc + kBS, p.v_scales + static_cast<int64_t>(page) * kBS,
-               kBS * sizeof(float), &bars[s]);
-    }
-    ++k_iss;
-    if (++iss_page == iss.npages) {
-      iss_idx += stride;
-      iss_seek();
-    }
-  };
+  const PrefixItems items{p, ps, M};
   if (warp == 0) {
-    iss_seek();
-    for (int s = 0; s < kPNB; ++s) issue_one();
-  }
+    tc_produce(items, p.block_tables, p.num_kv_heads, p.k_scales, p.v_scales,
+               &tmk, &tmv, smem, bars, failed, &g_prefix_status, lane);
+  } else if (warp == 1) {
+    tc_issue(items, smem, bars, tmem, failed, &g_prefix_status, lane);
+  } else if (warp < 4) {
+    tc_convert(items, smem, bars, failed, &g_prefix_status, threadIdx.x - 64,
+               lane);
+  } else {
+    // ================================================= softmax (4 warps)
+    // row r = member r / G of the round, head r % G; a member's G rows lie
+    // in one warp
+    const int r = threadIdx.x - 128;  // row = tensor-memory lane
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    const int mr = r / G, head = r % G;
+    uint8_t* q16 = smem + ExtPlan::kQ16;
+    const int nkt = (p.chunk_tokens + kKT - 1) / kKT;
+    uint32_t u = 0;
+    const int64_t n = items.size();
+    for (int64_t idx = blockIdx.x; idx < n; idx += gridDim.x) {
+      PrefixItem it;
+      int first;
+      if (!pitem_load(p, ps, M, idx, it, first, lane)) continue;
+      const int b = member_of(p, it.g, M * it.rnd + mr, lane);
+      const int tok0 = it.chunk * p.chunk_tokens;
+      int n_b = 0;
+      bool live = false;
+      if (b >= 0) {
+        n_b = p.context_lens[b];
+        live = n_b >= tok0 + p.chunk_tokens;
+        if (!live && head == 0) atomicOr(&g_prefix_status, KV8_DEV_BAD_PREFIX);
+      }
+      const int64_t row =
+          static_cast<int64_t>(live ? b : 0) * p.num_q_heads + it.kvh * G + head;
+      const float qf = tc_stage_q(p.q + row * kD, live, r, q16, p.q_scale);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_Q_FULL]);
 
-  MmaMath<G, true> math;
-  math.attach(nullptr);
-  uint32_t k = 0;  // pages consumed by this CTA
-  for (int64_t idx = blockIdx.x; idx < n_items; idx += stride) {
-    PrefixItem it;
-    if (!pitem_load(p, ps, idx, it)) continue;
-    int first, b_w, b_lead;
-    find_members(p, it.g, 8 * it.rnd + warp, 8 * it.rnd, lane, first, b_w,
-                 b_lead);
-    if (b_lead < 0) continue;  // the same decision in every warp
-    int n_w = 0;
-    if (b_w >= 0) {
-      n_w = p.context_lens[b_w];
-      if (n_w < it.tok0 + p.chunk_tokens) {  // shorter than the prefix
-        if (lane == 0) atomicOr(&g_prefix_status, KV8_DEV_BAD_PREFIX);
-        b_w = -1;
+      // ---- the chunk's keys, all visible to every row
+      const RowSoftmax rs = tc_row_tiles(smem, bars, trow, r, lane, live,
+                                         p.chunk_tokens, qf, nkt, u, failed,
+                                         &g_prefix_status);
+      u += nkt;
+      ewait(&bars[B_O_DONE], (u - 1) & 1, failed, &g_prefix_status);
+      __syncwarp();
+      tc_fence_after();
+
+      // ---- the row's chunk result: the member's output row when the chunk
+      // is its whole context, else its chunk partial (m, l, o), o relative to
+      // m and unnormalised
+      const int nchunks = (n_b + p.chunk_tokens - 1) / p.chunk_tokens;
+      const bool single = nchunks <= 1;
+      const float f = single ? pow2i(rs.e) / (rs.l > 0.0f ? rs.l : 1.0f)
+                             : pow2i(rs.e);
+      const int64_t ci = row * p.max_chunks + it.chunk;
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        float o[32];
+        __syncwarp();  // the stores below diverge by row; reconverge first
+        tmem_ld32(trow + kColO + 32 * c, o);
+        if (!live) continue;
+        if (!single) {
+          float4* dst = reinterpret_cast<float4*>(p.ws_o + ci * kD + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(o[4 * i] * f, o[4 * i + 1] * f,
+                                 o[4 * i + 2] * f, o[4 * i + 3] * f);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            store_out(p.out, row * kD + 32 * c + i, o[i] * f, p.out_f32);
+        }
       }
-    }
-    const int64_t row0 =
-        static_cast<int64_t>(b_w < 0 ? 0 : b_w) * p.num_q_heads + it.kvh * G;
-    if (b_w >= 0) math.init(p.q + row0 * kD, p.q_scale, lane);
-    for (int j = 0; j < it.npages; ++j, ++k) {
-      const int s = k % kPNB;
-      pwait(&bars[s], (k / kPNB) & 1, k, fail);
-      // V page -> fp16 [16 tok][128 dims]: warp w converts tokens 2w, 2w+1;
-      // lane = (token, 16-byte code chunk, half)
-      {
-        const int t = 2 * warp + (lane >> 4);
-        const int cj = (lane & 15) >> 1, hf = lane & 1;
-        const uint8_t* src = tiles + s * 2 * kPageBytes + kPageBytes + t * 128 +
-                             ((cj ^ (t & 7)) << 4) + 8 * hf;
-        const uint2 w8 = *reinterpret_cast<const uint2*>(src);
-        const uint32_t x0 = w8.x ^ 0x80808080u, x1 = w8.y ^ 0x80808080u;
-        uint4 o;
-        o.x = hsub2_u32(prmt(x0, 0x64646464u, 0x4140u), kBias1152);
-        o.y = hsub2_u32(prmt(x0, 0x64646464u, 0x4342u), kBias1152);
-        o.z = hsub2_u32(prmt(x1, 0x64646464u, 0x4140u), kBias1152);
-        o.w = hsub2_u32(prmt(x1, 0x64646464u, 0x4342u), kBias1152);
-        const int ch = 2 * cj + hf;  // fp16 chunk: dims 8ch .. 8ch+7
-        *reinterpret_cast<uint4*>(vh + (k & 1) * 4096 + t * 256 + ((ch ^ (t & 7)) << 4)) = o;
+      if (live && !single) {
+        p.ws_ml[2 * ci] = rs.m;
+        p.ws_ml[2 * ci + 1] = rs.l;
       }
-      __syncthreads();
-      // every warp is past page k-1: its slot is free for page k-1+kPNB
-      if (warp == 0 && k >= 1) issue_one();
-      if (b_w >= 0) {
-        const uint8_t* tk = tiles + s * 2 * kPageBytes;
-        const float* ks = scl + s * 2 * kBS;
-        uint32_t h0, h2, g0, g2;
-        math.template qk_softmax<true>(tk, ks, ks + kBS, kBS, h0, h2, g0, g2);
-        math.pv_f16(smem_u32(vh + (k & 1) * 4096), h0, h2, g0, g2);
-      }
-    }
-    if (b_w < 0) continue;
-    // ---- this member's chunk: partial (or the output row), ticket, merge
-    const int nchunks = (n_w + p.chunk_tokens - 1) / p.chunk_tokens;
-    ChunkSink sk;
-    sk.out = p.out;
-    sk.ws_o = p.ws_o;
-    sk.ws_ml = p.ws_ml;
-    sk.row0 = row0;
-    sk.ci0 = row0 * p.max_chunks + it.chunk;
-    sk.max_chunks = p.max_chunks;
-    sk.single = nchunks <= 1;
-    sk.out_f32 = p.out_f32;
-    math.finish(sk);
-    if (!sk.single) {
+      tc_fence_before();
+
+      // ---- each member's ticket (taken by its head-0 row once the G rows
+      // are written); the last of the member's chunks merges them
       __threadfence();
       __syncwarp();
+      const bool lead = live && !single && head == 0;
       unsigned int ticket = 0;
-      if (lane == 0) ticket = atomicAdd(&p.ws_ctr[row0], 1u);
-      ticket = __shfl_sync(kFull, ticket, 0);
-      if (ticket == static_cast<unsigned int>(nchunks - 1)) {
+      if (lead) ticket = atomicAdd(&p.ws_ctr[row], 1u);
+      uint32_t mm = __ballot_sync(
+          kFull, lead && ticket == static_cast<unsigned int>(nchunks - 1));
+      while (mm) {
+        const int src = __ffs(mm) - 1;
+        mm &= mm - 1;
+        const int bs = __shfl_sync(kFull, b, src);
+        const int nch = __shfl_sync(kFull, nchunks, src);
+        const int64_t r0 = static_cast<int64_t>(bs) * p.num_q_heads + it.kvh * G;
         __threadfence();
         for (int h = 0; h < G; ++h)
-          merge_head_warp(p.ws_ml + (row0 + h) * p.max_chunks * 2,
-                          p.ws_o + (row0 + h) * p.max_chunks * kD, nchunks,
-                          p.out, row0 + h, p.out_f32);
+          merge_head_warp(p.ws_ml + (r0 + h) * p.max_chunks * 2,
+                          p.ws_o + (r0 + h) * p.max_chunks * kD, nch, p.out,
+                          r0 + h, p.out_f32);
       }
     }
   }
-  // a wait gave up: wait (bounded) for every copy that may still be in
-  // flight (pages from the first one not waited for), then stop
-  __syncthreads();
-  if (fail[0] && warp == 0 && lane == 0) {
-    for (uint32_t kk = static_cast<uint32_t>(fail[1]); kk < k_iss; ++kk)
-      mbar_wait(&bars[kk % kPNB], (kk / kPNB) & 1, &g_prefix_status);
-  }
+  tc_teardown(tmem, warp);
 }
 
 template <int G>
-int launch_prefix_group(const DecodeParams& p, const PrefixShape& ps,
+int launch_prefix_group(const DecodeParams& p, PrefixShape ps,
                         const CUtensorMap& tmk, const CUtensorMap& tmv,
                         cudaStream_t stream) {
   auto kern = prefix_kernel<G>;
-  constexpr int smem = PrefixPlan::kBytes;
+  constexpr int smem = ExtPlan::kBytes;
   static LaunchFacts table[kMaxDevices];
   LaunchFacts* f = facts_for_current_device(table);
   if (!f) return -1;
@@ -309,12 +239,14 @@ int launch_prefix_group(const DecodeParams& p, const PrefixShape& ps,
     f->resident.store(1, std::memory_order_release);
     f->sms.store(sms, std::memory_order_release);
   }
+  constexpr int M = kRows / G;
+  ps.rounds = (ps.max_group_size + M - 1) / M;
   const int64_t n_items = static_cast<int64_t>(ps.prefix_chunks) *
                           p.num_kv_heads * ps.num_groups * ps.rounds;
   if (n_items == 0) return 0;
   int64_t ctas = sms;
   if (ctas > n_items) ctas = n_items;
-  kern<<<static_cast<unsigned>(ctas), kPW * 32, smem, stream>>>(p, ps, tmk, tmv);
+  kern<<<static_cast<unsigned>(ctas), kThreads, smem, stream>>>(p, ps, tmk, tmv);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -1,12 +1,17 @@
 """kv8_paged_decode_attention_prefix on the GPU (through the C ABI).
 
 Groups of sequences that share the blocks at the start of their block tables
-are decoded with the shared pages read and scored once per group; the
-results must be those of the plain decode call:
+are decoded with the shared pages read and scored once per group (on the
+tcgen05 tensor cores, all the group's query rows together).  The shared
+chunks' probabilities are rounded to fp16, as in extend attention, so the
+bound is the decode tolerance |gpu - oracle| <= 2e-3 (plus half a bf16 ulp
+for bf16 output) and not the 1e-4 the all-integer decode form keeps; the
+mean error stays below 1e-4 (a misplaced row, key or head would not):
   * the prefix-shared workload (6 groups x 8 sequences, 4096-token prefix,
     64 q / 8 KV heads), every (sequence, head) against the oracle, fp32 and
-    bf16 output, and against the plain call within 1e-5;
-  * ragged cases: group sizes 1, 3, 8 and 11 (more than one round of 8),
+    bf16 output, and against the plain call within 2e-3;
+  * ragged cases: group sizes 1, 3, 8 and 11, a group of 20 members at 8
+    query heads per KV head (two rounds of 16 members),
     sequences in no group, prefixes that are not a whole number of chunks,
     a member whose whole context is the prefix, every group size G;
   * a member shorter than its group's prefix sets bit 1 of the device
@@ -64,9 +69,9 @@ def test_prefix_shared_workload(pk, oracle_mod, chunk):
         got = _prefix_decode(pk, cache, q, bt, cl, w, groups, plens, chunk, dt)
         U.assert_close(got, ref, bf16=bf)
         if not bf:
-            assert np.abs(got - ref).max() < 1e-4
+            assert np.abs(got - ref).mean() < 1e-4
             plain = U.gpu_decode(cache, q, bt, cl, w, chunk_tokens=chunk)
-            assert np.abs(got - plain).max() <= 1e-5
+            assert np.abs(got - plain).max() <= 2e-3
 
 
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (8, 2), (16, 2)])
@@ -112,7 +117,38 @@ def test_prefix_ragged_groups(pk, oracle_mod, hq, hkv):
         got = _prefix_decode(pk, cache, q, btd, cl, w, grp, plens, chunk,
                              torch.float32)
         U.assert_close(got, ref, bf16=False)
-        assert np.abs(got - ref).max() < 1e-4
+        assert np.abs(got - ref).mean() < 1e-4
+
+
+def test_prefix_two_rounds(pk, oracle_mod):
+    # 20 members at G = 8: rows of 16 members per item, so two rounds
+    grp = [0] * 20 + [-1]
+    plen = 128
+    lens = [plen + s for s in range(5, 105, 5)] + [70]
+    w = W.make_workload("pfx2", 6300, lens, 16, 2, extra_blocks=4,
+                        chunk_tokens=64)
+    bt = w.block_tables.copy()
+    for b in range(1, 20):
+        bt[b, :plen // 16] = bt[0, :plen // 16]
+    w.block_tables = bt
+    base = w.private_kv
+
+    def kv(b, _base=base):
+        k, v = _base(b)
+        if 0 < b < 20:
+            k0, v0 = _base(0)
+            k = np.concatenate([k0[:plen], k[plen:]])
+            v = np.concatenate([v0[:plen], v[plen:]])
+        return k, v
+    w.private_kv = kv
+    cache, q, btd, cl = U.device_inputs(w)
+    kc, vc, ks, vs = U.oracle_full_cache(oracle_mod, w)
+    ref = oracle_mod.decode_attention(w.q(), kc, vc, ks, vs, w.block_tables,
+                                      w.context_lens)
+    got = _prefix_decode(pk, cache, q, btd, cl, w, grp, [plen], 64,
+                         torch.float32)
+    U.assert_close(got, ref, bf16=False)
+    assert np.abs(got - ref).mean() < 1e-4
 
 
 def test_prefix_member_shorter_than_prefix_sets_status(pk):
