@@ -131,12 +131,14 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
   } else if (warp < 4) {
     tc_convert(items, smem, bars, failed, &g_ext_status, threadIdx.x - 64, lane);
   } else {
-    // ================================================= softmax (4 warps)
-    const int r = threadIdx.x - 128;  // row = tensor-memory lane
-    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    // ================================================= softmax (8 warps)
+    // rows r = 32 qd + lane (tensor-memory lane quarter qd); half hf takes
+    // key columns and output dims 64 hf .. 64 hf + 63
+    const int sw = warp - 4, qd = sw & 3, hf = sw >> 2;
+    const int r = 32 * qd + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * qd) << 16);
     const int pos = r / G, head = r % G;
-    uint8_t* q16 = smem + ExtPlan::kQ16;
-    uint32_t u = 0;
+    uint32_t u = 0, xk = 0;
     for (int64_t idx = blockIdx.x; idx < n_items; idx += gridDim.x) {
       ExtItem it;
       if (!eitem_load(p, idx, P, it)) continue;
@@ -144,37 +146,42 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
       const int64_t qrow =
           static_cast<int64_t>(p.q_start[it.b] + it.i0 + pos) * p.num_q_heads +
           it.kvh * G + head;
-      const float qf = tc_stage_q(p.q + qrow * kD, live, r, q16, p.q_scale);
+      const float qf =
+          tc_stage_q(smem, p.q + qrow * kD, live, r, hf, qd, p.q_scale, xk);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_Q_FULL]);
 
       // ---- key tiles
       const int key_lim = it.t_ctx - it.n_new + it.i0 + pos + 1;  // keys < this
-      const RowSoftmax rs = tc_row_tiles(smem, bars, trow, r, lane, live, key_lim,
-                                         qf, it.nkt, u, failed, &g_ext_status);
+      const RowSoftmax rs =
+          tc_row_tiles(smem, bars, trow, r, hf, qd, lane, live, key_lim, qf,
+                       it.nkt, u, xk, failed, &g_ext_status);
       u += it.nkt;
-      // ---- output: wait for the last O product, normalise, store
+      const float l = rs.l + pair_xch(smem, xk, hf, r, qd, make_float2(rs.l, 0.0f)).x;
+      // ---- output: wait for the last O product, normalise, store this
+      // half's dims
       ewait(&bars[B_O_DONE], (u - 1) & 1, failed, &g_ext_status);
       __syncwarp();
       tc_fence_after();
-      const float f = pow2i(rs.e) / (rs.l > 0.0f ? rs.l : 1.0f);
+      const float f = pow2i(rs.e) / (l > 0.0f ? l : 1.0f);
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = 0; c < kHalf / 32; ++c) {
         float o[32];
+        const int d0 = kHalf * hf + 32 * c;
         __syncwarp();  // the stores below diverge by row; reconverge first
-        tmem_ld32(trow + kColO + 32 * c, o);
+        tmem_ld32(trow + kColO + d0, o);
         if (live) {
           if (p.out_f32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) +
-                                                    qrow * kD + 32 * c);
+                                                    qrow * kD + d0);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               dst[i] = make_float4(o[4 * i] * f, o[4 * i + 1] * f,
                                    o[4 * i + 2] * f, o[4 * i + 3] * f);
           } else {
             uint4* dst = reinterpret_cast<uint4*>(
-                static_cast<__nv_bfloat16*>(p.out) + qrow * kD + 32 * c);
+                static_cast<__nv_bfloat16*>(p.out) + qrow * kD + d0);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               uint32_t w[4];

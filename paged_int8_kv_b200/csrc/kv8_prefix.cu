@@ -120,15 +120,16 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
     tc_convert(items, smem, bars, failed, &g_prefix_status, threadIdx.x - 64,
                lane);
   } else {
-    // ================================================= softmax (4 warps)
-    // row r = member r / G of the round, head r % G; a member's G rows lie
-    // in one warp
-    const int r = threadIdx.x - 128;  // row = tensor-memory lane
-    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    // ================================================= softmax (8 warps)
+    // row r = 32 qd + lane = member r / G of the round, head r % G (a
+    // member's G rows lie in one warp); half hf takes key columns and output
+    // dims 64 hf .. 64 hf + 63
+    const int sw = warp - 4, qd = sw & 3, hf = sw >> 2;
+    const int r = 32 * qd + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * qd) << 16);
     const int mr = r / G, head = r % G;
-    uint8_t* q16 = smem + ExtPlan::kQ16;
     const int nkt = (p.chunk_tokens + kKT - 1) / kKT;
-    uint32_t u = 0;
+    uint32_t u = 0, xk = 0;
     const int64_t n = items.size();
     for (int64_t idx = blockIdx.x; idx < n; idx += gridDim.x) {
       PrefixItem it;
@@ -141,40 +142,43 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
       if (b >= 0) {
         n_b = p.context_lens[b];
         live = n_b >= tok0 + p.chunk_tokens;
-        if (!live && head == 0) atomicOr(&g_prefix_status, KV8_DEV_BAD_PREFIX);
+        if (!live && head == 0 && hf == 0)
+          atomicOr(&g_prefix_status, KV8_DEV_BAD_PREFIX);
       }
       const int64_t row =
           static_cast<int64_t>(live ? b : 0) * p.num_q_heads + it.kvh * G + head;
-      const float qf = tc_stage_q(p.q + row * kD, live, r, q16, p.q_scale);
+      const float qf =
+          tc_stage_q(smem, p.q + row * kD, live, r, hf, qd, p.q_scale, xk);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_Q_FULL]);
 
       // ---- the chunk's keys, all visible to every row
-      const RowSoftmax rs = tc_row_tiles(smem, bars, trow, r, lane, live,
-                                         p.chunk_tokens, qf, nkt, u, failed,
-                                         &g_prefix_status);
+      const RowSoftmax rs =
+          tc_row_tiles(smem, bars, trow, r, hf, qd, lane, live, p.chunk_tokens,
+                       qf, nkt, u, xk, failed, &g_prefix_status);
       u += nkt;
+      const float l = rs.l + pair_xch(smem, xk, hf, r, qd, make_float2(rs.l, 0.0f)).x;
       ewait(&bars[B_O_DONE], (u - 1) & 1, failed, &g_prefix_status);
       __syncwarp();
       tc_fence_after();
 
-      // ---- the row's chunk result: the member's output row when the chunk
-      // is its whole context, else its chunk partial (m, l, o), o relative to
-      // m and unnormalised
+      // ---- the row's chunk result (this half's dims): the member's output
+      // row when the chunk is its whole context, else its chunk partial
+      // (m, l, o), o relative to m and unnormalised
       const int nchunks = (n_b + p.chunk_tokens - 1) / p.chunk_tokens;
       const bool single = nchunks <= 1;
-      const float f = single ? pow2i(rs.e) / (rs.l > 0.0f ? rs.l : 1.0f)
-                             : pow2i(rs.e);
+      const float f = single ? pow2i(rs.e) / (l > 0.0f ? l : 1.0f) : pow2i(rs.e);
       const int64_t ci = row * p.max_chunks + it.chunk;
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = 0; c < kHalf / 32; ++c) {
         float o[32];
+        const int d0 = kHalf * hf + 32 * c;
         __syncwarp();  // the stores below diverge by row; reconverge first
-        tmem_ld32(trow + kColO + 32 * c, o);
+        tmem_ld32(trow + kColO + d0, o);
         if (!live) continue;
         if (!single) {
-          float4* dst = reinterpret_cast<float4*>(p.ws_o + ci * kD + 32 * c);
+          float4* dst = reinterpret_cast<float4*>(p.ws_o + ci * kD + d0);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             dst[i] = make_float4(o[4 * i] * f, o[4 * i + 1] * f,
@@ -182,20 +186,21 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            store_out(p.out, row * kD + 32 * c + i, o[i] * f, p.out_f32);
+            store_out(p.out, row * kD + d0 + i, o[i] * f, p.out_f32);
         }
       }
-      if (live && !single) {
+      if (live && !single && hf == 0) {
         p.ws_ml[2 * ci] = rs.m;
-        p.ws_ml[2 * ci + 1] = rs.l;
+        p.ws_ml[2 * ci + 1] = l;
       }
       tc_fence_before();
 
-      // ---- each member's ticket (taken by its head-0 row once the G rows
-      // are written); the last of the member's chunks merges them
+      // ---- each member's ticket, taken by its head-0 row of half 0 once
+      // both halves of the member's G rows are written; the last of the
+      // member's chunks merges them
       __threadfence();
-      __syncwarp();
-      const bool lead = live && !single && head == 0;
+      pair_sync(qd);
+      const bool lead = live && !single && head == 0 && hf == 0;
       unsigned int ticket = 0;
       if (lead) ticket = atomicAdd(&p.ws_ctr[row], 1u);
       uint32_t mm = __ballot_sync(

@@ -21,7 +21,11 @@ constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kKT = 128;              // keys per tile
 constexpr int kTilePages = kKT / kBS;  // 8
 constexpr int kRows = 128;            // query rows per item (MMA M)
-constexpr int kThreads = 256;
+// warps: 0 TMA producer, 1 MMA issuer, 2-3 converters, 4-11 softmax (two
+// per tensor-memory lane quarter: warp 4 + q and 8 + q hold the same 32 rows,
+// one the key columns / output dims 0..63, the other 64..127)
+constexpr int kThreads = 384;
+constexpr int kHalf = 64;             // columns per softmax thread
 constexpr int kTmemCols = 512;        // S[2] (256) + O (128), power of two
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr float kSlack = 8.0f;        // scores may pass m by 2^8 before m moves
@@ -37,7 +41,10 @@ struct ExtPlan {
   static constexpr int kP16 = kQ16 + kOpBytes;
   static constexpr int kStageScl = kP16 + kOpBytes;         // [2][ks 128 | vs 128]
   static constexpr int kScl = kStageScl + 2 * 2 * kKT * 4;  // [4][ks 128 | vs 128]
-  static constexpr int kBar = kScl + 4 * 2 * kKT * 4;
+  // the two softmax halves of a row exchange per-row values here:
+  // [2 tile parities][2 halves][128 rows] float2
+  static constexpr int kXch = kScl + 4 * 2 * kKT * 4;
+  static constexpr int kBar = kXch + 2 * 2 * kRows * 8;
   // st_full[2] st_empty[2] k16_full k16_empty v16_full v16_empty s_full[2]
   // s_empty[2] p_full o_done q_full
   static constexpr int kBarCount = 15;
@@ -126,6 +133,12 @@ __device__ __forceinline__ float4 lds_f4v(uint32_t addr) {
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr)
                : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float lds_f1v(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
 }
 
@@ -400,34 +413,54 @@ __device__ __forceinline__ void tc_convert(const Items& items, uint8_t* smem,
   }
 }
 
-// A softmax thread's query row r, staged for the q.k product: q (bf16,
-// [128]; read only when live) times an exact power of two into fp16 (max
-// |q| 2^sh in [2^14, 2^15): exact), written to row r of the Q16 operand.
-// Returns the factor that turns an S entry back into a base-2 score.
-__device__ __forceinline__ float tc_stage_q(const __nv_bfloat16* qptr, bool live,
-                                            int r, uint8_t* q16, float q_scale) {
-  // ---- q row -> fp16 x 2^sh (max |q| 2^sh in [2^14, 2^15): exact), in
-  // two passes over the row (its max, then the conversion)
-  const uint4* qsrc = reinterpret_cast<const uint4*>(qptr);
+// The two softmax warps of a lane quarter (qd = 0..3) meet at named
+// barrier 1 + qd.
+__device__ __forceinline__ void pair_sync(int qd) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + qd) : "memory");
+}
+
+// Exchange one float2 per row with the other half of the row's pair: write
+// mine, meet, read the other's.  Consecutive exchanges (counted by xk)
+// alternate between two slots, so a fast half cannot overwrite a value the
+// slow half has not read yet (that needs it past the next meeting).
+__device__ __forceinline__ float2 pair_xch(uint8_t* smem, uint32_t& xk, int hf,
+                                           int r, int qd, float2 mine) {
+  float2* x =
+      reinterpret_cast<float2*>(smem + ExtPlan::kXch) + (xk & 1) * 2 * kRows;
+  ++xk;
+  x[hf * kRows + r] = mine;
+  pair_sync(qd);
+  return x[(1 - hf) * kRows + r];
+}
+
+// A softmax thread's half (dims 64 hf .. 64 hf + 63) of query row r, staged
+// for the q.k product: q (bf16 [128]; read only when live) times an exact
+// power of two into fp16 (max |q| 2^sh in [2^14, 2^15), the row's max taken
+// over both halves: exact), written to row r of the Q16 operand.  Returns
+// the factor that turns an S entry back into a base-2 score.
+__device__ __forceinline__ float tc_stage_q(uint8_t* smem, const __nv_bfloat16* qptr,
+                                            bool live, int r, int hf, int qd,
+                                            float q_scale, uint32_t& xk) {
+  uint8_t* q16 = smem + ExtPlan::kQ16;
+  const uint4* qsrc = reinterpret_cast<const uint4*>(qptr) + 8 * hf;
+  uint4 w[8];
   float amax = 0.0f;
-  if (live) {
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-      const uint4 w = qsrc[i];
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(ww[k] << 16)),
-                                 fabsf(__uint_as_float(ww[k] & 0xFFFF0000u))));
-    }
+  for (int i = 0; i < 8; ++i) {
+    w[i] = live ? qsrc[i] : make_uint4(0, 0, 0, 0);
+    const uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(ww[k] << 16)),
+                               fabsf(__uint_as_float(ww[k] & 0xFFFF0000u))));
   }
+  amax = fmaxf(amax, pair_xch(smem, xk, hf, r, qd, make_float2(amax, 0.0f)).x);
   const int sh = amax > 0.0f ? 15 - exp_frexp(amax) : 0;
   const float f1 = pow2i(sh / 2), f2 = pow2i(sh - sh / 2);
   // the previous item's products are done (its o_done was awaited)
-#pragma unroll 4
-  for (int c = 0; c < 16; ++c) {
-    const uint4 w = live ? qsrc[c] : make_uint4(0, 0, 0, 0);
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t ww[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
     uint32_t h[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -436,69 +469,81 @@ __device__ __forceinline__ float tc_stage_q(const __nv_bfloat16* qptr, bool live
           __uint_as_float(ww[k] & 0xFFFF0000u) * f1 * f2);
       h[k] = *reinterpret_cast<const uint32_t*>(&v);
     }
-    *reinterpret_cast<uint4*>(q16 + op_off(r, c)) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(q16 + op_off(r, 8 * hf + c)) =
+        make_uint4(h[0], h[1], h[2], h[3]);
   }
-  const float qf = q_scale * pow2i(-(sh / 2)) * pow2i(-(sh - sh / 2));
-  return qf;
+  return q_scale * pow2i(-(sh / 2)) * pow2i(-(sh - sh / 2));
 }
 
-// Running softmax state of one row, base 2: max m, sum l, V-scale exponent e.
+// Running softmax state of one row, base 2: max m, V-scale exponent e (the
+// same in both halves of the row) and this half's share of the sum l.
 struct RowSoftmax {
   float m, l;
   int e;
 };
 
 // A softmax thread's pass over its item's nkt key tiles (tiles u .. u+nkt-1
-// of the CTA): reads S from tensor memory, masks keys >= key_lim (all keys
-// when the row is not live), keeps the lazy online softmax, rescales O in
-// tensor memory when the references move, and writes P16 for the O product.
+// of the CTA), for key columns (and output dims) 64 hf .. 64 hf + 63 of row
+// r: reads its half of S from tensor memory, masks keys >= key_lim (all keys
+// when the row is not live), takes the row's maxima with the other half,
+// keeps the lazy online softmax, rescales its half of O in tensor memory
+// when the references move, and writes its half of P16 for the O product.
 __device__ __forceinline__ RowSoftmax tc_row_tiles(uint8_t* smem, uint64_t* bars,
-                                                   uint32_t trow, int r, int lane,
-                                                   bool live, int key_lim,
-                                                   float qf, int nkt, uint32_t u,
+                                                   uint32_t trow, int r, int hf,
+                                                   int qd, int lane, bool live,
+                                                   int key_lim, float qf, int nkt,
+                                                   uint32_t u, uint32_t& xk,
                                                    bool& failed, uint32_t* status) {
   uint8_t* p16 = smem + ExtPlan::kP16;
   float m_run = -INFINITY, l_run = 0.0f;
   int e_run = -126;
   float vlim = 0.0f, fs = 1.0f;
+  const int c0 = kHalf * hf;  // this half's first key column
   for (int j = 0; j < nkt; ++j) {
     const uint32_t t = u + j;
     ewait(&bars[B_S_FULL + (t & 1)], (t >> 1) & 1, failed, status);
     __syncwarp();  // converged for the warp-collective tensor-memory loads
     tc_fence_after();
-    const uint32_t ks_s = smem_u32(smem + ExtPlan::kScl) + (t & 3) * 2 * kKT * 4;
-    // the four loads in flight together, then one wait; the registers are
-    // reused in place as the tile's scores
-    uint32_t sr[kKT];
+    // both loads in flight together, then one wait; the registers are
+    // reused in place as the half tile's scores
+    uint32_t sr[kHalf];
     {
       using Block = uint32_t[32];
       Block* blk = reinterpret_cast<Block*>(sr);
-      const uint32_t sa = trow + kColS + (t & 1) * kKT;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32_async(sa + 32 * q, blk[q]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_wait32(blk[q]);
+      const uint32_t sa = trow + kColS + (t & 1) * kKT + c0;
+      tmem_ld32_async(sa, blk[0]);
+      tmem_ld32_async(sa + 32, blk[1]);
+      tmem_wait32(blk[0]);
+      tmem_wait32(blk[1]);
     }
     float* sv = reinterpret_cast<float*>(sr);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars[B_S_EMPTY + (t & 1)]);
-    // scores and the tile's maxima
+    // scores and the half tile's maxima, then the row's with the other half
     float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     float vx4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const float* ks = reinterpret_cast<const float*>(smem + ExtPlan::kScl +
-                                                     (t & 3) * 2 * kKT * 4);
-    const float* vs = ks + kKT;
-    const int lim = live ? key_lim - j * kKT : 0;  // keys c < lim are visible
+    // the tile's K and V scales (the same for every row): shared-memory
+    // loads by 32-bit address
+    const uint32_t ks_s =
+        smem_u32(smem + ExtPlan::kScl) + (t & 3) * 2 * kKT * 4 + 4 * c0;
+    const uint32_t vs_s = ks_s + kKT * 4;
+    const int lim = live ? key_lim - j * kKT - c0 : 0;  // columns c < lim visible
 #pragma unroll
-    for (int c = 0; c < kKT; ++c) {
+    for (int c = 0; c < kHalf; ++c) {
       const bool ok = c < lim;
-      sv[c] = ok ? sv[c] * qf * ks[c] : -INFINITY;
+      sv[c] = ok ? sv[c] * qf * lds_f1v(ks_s + 4 * c) : -INFINITY;
       mx4[c & 3] = fmaxf(mx4[c & 3], sv[c]);
-      vx4[c & 3] = fmaxf(vx4[c & 3], ok ? vs[c] : 0.0f);
+      vx4[c & 3] = fmaxf(vx4[c & 3], ok ? lds_f1v(vs_s + 4 * c) : 0.0f);
     }
-    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-    const float vx = fmaxf(fmaxf(vx4[0], vx4[1]), fmaxf(vx4[2], vx4[3]));
+    float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+    float vx = fmaxf(fmaxf(vx4[0], vx4[1]), fmaxf(vx4[2], vx4[3]));
+    {
+      const float2 o = pair_xch(smem, xk, hf, r, qd, make_float2(mx, vx));
+      mx = fmaxf(mx, o.x);
+      vx = fmaxf(vx, o.y);
+    }
+    // both halves see the same maxima and take the same decisions
     float a_o = 1.0f;
     bool moved = false;
     if (mx > m_run + kSlack || vx > vlim) {
@@ -516,15 +561,15 @@ __device__ __forceinline__ RowSoftmax tc_row_tiles(uint8_t* smem, uint64_t* bars
     const float mu = m_run == -INFINITY ? 0.0f : m_run;
     // probabilities first (packed fp16 in registers), so that the
     // exponentials overlap the previous O product on the tensor cores
-    uint32_t ph[kKT / 2];
+    uint32_t ph[kHalf / 2];
     float ls4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int c = 0; c < kKT / 2; ++c) {
+    for (int c = 0; c < kHalf / 2; ++c) {
       const float p0 = ex2(sv[2 * c] - mu), p1 = ex2(sv[2 * c + 1] - mu);
       ls4[(2 * c) & 3] += p0;
       ls4[(2 * c + 1) & 3] += p1;
-      const float v0 = sv[2 * c] == -INFINITY ? 0.0f : vs[2 * c];
-      const float v1 = sv[2 * c + 1] == -INFINITY ? 0.0f : vs[2 * c + 1];
+      const float v0 = sv[2 * c] == -INFINITY ? 0.0f : lds_f1v(vs_s + 8 * c);
+      const float v1 = sv[2 * c + 1] == -INFINITY ? 0.0f : lds_f1v(vs_s + 8 * c + 4);
       const __half2 hv = __floats2half2_rn(p0 * (v0 * fs), p1 * (v1 * fs));
       ph[c] = *reinterpret_cast<const uint32_t*>(&hv);
     }
@@ -533,25 +578,25 @@ __device__ __forceinline__ RowSoftmax tc_row_tiles(uint8_t* smem, uint64_t* bars
     if (t >= 1) ewait(&bars[B_O_DONE], (t - 1) & 1, failed, status);
     __syncwarp();
     tc_fence_after();
-    // rescale O in tensor memory where the row's references moved; the
-    // tensor-memory loads and stores are warp-collective, so the whole
-    // warp takes the branch (rows that did not move multiply by 1)
+    // rescale this half of O in tensor memory where the row's references
+    // moved; the tensor-memory loads and stores are warp-collective, so the
+    // whole warp takes the branch (rows that did not move multiply by 1)
     const bool rescale = moved && j > 0;
     if (__any_sync(kFull, rescale)) {
       const float f = rescale ? a_o : 1.0f;
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = 0; c < kHalf / 32; ++c) {
         float o[32];
         __syncwarp();
-        tmem_ld32(trow + kColO + 32 * c, o);
+        tmem_ld32(trow + kColO + c0 + 32 * c, o);
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] *= f;
-        tmem_st32(trow + kColO + 32 * c, o);
+        tmem_st32(trow + kColO + c0 + 32 * c, o);
       }
     }
 #pragma unroll
-    for (int c = 0; c < kKT / 8; ++c)
-      *reinterpret_cast<uint4*>(p16 + op_off(r, c)) =
+    for (int c = 0; c < kHalf / 8; ++c)
+      *reinterpret_cast<uint4*>(p16 + op_off(r, c0 / 8 + c)) =
           make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
     l_run += lsum;
     fence_proxy_async_smem();
@@ -572,7 +617,7 @@ __device__ __forceinline__ uint32_t tc_setup(uint8_t* smem, const CUtensorMap* t
     prefetch_tensormap(tmk);
     prefetch_tensormap(tmv);
     const uint32_t counts[ExtPlan::kBarCount] = {1, 1, 2, 2, 2, 1, 2, 1,
-                                                 1, 1, 4, 4, 4, 1, 4};
+                                                 1, 1, 8, 8, 8, 1, 8};
     for (int i = 0; i < ExtPlan::kBarCount; ++i) mbar_init(&bars[i], counts[i]);
     fence_mbar_init();
   }
