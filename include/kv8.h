@@ -117,11 +117,12 @@ KV8_API size_t kv8_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
  * hands one (sequence, KV head, chunk) to each warp at a time, about 12
  * warps per SM; with few sequences or short contexts whole chunks leave
  * warps idle and make the slowest warp's chain of pages the launch time.
- * This returns the chunk length, a multiple of 16 between 64 and 512, that
- * cuts max_context_len into equal chunks so that batch * num_kv_heads *
- * chunks is at least about three times the resident warps of the current
- * device (148 SMs are assumed when no device can be queried), or 0 (no
- * split) when max_context_len <= 64.  Size the workspace with the returned
+ * Finer chunks are not free: each costs its warp a q load, a partial written
+ * and read back and a merge step.  This returns the chunk length, a multiple
+ * of 16 between 64 and 512, that cuts max_context_len into equal chunks so
+ * that batch * num_kv_heads * chunks is at least the resident warps of the
+ * current device (148 SMs are assumed when no device can be queried), or 0
+ * (no split) when max_context_len <= 64.  Size the workspace with the returned
  * value (kv8_decode_workspace_bytes).  Returns 0 for non-positive arguments.
  */
 KV8_API int32_t kv8_decode_chunk_tokens(int32_t batch, int32_t num_kv_heads,

@@ -258,7 +258,9 @@ int32_t kv8_decode_chunk_tokens(int32_t batch, int32_t num_kv_heads,
     cudaGetLastError();  // no device here: clear the sticky error
     sms = 148;
   }
-  const int64_t want_items = 3 * kWarpsPerSM * sms;
+  // one item per resident warp: past that, a warp's per-item work (loading
+  // q, writing and merging partials) costs more than the finer split saves
+  const int64_t want_items = kWarpsPerSM * sms;
   const int64_t units = static_cast<int64_t>(batch) * num_kv_heads;
   const int64_t splits = (want_items + units - 1) / units;
   int64_t chunk = (max_context_len + splits - 1) / splits;

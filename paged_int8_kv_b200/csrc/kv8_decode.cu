@@ -235,6 +235,14 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
           write_empty<G>(p, it, lane);
           continue;
         }
+        if (live && lane < 2 * G) {
+          // the item's q rows (G x 256 B) into L1 now, SPW pages before the
+          // compute side loads them
+          const __nv_bfloat16* qrow =
+              p.q + (static_cast<int64_t>(it.b) * p.num_q_heads + it.kvh * G) * kD;
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(
+              reinterpret_cast<const char*>(qrow) + 128 * lane));
+        }
         if (lane == 0) wq[q_tail % kQueue] = live ? static_cast<int>(idx) : -1;
         ++q_tail;
         __syncwarp();
@@ -374,10 +382,8 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       ticket = __shfl_sync(kFull, ticket, 0);
       if (ticket == static_cast<unsigned int>(nchunks - 1)) {
         __threadfence();
-        for (int h = 0; h < G; ++h)
-          merge_head_warp(p.ws_ml + (row0 + h) * p.max_chunks * 2,
-                          p.ws_o + (row0 + h) * p.max_chunks * kD, nchunks,
-                          p.out, row0 + h, p.out_f32);
+        merge_group_warp<G>(p.ws_ml, p.ws_o, row0, p.max_chunks, nchunks,
+                            p.out, p.out_f32);
       }
     }
     cmp_live = pop(cmp);

@@ -82,5 +82,72 @@ __device__ __forceinline__ void merge_head_warp(const float* ml, const float* o,
   store_out(out, base + 3, acc.w * inv, out_f32);
 }
 
+// merge_head_warp for the G consecutive query heads row0 .. row0 + G - 1
+// of a KV group (partials at ws_ml + row * max_chunks * 2, ws_o + row *
+// max_chunks * kHeadDim): the same arithmetic, in the same order, per head
+// (so the results equal G calls of merge_head_warp bit for bit), with the
+// heads' loads of each chunk issued together so that G times more of them
+// are in flight.
+template <int G>
+__device__ __forceinline__ void merge_group_warp(const float* ws_ml,
+                                                 const float* ws_o,
+                                                 int64_t row0, int max_chunks,
+                                                 int nchunks, void* out,
+                                                 int out_f32) {
+  const int lane = threadIdx.x & 31;
+  float mx[G], ls[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) mx[h] = -INFINITY;
+  for (int c = lane; c < nchunks; c += 32)
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      mx[h] = fmaxf(mx[h], __ldcg(&ws_ml[((row0 + h) * max_chunks + c) * 2]));
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1)
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], m));
+    ls[h] = 0.0f;
+  }
+  for (int c = lane; c < nchunks; c += 32)
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float* ml = ws_ml + ((row0 + h) * max_chunks + c) * 2;
+      const float mc = __ldcg(&ml[0]);
+      ls[h] += (mc == -INFINITY) ? 0.0f : __ldcg(&ml[1]) * ex2(mc - mx[h]);
+    }
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) ls[h] += __shfl_xor_sync(0xffffffffu, ls[h], m);
+  float4 acc[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) acc[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+  for (int c = 0; c < nchunks; ++c) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const int64_t ci = (row0 + h) * max_chunks + c;
+      const float mc = __ldcg(&ws_ml[2 * ci]);
+      const float w = (mc == -INFINITY) ? 0.0f : ex2(mc - mx[h]);
+      const float4 v =
+          __ldcg(reinterpret_cast<const float4*>(ws_o + ci * kHeadDim) + lane);
+      acc[h].x += w * v.x;
+      acc[h].y += w * v.y;
+      acc[h].z += w * v.z;
+      acc[h].w += w * v.w;
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const float inv = ls[h] > 0.0f ? 1.0f / ls[h] : 0.0f;
+    const int64_t base = (row0 + h) * kHeadDim + 4 * lane;
+    store_out(out, base + 0, acc[h].x * inv, out_f32);
+    store_out(out, base + 1, acc[h].y * inv, out_f32);
+    store_out(out, base + 2, acc[h].z * inv, out_f32);
+    store_out(out, base + 3, acc[h].w * inv, out_f32);
+  }
+}
+
 }  // namespace
 }  // namespace kv8

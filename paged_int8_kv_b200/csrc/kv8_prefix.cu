@@ -212,10 +212,8 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
         const int nch = __shfl_sync(kFull, nchunks, src);
         const int64_t r0 = static_cast<int64_t>(bs) * p.num_q_heads + it.kvh * G;
         __threadfence();
-        for (int h = 0; h < G; ++h)
-          merge_head_warp(p.ws_ml + (r0 + h) * p.max_chunks * 2,
-                          p.ws_o + (r0 + h) * p.max_chunks * kD, nch, p.out,
-                          r0 + h, p.out_f32);
+        merge_group_warp<G>(p.ws_ml, p.ws_o, r0, p.max_chunks, nch, p.out,
+                            p.out_f32);
       }
     }
   }

@@ -124,13 +124,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// 16 bytes of shared memory by 32-bit address; volatile, so a run of them
-// stays interleaved with the arithmetic that consumes it (no hoisting of all
-// loads ahead, which would need a register each).
-__device__ __forceinline__ float4 lds_f4v(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+// Shared-memory loads by 32-bit address; volatile, so a run of them stays
+// interleaved with the arithmetic that consumes it (no hoisting of all loads
+// ahead, which would need a register each).
+__device__ __forceinline__ uint4 lds_u4v(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(addr)
                : "memory");
   return v;
@@ -393,10 +393,11 @@ __device__ __forceinline__ void tc_convert(const Items& items, uint8_t* smem,
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           const int t = ct + 64 * h;
-          const uint8_t* row = src + (t >> 4) * kPageBytes + (t & 15) * 128;
+          const uint32_t row =
+              smem_u32(src) + (t >> 4) * kPageBytes + (t & 15) * 128;
 #pragma unroll
           for (int j8 = 0; j8 < 8; ++j8) {
-            const uint4 w = *reinterpret_cast<const uint4*>(row + ((j8 ^ (t & 7)) << 4));
+            const uint4 w = lds_u4v(row + ((j8 ^ (t & 7)) << 4));
             uint4 lo, hi;
             codes16_to_f16(w, lo, hi);
             *reinterpret_cast<uint4*>(dst + op_off(t, 2 * j8)) = lo;
@@ -529,12 +530,24 @@ __device__ __forceinline__ RowSoftmax tc_row_tiles(uint8_t* smem, uint64_t* bars
         smem_u32(smem + ExtPlan::kScl) + (t & 3) * 2 * kKT * 4 + 4 * c0;
     const uint32_t vs_s = ks_s + kKT * 4;
     const int lim = live ? key_lim - j * kKT - c0 : 0;  // columns c < lim visible
+    // every row of the warp sees all 64 columns (all but the diagonal and
+    // the last tiles): no masking
+    const bool all_visible = __all_sync(kFull, lim >= kHalf);
+    if (all_visible) {
 #pragma unroll
-    for (int c = 0; c < kHalf; ++c) {
-      const bool ok = c < lim;
-      sv[c] = ok ? sv[c] * qf * lds_f1v(ks_s + 4 * c) : -INFINITY;
-      mx4[c & 3] = fmaxf(mx4[c & 3], sv[c]);
-      vx4[c & 3] = fmaxf(vx4[c & 3], ok ? lds_f1v(vs_s + 4 * c) : 0.0f);
+      for (int c = 0; c < kHalf; ++c) {
+        sv[c] = sv[c] * qf * lds_f1v(ks_s + 4 * c);
+        mx4[c & 3] = fmaxf(mx4[c & 3], sv[c]);
+        vx4[c & 3] = fmaxf(vx4[c & 3], lds_f1v(vs_s + 4 * c));
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kHalf; ++c) {
+        const bool ok = c < lim;
+        sv[c] = ok ? sv[c] * qf * lds_f1v(ks_s + 4 * c) : -INFINITY;
+        mx4[c & 3] = fmaxf(mx4[c & 3], sv[c]);
+        vx4[c & 3] = fmaxf(vx4[c & 3], ok ? lds_f1v(vs_s + 4 * c) : 0.0f);
+      }
     }
     float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
     float vx = fmaxf(fmaxf(vx4[0], vx4[1]), fmaxf(vx4[2], vx4[3]));
@@ -563,15 +576,27 @@ __device__ __forceinline__ RowSoftmax tc_row_tiles(uint8_t* smem, uint64_t* bars
     // exponentials overlap the previous O product on the tensor cores
     uint32_t ph[kHalf / 2];
     float ls4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (all_visible) {
 #pragma unroll
-    for (int c = 0; c < kHalf / 2; ++c) {
-      const float p0 = ex2(sv[2 * c] - mu), p1 = ex2(sv[2 * c + 1] - mu);
-      ls4[(2 * c) & 3] += p0;
-      ls4[(2 * c + 1) & 3] += p1;
-      const float v0 = sv[2 * c] == -INFINITY ? 0.0f : lds_f1v(vs_s + 8 * c);
-      const float v1 = sv[2 * c + 1] == -INFINITY ? 0.0f : lds_f1v(vs_s + 8 * c + 4);
-      const __half2 hv = __floats2half2_rn(p0 * (v0 * fs), p1 * (v1 * fs));
-      ph[c] = *reinterpret_cast<const uint32_t*>(&hv);
+      for (int c = 0; c < kHalf / 2; ++c) {
+        const float p0 = ex2(sv[2 * c] - mu), p1 = ex2(sv[2 * c + 1] - mu);
+        ls4[(2 * c) & 3] += p0;
+        ls4[(2 * c + 1) & 3] += p1;
+        const __half2 hv = __floats2half2_rn(p0 * (lds_f1v(vs_s + 8 * c) * fs),
+                                             p1 * (lds_f1v(vs_s + 8 * c + 4) * fs));
+        ph[c] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kHalf / 2; ++c) {
+        const float p0 = ex2(sv[2 * c] - mu), p1 = ex2(sv[2 * c + 1] - mu);
+        ls4[(2 * c) & 3] += p0;
+        ls4[(2 * c + 1) & 3] += p1;
+        const float v0 = sv[2 * c] == -INFINITY ? 0.0f : lds_f1v(vs_s + 8 * c);
+        const float v1 = sv[2 * c + 1] == -INFINITY ? 0.0f : lds_f1v(vs_s + 8 * c + 4);
+        const __half2 hv = __floats2half2_rn(p0 * (v0 * fs), p1 * (v1 * fs));
+        ph[c] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
     }
     const float lsum = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
     // P16 is free and O is up to date once the previous O product is done

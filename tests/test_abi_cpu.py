@@ -114,13 +114,13 @@ def test_host_validation_rejects_before_launch(lib):
 def test_chunk_suggestion(lib):
     # no GPU here: the suggestion assumes 148 SMs x 12 resident warps and
     # cuts the longest context into equal block-aligned chunks of 64..512
-    # tokens so that sequences x KV heads x chunks >= 3 x 1776 warps
+    # tokens so that sequences x KV heads x chunks >= 1776 warps
     f = lib.kv8_decode_chunk_tokens
     f.restype = ctypes.c_int32
     f.argtypes = [ctypes.c_int32] * 3
     assert f(64, 8, 32768) == 512          # 64 chunks: already 9x the warps
-    assert f(32, 8, 4017) == 192           # 21 chunks of <= 192 tokens
-    assert f(256, 8, 544) == 192           # 3 chunks: 192, 192, 160
+    assert f(32, 8, 4017) == 512           # 7 splits wanted: 8 chunks of <= 512
+    assert f(256, 8, 544) == 272           # enough items unsplit; 2 of <= 512
     assert f(2, 2, 256) == 64              # floor of 4 pages per chunk
     assert f(1, 1, 64) == 0 and f(1, 1, 65) == 64
     assert f(0, 8, 100) == 0 and f(4, 0, 100) == 0 and f(4, 8, 0) == 0
