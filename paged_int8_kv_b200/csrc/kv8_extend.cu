@@ -151,6 +151,19 @@ extend_kernel(const ExtParams p, const __grid_constant__ CUtensorMap tmk,
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_Q_FULL]);
+      {
+        // the next item's q row (this half: 128 bytes) into L1 while this
+        // item's tiles run, so its staging does not wait on L2
+        ExtItem nx;
+        if (idx + gridDim.x < n_items && eitem_load(p, idx + gridDim.x, P, nx) &&
+            pos < nx.npos) {
+          const int64_t nrow =
+              static_cast<int64_t>(p.q_start[nx.b] + nx.i0 + pos) * p.num_q_heads +
+              nx.kvh * G + head;
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(
+              reinterpret_cast<const char*>(p.q + nrow * kD) + 128 * hf));
+        }
+      }
 
       // ---- key tiles
       const int key_lim = it.t_ctx - it.n_new + it.i0 + pos + 1;  // keys < this

@@ -152,6 +152,22 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_Q_FULL]);
+      {
+        // the next item's q rows (this half: 128 bytes) into L1 while this
+        // item's tiles run, so its staging does not wait on L2
+        PrefixItem nx;
+        int nfirst;
+        const int64_t nidx = idx + gridDim.x;
+        if (nidx < n && pitem_load(p, ps, M, nidx, nx, nfirst, lane)) {
+          const int nb = member_of(p, nx.g, M * nx.rnd + mr, lane);
+          if (nb >= 0) {
+            const __nv_bfloat16* nq =
+                p.q + (static_cast<int64_t>(nb) * p.num_q_heads + nx.kvh * G + head) * kD;
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(
+                reinterpret_cast<const char*>(nq) + 128 * hf));
+          }
+        }
+      }
 
       // ---- the chunk's keys, all visible to every row
       const RowSoftmax rs =
