@@ -108,6 +108,8 @@ struct PrefixShape {
   int32_t rounds;          // set by launch_prefix: ceil(max_group_size /
                            // members per round)
   int32_t prefix_chunks;   // max over groups of prefix_lens / chunk_tokens
+  int32_t chunks_per_item; // set by launch_prefix: whole prefix chunks a
+                           // prefix-kernel item covers
 };
 
 // Workspace carve-up shared by the decode and reduce launchers.

@@ -41,7 +41,9 @@ __device__ __forceinline__ int exp_frexp(float x) {
 
 // Log-sum-exp merge of one query head's C chunk partials into its output
 // row, by one warp: chunk c holds m_c (base-2 max), l_c (sum of
-// 2^(s - m_c)) and o_c[d] (sum of 2^(s - m_c) v_hat[d]);
+// 2^(s - m_c)) and o_c[d] (sum of 2^(s - m_c) v_hat[d]); an empty slot
+// (m_c = -inf: no token, or a slot whose chunk another slot's partial
+// covers) contributes nothing and its o_c is not read;
 //   M = max_c m_c,  L = sum_c l_c 2^(m_c - M),
 //   out[d] = sum_c o_c[d] 2^(m_c - M) / L.
 // Lanes split the chunks for M and L, then each lane accumulates 4 dims over
@@ -66,7 +68,8 @@ __device__ __forceinline__ void merge_head_warp(const float* ml, const float* o,
 #pragma unroll 8
   for (int c = 0; c < nchunks; ++c) {
     const float mc = __ldcg(&ml[2 * c]);
-    const float w = (mc == -INFINITY) ? 0.0f : ex2(mc - mx);
+    if (mc == -INFINITY) continue;  // an empty slot: its o is not read
+    const float w = ex2(mc - mx);
     const float4 v =
         __ldcg(reinterpret_cast<const float4*>(o + static_cast<int64_t>(c) * kHeadDim) + lane);
     acc.x += w * v.x;
@@ -129,7 +132,8 @@ __device__ __forceinline__ void merge_group_warp(const float* ws_ml,
     for (int h = 0; h < G; ++h) {
       const int64_t ci = (row0 + h) * max_chunks + c;
       const float mc = __ldcg(&ws_ml[2 * ci]);
-      const float w = (mc == -INFINITY) ? 0.0f : ex2(mc - mx[h]);
+      if (mc == -INFINITY) continue;  // an empty slot: its o is not read
+      const float w = ex2(mc - mx[h]);
       const float4 v =
           __ldcg(reinterpret_cast<const float4*>(ws_o + ci * kHeadDim) + lane);
       acc[h].x += w * v.x;

@@ -51,9 +51,10 @@ __device__ __forceinline__ int member_of(const DecodeParams& p, int g, int rank,
   return found;
 }
 
-// Item idx = ((chunk * H_kv + kvh) * groups + g) * rounds + rnd.
+// Item idx = ((cg * H_kv + kvh) * groups + g) * rounds + rnd: chunks
+// [c0, c1) of group g's whole prefix chunks, c0 = cg * chunks_per_item.
 struct PrefixItem {
-  int chunk, kvh, g, rnd;
+  int c0, c1, kvh, g, rnd;
 };
 __device__ __forceinline__ bool pitem_load(const DecodeParams& p,
                                            const PrefixShape& ps, int members,
@@ -64,8 +65,10 @@ __device__ __forceinline__ bool pitem_load(const DecodeParams& p,
   it.g = static_cast<int>(idx % ps.num_groups);
   idx /= ps.num_groups;
   it.kvh = static_cast<int>(idx % p.num_kv_heads);
-  it.chunk = static_cast<int>(idx / p.num_kv_heads);
-  if (it.chunk >= p.prefix_lens[it.g] / p.chunk_tokens) return false;
+  it.c0 = static_cast<int>(idx / p.num_kv_heads) * ps.chunks_per_item;
+  const int whole = p.prefix_lens[it.g] / p.chunk_tokens;
+  if (it.c0 >= whole) return false;
+  it.c1 = min(whole, it.c0 + ps.chunks_per_item);
   // lane 0: the group's first member (its table lists the prefix blocks);
   // lane 1: the round's first member (none: the round is empty)
   const int b = member_of(p, it.g, lane == 1 ? members * it.rnd : 0, lane);
@@ -79,18 +82,20 @@ struct PrefixItems {
   const PrefixShape& ps;
   int members;  // per round: 128 / G
   __device__ __forceinline__ int64_t size() const {
-    return static_cast<int64_t>(ps.prefix_chunks) * p.num_kv_heads *
-           ps.num_groups * ps.rounds;
+    const int64_t groups_of_chunks =
+        (ps.prefix_chunks + ps.chunks_per_item - 1) / ps.chunks_per_item;
+    return groups_of_chunks * p.num_kv_heads * ps.num_groups * ps.rounds;
   }
   __device__ __forceinline__ bool load(int64_t idx, TileItem& t, int lane) const {
     PrefixItem it;
     int first;
     if (!pitem_load(p, ps, members, idx, it, first, lane)) return false;
+    const int keys = (it.c1 - it.c0) * p.chunk_tokens;
     t.tab = static_cast<int64_t>(first) * p.max_blocks_per_seq +
-            it.chunk * (p.chunk_tokens / kBS);
+            it.c0 * (p.chunk_tokens / kBS);
     t.kvh = it.kvh;
-    t.npages = p.chunk_tokens / kBS;
-    t.nkt = (p.chunk_tokens + kKT - 1) / kKT;
+    t.npages = keys / kBS;
+    t.nkt = (keys + kKT - 1) / kKT;
     return true;
   }
 };
@@ -128,7 +133,6 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
     const int r = 32 * qd + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * qd) << 16);
     const int mr = r / G, head = r % G;
-    const int nkt = (p.chunk_tokens + kKT - 1) / kKT;
     uint32_t u = 0, xk = 0;
     const int64_t n = items.size();
     for (int64_t idx = blockIdx.x; idx < n; idx += gridDim.x) {
@@ -136,12 +140,13 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
       int first;
       if (!pitem_load(p, ps, M, idx, it, first, lane)) continue;
       const int b = member_of(p, it.g, M * it.rnd + mr, lane);
-      const int tok0 = it.chunk * p.chunk_tokens;
+      const int keys = (it.c1 - it.c0) * p.chunk_tokens;  // this item's keys
+      const int nkt = (keys + kKT - 1) / kKT;
       int n_b = 0;
       bool live = false;
       if (b >= 0) {
         n_b = p.context_lens[b];
-        live = n_b >= tok0 + p.chunk_tokens;
+        live = n_b >= it.c1 * p.chunk_tokens;
         if (!live && head == 0 && hf == 0)
           atomicOr(&g_prefix_status, KV8_DEV_BAD_PREFIX);
       }
@@ -169,23 +174,27 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
         }
       }
 
-      // ---- the chunk's keys, all visible to every row
+      // ---- the item's keys (its chunks, one after the other), all visible
+      // to every row
       const RowSoftmax rs =
-          tc_row_tiles(smem, bars, trow, r, hf, qd, lane, live, p.chunk_tokens,
-                       qf, nkt, u, xk, failed, &g_prefix_status);
+          tc_row_tiles(smem, bars, trow, r, hf, qd, lane, live, keys, qf, nkt,
+                       u, xk, failed, &g_prefix_status);
       u += nkt;
       const float l = rs.l + pair_xch(smem, xk, hf, r, qd, make_float2(rs.l, 0.0f)).x;
       ewait(&bars[B_O_DONE], (u - 1) & 1, failed, &g_prefix_status);
       __syncwarp();
       tc_fence_after();
 
-      // ---- the row's chunk result (this half's dims): the member's output
-      // row when the chunk is its whole context, else its chunk partial
-      // (m, l, o), o relative to m and unnormalised
+      // ---- the row's result over the item's chunks (this half's dims): the
+      // member's output row when they are its whole context, else one
+      // partial (m, l, o) in the slot of the first chunk, o relative to m and
+      // unnormalised, and empty partials (m = -inf, l = 0; a merge reads
+      // nothing else of them) in the slots of the others
       const int nchunks = (n_b + p.chunk_tokens - 1) / p.chunk_tokens;
-      const bool single = nchunks <= 1;
+      const int nmine = it.c1 - it.c0;
+      const bool single = nchunks <= nmine;
       const float f = single ? pow2i(rs.e) / (l > 0.0f ? l : 1.0f) : pow2i(rs.e);
-      const int64_t ci = row * p.max_chunks + it.chunk;
+      const int64_t ci = row * p.max_chunks + it.c0;
 #pragma unroll 1
       for (int c = 0; c < kHalf / 32; ++c) {
         float o[32];
@@ -208,6 +217,10 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
       if (live && !single && hf == 0) {
         p.ws_ml[2 * ci] = rs.m;
         p.ws_ml[2 * ci + 1] = l;
+        for (int k = 1; k < nmine; ++k) {
+          p.ws_ml[2 * (ci + k)] = -INFINITY;
+          p.ws_ml[2 * (ci + k) + 1] = 0.0f;
+        }
       }
       tc_fence_before();
 
@@ -218,9 +231,9 @@ prefix_kernel(const DecodeParams p, const PrefixShape ps,
       pair_sync(qd);
       const bool lead = live && !single && head == 0 && hf == 0;
       unsigned int ticket = 0;
-      if (lead) ticket = atomicAdd(&p.ws_ctr[row], 1u);
+      if (lead) ticket = atomicAdd(&p.ws_ctr[row], static_cast<unsigned int>(nmine));
       uint32_t mm = __ballot_sync(
-          kFull, lead && ticket == static_cast<unsigned int>(nchunks - 1));
+          kFull, lead && ticket + nmine == static_cast<unsigned int>(nchunks));
       while (mm) {
         const int src = __ffs(mm) - 1;
         mm &= mm - 1;
@@ -260,8 +273,14 @@ int launch_prefix_group(const DecodeParams& p, PrefixShape ps,
   }
   constexpr int M = kRows / G;
   ps.rounds = (ps.max_group_size + M - 1) / M;
-  const int64_t n_items = static_cast<int64_t>(ps.prefix_chunks) *
-                          p.num_kv_heads * ps.num_groups * ps.rounds;
+  // items of about 512 keys (4 tiles): with finer chunks an item covers
+  // several, so the call can split the suffixes finely without one-tile
+  // items here
+  ps.chunks_per_item = p.chunk_tokens >= 512 ? 1 : 512 / p.chunk_tokens;
+  const int64_t n_items =
+      static_cast<int64_t>((ps.prefix_chunks + ps.chunks_per_item - 1) /
+                           ps.chunks_per_item) *
+      p.num_kv_heads * ps.num_groups * ps.rounds;
   if (n_items == 0) return 0;
   int64_t ctas = sms;
   if (ctas > n_items) ctas = n_items;
