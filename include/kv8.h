@@ -182,8 +182,13 @@ KV8_API int32_t kv8_paged_decode_attention(
  * for the whole group instead of once per member, the way serving systems
  * group the requests that share a prefix [garden.houmin.site
  * infra/kv-cache-optimize, §4.3.1 Prefix-aware Scheduling (BatchLLM)].
- * The results are those of kv8_paged_decode_attention on the same inputs
- * (up to rounding order, within the same accuracy).
+ * The shared chunks run on the 5th-generation tensor cores, all of a group's
+ * query rows (members x heads of a KV head) against each shared key tile,
+ * with fp16 operands as in kv8_paged_extend_attention: the K and V codes
+ * exactly, q scaled per row by a power of two, the probabilities rounded to
+ * fp16.  Results are those of kv8_paged_decode_attention on the same inputs
+ * within the decode tolerance (|difference| <= 2e-3 for unit-scale V; the
+ * probability rounding bounds it by 2^-11 max |v_hat|), not bit for bit.
  *
  * Arguments as kv8_paged_decode_attention (form KV8_FORM_AUTO), plus
  *   prefix_group    int32 [batch] device: the group of sequence b, or -1
@@ -198,7 +203,8 @@ KV8_API int32_t kv8_paged_decode_attention(
  *                   word and its row is left incomplete).
  *   num_groups      number of groups (0: a plain decode call)
  *   max_group_size  host bound on the members of any group (any size;
- *                   members are served 8 at a time)
+ *                   members are served 128 / G at a time, G = query heads
+ *                   per KV head)
  *   max_prefix_len  host bound on prefix_lens (<= max_context_len)
  *   chunk_tokens    must be > 0
  * A sequence belongs to at most one group.  The call enqueues a memset of
