@@ -207,9 +207,24 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
   // end marker.
   int* wq = reinterpret_cast<int*>(bars + SPW);  // kQueue entries per warp
   uint32_t q_tail = 0, q_head = 0;
-  // item indices fit 31 bits (the host checks max_chunks * H_kv * B)
-  const uint32_t n_items = static_cast<uint32_t>(p.max_chunks) *
-                           p.num_kv_heads * p.batch;
+  // item indices fit 31 bits (the host checks max_chunks * H_kv * B).  In a
+  // launch beside a shared-prefix launch, the chunks every sequence leaves
+  // to that launch (the fewest whole prefix chunks of any sequence) are not
+  // enumerated at all: items start at chunk c_first.
+  const uint32_t per_chunk = static_cast<uint32_t>(p.num_kv_heads) * p.batch;
+  uint32_t c_first = 0;
+  if (p.prefix_group) {
+    int mn = p.max_chunks;
+    for (int b = lane; b < p.batch; b += 32) {
+      const int g = p.prefix_group[b];
+      mn = min(mn, g >= 0 ? p.prefix_lens[g] / p.chunk_tokens : 0);
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) mn = min(mn, __shfl_xor_sync(kFull, mn, m));
+    c_first = static_cast<uint32_t>(mn);
+  }
+  const uint32_t base = c_first * per_chunk;
+  const uint32_t n_items = (static_cast<uint32_t>(p.max_chunks) - c_first) * per_chunk;
   const uint32_t W = gridDim.x * WPC;
   uint32_t next_idx = blockIdx.x * WPC + warp;
   bool first_take = true;
@@ -229,7 +244,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       first_take = false;
       next_idx = idx;
       const bool live = idx < n_items;  // (no wrap: W + counter < 2^32)
-      if (live) item_set(p, idx, it);
+      if (live) item_set(p, base + idx, it);
       if (!live || item_fill(p, it)) {
         if (live && it.npages == 0) {
           write_empty<G>(p, it, lane);
@@ -243,7 +258,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
           asm volatile("prefetch.global.L1 [%0];" ::"l"(
               reinterpret_cast<const char*>(qrow) + 128 * lane));
         }
-        if (lane == 0) wq[q_tail % kQueue] = live ? static_cast<int>(idx) : -1;
+        if (lane == 0) wq[q_tail % kQueue] = live ? static_cast<int>(base + idx) : -1;
         ++q_tail;
         __syncwarp();
         return live;
