@@ -350,7 +350,25 @@ class DeviceWorkload:
             self.cl if cl is None else cl, self.out, self.w.max_context_len,
             chunk_tokens=self.chunk, workspace=self.ws, form=form)
 
+    def fused(self, form) -> bool:
+        """Whether a step goes through the one-launch entry point (the
+        automatic form without shared prefixes)."""
+        return form == 0 and not self.use_prefix
+
+    def step_fused(self, q=None, k=None, v=None, bt=None, cl=None):
+        import paged_int8_kv_b200 as pk
+        c = self.cache
+        pk.kv8_paged_decode_attention_append(
+            self.q if q is None else q, self.k_new if k is None else k,
+            self.v_new if v is None else v, c.k_cache, c.v_cache, c.k_scales,
+            c.v_scales, self.bt if bt is None else bt,
+            self.cl if cl is None else cl, self.out, self.w.max_context_len,
+            chunk_tokens=self.chunk, workspace=self.ws)
+
     def step(self, form):
+        if self.fused(form):
+            self.step_fused()
+            return
         self.append()
         self.decode(form)
 
@@ -491,9 +509,15 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     ab = algorithmic_bytes(w)
     if ab["total"] <= 4 * 126e6:
         flush = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
-    # per step: the quantize-append kernel and the decode kernel (a split
-    # launch also enqueues a small memset of its merge tickets)
-    launches_per_step = 2
+    # per step: one decode kernel with the append fused in (automatic form),
+    # else the quantize-append kernel and the decode kernel; a split launch
+    # also enqueues a small memset of its merge tickets
+    fused = dw.fused(form)
+    launches_per_step = 1 if fused else 2
+    if fused:  # the step's new K/V read and their codes and scales written
+        nt = w.batch * w.num_kv_heads * 2
+        ab = dict(ab, append=nt * (w.head_dim * 2 + w.head_dim + 4),
+                  total=ab["total"] + nt * (w.head_dim * 2 + w.head_dim + 4))
     memsets_per_step = 1 if dw.ws is not None else 0
 
     def barrier():
@@ -534,21 +558,49 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
         if flush is not None:
             flush_l2(flush)
         ev[i][0].record(stream)
-        dw.append()
-        dec[i][0].record(stream)
-        dw.decode(form)
-        dec[i][1].record(stream)
+        if fused:
+            dw.step_fused()
+        else:
+            dw.append()
+            dec[i][0].record(stream)
+            dw.decode(form)
+            dec[i][1].record(stream)
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    dec_ms = [a.elapsed_time(b) for a, b in dec]
+    # the decode kernel's time: the whole step when the append is fused in
+    dec_ms = step_ms if fused else [a.elapsed_time(b) for a, b in dec]
     ms = sum(step_ms) / len(step_ms)
     if flush is None:
         ms = t_start.elapsed_time(t_end) / args.steps
     dms = sum(dec_ms) / len(dec_ms)
+
+    # ---- for comparison: the same steps as two calls (quantize-append, then
+    # the decode call), device-resident like the above
+    two_ms = two_dec_ms = None
+    if fused:
+        tev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for _ in range(args.warmup):
+            dw.append()
+            dw.decode(form)
+        torch.cuda.synchronize()
+        barrier()
+        for i in range(args.steps):
+            if flush is not None:
+                flush_l2(flush)
+            tev[i][0].record(stream)
+            dw.append()
+            tev[i][1].record(stream)
+            dw.decode(form)
+            tev[i][2].record(stream)
+        torch.cuda.synchronize()
+        two_ms = statistics.mean(a.elapsed_time(c) for a, _, c in tev)
+        two_dec_ms = statistics.mean(b.elapsed_time(c) for _, b, c in tev)
+        barrier()
 
     # ---- end to end through the public API: host buffers in, result out
     kn, vn, sl = dw.host_step
@@ -556,7 +608,9 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
     h_k, h_v, h_s = pin(kn), pin(vn), pin(sl)
     h_q, h_bt, h_cl = pin(w.q()), pin(w.block_tables), pin(w.context_lens)
     h_out = torch.empty(dw.q.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (h_k, h_v, h_s, h_q, h_bt, h_cl))
+    h2d = sum(t.numel() * t.element_size()
+              for t in ((h_k, h_v, h_q, h_bt, h_cl) if fused else
+                        (h_k, h_v, h_s, h_q, h_bt, h_cl)))
     d2h = h_out.numel() * h_out.element_size()
     d_k, d_v, d_s = torch.empty_like(dw.k_new), torch.empty_like(dw.v_new), torch.empty_like(dw.slots)
     d_q, d_bt, d_cl = torch.empty_like(dw.q), torch.empty_like(dw.bt), torch.empty_like(dw.cl)
@@ -568,8 +622,11 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
         d_q.view(torch.int16).copy_(h_q.view(torch.int16), non_blocking=True)
         d_bt.copy_(h_bt, non_blocking=True)
         d_cl.copy_(h_cl, non_blocking=True)
-        dw.append(d_k, d_v, d_s)
-        dw.decode(form, d_q, d_bt, d_cl)
+        if fused:
+            dw.step_fused(d_q, d_k, d_v, d_bt, d_cl)
+        else:
+            dw.append(d_k, d_v, d_s)
+            dw.decode(form, d_q, d_bt, d_cl)
         h_out.copy_(dw.out, non_blocking=True)
 
     # the same lead-in as the device-timed region: about a second of the same
@@ -598,6 +655,8 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
 
     # ---- max over ranks
     ms, dms, e2e_ms = max_over_ranks([ms, dms, e2e_ms], dist, dev)
+    if two_ms is not None:
+        two_ms, two_dec_ms = max_over_ranks([two_ms, two_dec_ms], dist, dev)
 
     status = pk.kv8_read_device_status(clear=True)
     peak, peak_kind = measured_peaks()
@@ -645,13 +704,24 @@ def run_kv8(args, w: W.Workload, rank: int, world: int, dist):
                      "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                                     if peak_kind == "measured" else "fallback 6650 GB/s",
-                     "kernel": "decode kernel (split-K pages + fused chunk merge), "
-                               "timed as the kv8_paged_decode_attention call",
+                     "kernel": ("decode kernel (fused append, split-K pages, fused "
+                                "chunk merge), timed as the whole "
+                                "kv8_paged_decode_attention_append step" if fused else
+                                "decode kernel (split-K pages + fused chunk merge), "
+                                "timed as the kv8_paged_decode_attention call"),
                      "algorithmic_bytes": ab["total"],
                      "traffic": recorded_traffic(w.name)},
         "e2e": {"value": whole_job_rate(w.batch, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "clocks": e2e_clocks},
+        "step_entry_point": ("kv8_paged_decode_attention_append (append fused "
+                             "into the decode kernel)" if fused else
+                             "kv8_quantize_append + the decode call"),
+        "two_call_step": (
+            {"ms_per_step": two_ms, "decode_us": two_dec_ms * 1e3,
+             "value": whole_job_rate(w.batch, world, two_ms), "unit": UNIT,
+             "entry_points": "kv8_quantize_append, kv8_paged_decode_attention"}
+            if two_ms is not None else None),
         "gpu_launches": launches_per_step * args.steps,
         "memsets": memsets_per_step * args.steps,
         "clocks": clocks,

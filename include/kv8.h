@@ -174,6 +174,38 @@ KV8_API int32_t kv8_paged_decode_attention(
     size_t workspace_bytes, void *out, int32_t out_dtype, void *stream);
 
 /*
+ * kv8_paged_decode_attention_append -- one decode step in one launch: the
+ * step's new token of every sequence is quantised into the cache and then
+ * attended to, as kv8_quantize_append followed by kv8_paged_decode_attention
+ * [大模型推理加速：KV Cache与vLLM技术解析, §2.1: the new K/V join the cache
+ * before the step attends to it], with the same codes, scales and output bit
+ * for bit.
+ *
+ * Arguments as kv8_paged_decode_attention (form KV8_FORM_AUTO), with the
+ * caches and scales writable, plus
+ *   k_new, v_new   bf16 [batch][num_kv_heads][head_dim] device, read only:
+ *                  sequence b's new token, which sits at position
+ *                  context_lens[b] - 1 (context_lens counts it) in the block
+ *                  block_tables[b][(context_lens[b] - 1) / block_size]; a
+ *                  sequence with context_lens[b] == 0 has no new token
+ * The warp that takes a sequence's last chunk (its last page) quantises the
+ * token for its KV head before copying that page, so no other launch is
+ * needed and no other warp reads the page.  As for kv8_quantize_append the
+ * caller must not point the position at a block other sequences share.  The
+ * call enqueues a memset of the merge tickets (split launches) and one
+ * kernel.
+ */
+KV8_API int32_t kv8_paged_decode_attention_append(
+    const void *q, const void *k_new, const void *v_new, int8_t *k_cache,
+    int8_t *v_cache, float *k_scales, float *v_scales,
+    const int32_t *block_tables, const int32_t *context_lens, int32_t batch,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, float softmax_scale, int32_t chunk_tokens,
+    void *workspace, size_t workspace_bytes, void *out, int32_t out_dtype,
+    void *stream);
+
+/*
  * kv8_paged_decode_attention_prefix -- kv8_paged_decode_attention for a
  * batch in which groups of sequences share the first tokens of their
  * context, stored once: the same physical blocks open every member's block

@@ -23,7 +23,7 @@ _BINDING_NAMES = {
     "kv8_paged_decode_attention_prefix", "kv8_paged_extend_attention",
     "kv8_decode_partials_bytes", "kv8_paged_decode_attention_partials",
     "kv8_merge_partials",
-    "kv8_paged_decode_attention_noalloc",
+    "kv8_paged_decode_attention_noalloc", "kv8_paged_decode_attention_append",
     "kv8_quantize_append", "kv8_int4_quantize_append",
     "kv8_int4_paged_decode_attention",
     "kv8_read_device_status", "kv8_split_reduce",

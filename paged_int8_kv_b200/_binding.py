@@ -45,6 +45,7 @@ EXPORTED = (
     "kv8_merge_partials",
     "kv8_read_device_status",
     "kv8_paged_decode_attention_noalloc",
+    "kv8_paged_decode_attention_append",
     "kv8_int4_quantize_append",
     "kv8_int4_paged_decode_attention",
 )
@@ -103,6 +104,10 @@ def _load() -> ctypes.CDLL:
     lib.kv8_paged_decode_attention_noalloc.argtypes = [
         P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
         P, i32, P]
+    lib.kv8_paged_decode_attention_append.restype = i32
+    lib.kv8_paged_decode_attention_append.argtypes = [
+        P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32,
+        i32, P, sz, P, i32, P]
     lib.kv8_int4_quantize_append.restype = i32
     lib.kv8_int4_quantize_append.argtypes = [P, P, P, i64, i32, i32, i32, i64, P, P, P, P, P]
     lib.kv8_int4_paged_decode_attention.restype = i32
@@ -247,6 +252,35 @@ def kv8_int4_paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor,
                              block_tables, context_lens, out, max_context_len,
                              chunk_tokens, workspace, softmax_scale),
                _stream(stream)))
+    return out
+
+
+def kv8_paged_decode_attention_append(q: torch.Tensor, k_new: torch.Tensor,
+                                      v_new: torch.Tensor, k_cache: torch.Tensor,
+                                      v_cache: torch.Tensor,
+                                      k_scales: torch.Tensor,
+                                      v_scales: torch.Tensor,
+                                      block_tables: torch.Tensor,
+                                      context_lens: torch.Tensor,
+                                      out: torch.Tensor, max_context_len: int,
+                                      chunk_tokens: int = 512,
+                                      workspace: torch.Tensor | None = None,
+                                      softmax_scale: float = 0.0,
+                                      stream=None) -> torch.Tensor:
+    """One decode step in one launch: k_new / v_new bf16 [B, H_kv, D] (token
+    b at position context_lens[b] - 1) quantised into the cache, then the
+    decode attention; out written in place."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    out_dtype = KV8_OUT_F32 if out.dtype == torch.float32 else KV8_OUT_BF16
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("kv8_paged_decode_attention_append",
+           lib.kv8_paged_decode_attention_append(
+               _p(q), _p(k_new), _p(v_new), _p(k_cache), _p(v_cache),
+               _p(k_scales), _p(v_scales), _p(block_tables), _p(context_lens),
+               B, hq, hkv, d, bs, block_tables.shape[1], nb,
+               int(max_context_len), float(softmax_scale), int(chunk_tokens),
+               _p(workspace), ws_bytes, _p(out), out_dtype, _stream(stream)))
     return out
 
 

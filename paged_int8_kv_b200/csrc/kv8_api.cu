@@ -178,6 +178,12 @@ int32_t prepare_decode(
   p.prefix_group = nullptr;
   p.prefix_lens = nullptr;
   p.partials_only = partials_only ? 1 : 0;
+  p.k_new = nullptr;
+  p.v_new = nullptr;
+  p.k_cache_w = nullptr;
+  p.v_cache_w = nullptr;
+  p.k_scales_w = nullptr;
+  p.v_scales_w = nullptr;
   p.work_ctr = ws_ctr ? ws_ctr + static_cast<size_t>(batch) * num_q_heads : nullptr;
   return KV8_OK;
 }
@@ -313,6 +319,38 @@ int32_t kv8_paged_decode_attention_form(
   int rc = form == KV8_FORM_TCGEN05
                ? kv8::launch_decode_tc(d.p, d.tmk, d.tmv, st)
                : kv8::launch_decode(d.p, d.tmk, d.tmv, form, st);
+  if (rc == -2) return KV8_ERR_UNSUPPORTED;
+  if (rc != 0) return KV8_ERR_CUDA;
+  return KV8_OK;
+}
+
+int32_t kv8_paged_decode_attention_append(
+    const void* q, const void* k_new, const void* v_new, int8_t* k_cache,
+    int8_t* v_cache, float* k_scales, float* v_scales,
+    const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, float softmax_scale, int32_t chunk_tokens,
+    void* workspace, size_t workspace_bytes, void* out, int32_t out_dtype,
+    void* stream) {
+  DecodeSetup d;
+  const int32_t rc0 = prepare_decode(
+      q, k_cache, v_cache, k_scales, v_scales, block_tables, context_lens,
+      batch, num_q_heads, num_kv_heads, head_dim, block_size,
+      max_blocks_per_seq, num_blocks, max_context_len, softmax_scale,
+      chunk_tokens, workspace, workspace_bytes, out, out_dtype, &d);
+  if (rc0 != KV8_OK || d.nothing) return rc0;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))
+    return KV8_ERR_INVALID_ARG;
+  d.p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  d.p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  d.p.k_cache_w = k_cache;
+  d.p.v_cache_w = v_cache;
+  d.p.k_scales_w = k_scales;
+  d.p.v_scales_w = v_scales;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!clear_tickets(d, batch, num_q_heads, st)) return KV8_ERR_CUDA;
+  const int rc = kv8::launch_decode(d.p, d.tmk, d.tmv, KV8_FORM_AUTO, st);
   if (rc == -2) return KV8_ERR_UNSUPPORTED;
   if (rc != 0) return KV8_ERR_CUDA;
   return KV8_OK;

@@ -50,6 +50,12 @@ __device__ __forceinline__ void fence_mbar_init() {
 
 // Order this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (TMA) writes to the same addresses.
+// Order this thread's earlier generic-proxy global writes before its later
+// async-proxy (TMA) reads of the same addresses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -120,6 +120,51 @@ __device__ __forceinline__ bool item_fill(const DecodeParams& p, Item& it) {
   return true;
 }
 
+// Fused append, by one warp: quantise token T_b - 1 of sequence b for KV
+// head kvh (its K and V rows, 128 bf16 each) into the INT8 cache at the
+// slot the block table gives for that position -- the arithmetic of
+// kv8_quantize_append (s = fl32(max|x| / 127), codes rint(fl32(x / s))
+// clamped to +-127, IEEE divisions), so the codes and scales are the same
+// bit for bit -- then make the writes visible to this thread's later TMA
+// copies.  Each lane handles 4 dims.
+__device__ __forceinline__ void append_token(const DecodeParams& p, int b,
+                                             int kvh, int n, int lane) {
+  const int pos = n - 1;
+  const int64_t blk = p.block_tables[static_cast<int64_t>(b) * p.max_blocks_per_seq +
+                                     pos / kBS];
+  const int64_t slot = (blk * p.num_kv_heads + kvh) * kBS + pos % kBS;
+  const int64_t row = static_cast<int64_t>(b) * p.num_kv_heads + kvh;
+#pragma unroll
+  for (int kv = 0; kv < 2; ++kv) {
+    const __nv_bfloat16* src = (kv ? p.v_new : p.k_new) + row * kD;
+    const uint2 raw = reinterpret_cast<const uint2*>(src)[lane];
+    float x[4];
+    x[0] = __uint_as_float(raw.x << 16);
+    x[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(raw.y << 16);
+    x[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    float a = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, m));
+    const float sc = (a == 0.0f) ? 0.0f : __fdiv_rn(a, 127.0f);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int c = 0;
+      if (sc != 0.0f) {
+        const float r = fminf(fmaxf(rintf(__fdiv_rn(x[i], sc)), -127.0f), 127.0f);
+        c = static_cast<int>(r);
+      }
+      packed |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * i);
+    }
+    reinterpret_cast<uint32_t*>((kv ? p.v_cache_w : p.k_cache_w) + slot * kD)[lane] =
+        packed;
+    if (lane == 0) (kv ? p.v_scales_w : p.k_scales_w)[slot] = sc;
+  }
+  fence_proxy_async_global();
+  __syncwarp();
+}
+
 // The result of an item without pages: a zero output row for an empty
 // context (a single-chunk item), else an empty partial (m = -inf, l = 0,
 // o = 0) that a merge skips.  Warp-cooperative.
@@ -250,6 +295,10 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
           write_empty<G>(p, it, lane);
           continue;
         }
+        // fused append: the item holding the sequence's last page, before
+        // any of its pages is copied (no other item reads that page)
+        if (live && p.k_new && it.tok1 == it.n && it.n > 0)
+          append_token(p, it.b, it.kvh, it.n, lane);
         if (live && lane < 2 * G) {
           // the item's q rows (G x 256 B) into L1 now, SPW pages before the
           // compute side loads them

@@ -98,6 +98,16 @@ struct DecodeParams {
   // every (sequence, query head), empty chunks as (-inf, 0, 0), and merge
   // nothing (the partials of several launches are merged afterwards)
   int32_t partials_only;
+  // fused append (nullptr: none): before a sequence's last page is copied,
+  // the warp that takes the sequence's last chunk quantises the step's new
+  // token, k_new / v_new bf16 [B][H_kv][128] at position context_lens[b] - 1,
+  // into the caches through these writable views of them
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  int8_t* k_cache_w;
+  int8_t* v_cache_w;
+  float* k_scales_w;
+  float* v_scales_w;
 };
 
 
