@@ -127,3 +127,26 @@ def test_chunk_suggestion(lib):
     for b, h, t in ((1, 1, 10**6), (7, 3, 12345), (512, 8, 128)):
         c = f(b, h, t)
         assert c % 16 == 0 and 64 <= c <= 512
+
+
+def test_product_path_is_independent_of_the_oracle():
+    # the library and its binding neither import, link nor load anything
+    # under oracle/ (the oracle is test infrastructure only), and the oracle
+    # shares no source with the CUDA path
+    import glob
+    import os
+    import re
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "paged_int8_kv_b200")
+    for path in glob.glob(os.path.join(pkg, "**", "*"), recursive=True):
+        if not path.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+            continue
+        text = open(path, encoding="utf-8").read()
+        assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), path
+        assert "kv8_oracle" not in text and "oracle/" not in text, path
+    for path in glob.glob(os.path.join(root, "oracle", "*")):
+        if path.endswith((".c", ".h", ".py")):
+            text = open(path, encoding="utf-8").read()
+            assert not re.search(r"^\s*(import|from)\s+paged_int8_kv_b200\b", text, re.M), path
+            assert not re.search(r"#\s*include\s*[<\"].*(csrc|kv8_|kv8\.h)", text), path
+            assert not re.search(r"libkv8(?!_oracle)", text), path
