@@ -491,10 +491,10 @@ KV8_API int32_t kv8_int4_quantize_append(const void *k_new, const void *v_new,
  * kv8_int4_paged_decode_attention -- kv8_paged_decode_attention over the
  * INT4 cache: k_hat = c * ks, v_hat = c * vs with c = nibble - 8.  Same
  * arguments, workspace (kv8_decode_workspace_bytes), split and status codes;
- * groups of 1, 2 or 4 query heads per KV head (a larger group returns
- * KV8_ERR_UNSUPPORTED).  Both products run on the warp tensor cores with
- * the nibbles as unsigned 8-bit operands; the +8 bias is removed exactly in
- * integer arithmetic.
+ * groups of 1, 2, 4 or 8 query heads per KV head (8: two sub-groups of 4,
+ * each its own item, reading the same pages).  Both products run on the
+ * warp tensor cores with the nibbles as unsigned 8-bit operands; the +8 bias
+ * is removed exactly in integer arithmetic.
  */
 KV8_API int32_t kv8_int4_paged_decode_attention(
     const void *q, const uint8_t *k_cache, const uint8_t *v_cache,

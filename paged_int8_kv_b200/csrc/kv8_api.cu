@@ -178,6 +178,7 @@ int32_t prepare_decode(
   p.prefix_group = nullptr;
   p.prefix_lens = nullptr;
   p.partials_only = partials_only ? 1 : 0;
+  p.kv_sub_shift = 0;
   p.k_new = nullptr;
   p.v_new = nullptr;
   p.k_cache_w = nullptr;
@@ -584,9 +585,6 @@ int32_t kv8_int4_paged_decode_attention(
     int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
     float softmax_scale, int32_t chunk_tokens, void* workspace,
     size_t workspace_bytes, void* out, int32_t out_dtype, void* stream) {
-  if (num_kv_heads > 0 && num_q_heads > 0 && num_q_heads % num_kv_heads == 0 &&
-      num_q_heads / num_kv_heads > 4)
-    return KV8_ERR_UNSUPPORTED;
   DecodeSetup d;
   const int32_t rc0 = prepare_decode(
       q, reinterpret_cast<const int8_t*>(k_cache),

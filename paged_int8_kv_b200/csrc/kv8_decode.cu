@@ -363,7 +363,8 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmk,
       const uint32_t bar = bars_s + slot_iss * 8;
       mbar_arrive_expect_tx_s(bar, kPageTx);
       if (issue_copies) {
-        const int page = blk * p.num_kv_heads + iss_kvh;
+        const int page = blk * (p.num_kv_heads >> p.kv_sub_shift) +
+                         (iss_kvh >> p.kv_sub_shift);
         const uint32_t tk = tiles_s + slot_iss * (2 * kCB);
         const uint32_t sc = scl_s + slot_iss * (2 * kBS * 4);
         tma_load_3d_s(tk, &tmk, 0, 0, page, bar);
@@ -681,6 +682,19 @@ int launch_decode_int4(const DecodeParams& p, const CUtensorMap& tmk,
     case 1: return launch_group_int4<1>(p, tmk, tmv, stream);
     case 2: return launch_group_int4<2>(p, tmk, tmv, stream);
     case 4: return launch_group_int4<4>(p, tmk, tmv, stream);
+    case 8: {
+      // groups of 8: two sub-groups of 4 query heads per KV head, each its
+      // own item (a warp's integer accumulators hold 4 heads); the two
+      // warps of a KV head read the same pages at about the same time
+      // (sub-groups are numbered fastest), so the second read hits L2
+      if (static_cast<int64_t>(p.max_chunks) * 2 * p.num_kv_heads * p.batch >
+          INT32_MAX)
+        return -2;
+      DecodeParams q = p;
+      q.num_kv_heads = 2 * p.num_kv_heads;
+      q.kv_sub_shift = 1;
+      return launch_group_int4<4>(q, tmk, tmv, stream);
+    }
     default: return -2;
   }
 }

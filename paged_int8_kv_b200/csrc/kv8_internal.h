@@ -102,6 +102,10 @@ struct DecodeParams {
   // the warp that takes the sequence's last chunk quantises the step's new
   // token, k_new / v_new bf16 [B][H_kv][128] at position context_lens[b] - 1,
   // into the caches through these writable views of them
+  // KV heads split into 2^kv_sub_shift sub-groups of query heads, each its
+  // own item (num_kv_heads then counts the sub-groups; the page of item KV
+  // index v is that of KV head v >> kv_sub_shift).  0: no split.
+  int32_t kv_sub_shift;
   const __nv_bfloat16* k_new;
   const __nv_bfloat16* v_new;
   int8_t* k_cache_w;

@@ -7,7 +7,8 @@
     decode tolerance (2e-3 for fp32 output, plus half a bf16 ulp for bf16
     output), for groups of 1, 2 and 4 query heads, split and unsplit, with
     ragged and empty contexts;
-  * a group of 8 is refused with KV8_ERR_UNSUPPORTED.
+  * groups of 8 (two sub-groups of 4 heads per KV head): the prefix-shared
+    70B batch and ragged contexts.
 """
 import numpy as np
 import pytest
@@ -48,6 +49,8 @@ CASES = {
     "ragged_g1": lambda: _ragged_g(1),
     "ragged_g2": lambda: _ragged_g(2),
     "ragged_g4": lambda: _ragged_g(4),
+    "ragged_g8": lambda: _ragged_g(8),
+    "prefix_shared_70b": W.prefix_shared_70b,
 }
 
 _cache = {}
@@ -136,11 +139,3 @@ def test_int4_decode_all_pairs(built, oracle_mod, name, chunk_tokens, out_dtype)
     U.assert_close(gpu, ref, bf16=(out_dtype == "bf16"))
     if out_dtype == "f32":
         assert np.abs(gpu - ref).max() < 1e-4
-
-
-def test_int4_group_of_8_unsupported(built):
-    w = W.make_workload("g8", 77, [40, 20], 16, 2, extra_blocks=1)
-    dev = _device_int4(built, w)
-    with pytest.raises(built.Kv8Error) as e:
-        _decode(built, w, dev, 0, torch.float32)
-    assert e.value.status == built.KV8_ERR_UNSUPPORTED
