@@ -11,22 +11,28 @@
 // one (sequence, KV head, context chunk), handled by one warp):
 //   * A warp owns SPW shared-memory slots and streams its items' 16-token
 //     pages through them: lane 0 resolves each page through the block table
-//     [KV Cache 优化全景解析, §4.2] and issues two TMA tensor copies (the
-//     2 KB K page and the 2 KB V page, 128-byte swizzled so that the
-//     column reads below are bank-conflict free) plus two 64-byte bulk
-//     copies (the K and V scales) that complete on the slot's mbarrier.
-//     There is no producer warp and no cross-warp handshake on the ring:
-//     the warp that consumes a slot refills it.
+//     [KV Cache 优化全景解析, §4.2] and issues two TMA tensor copies (the K
+//     page and the V page, 128-byte swizzled so that the reads below are
+//     bank-conflict free) plus two 64-byte bulk copies (the K and V scales)
+//     that complete on the slot's mbarrier.  There is no producer warp and
+//     no cross-warp handshake on the ring: the warp that consumes a slot
+//     refills it.  Items come from a work counter, numbered chunk-major with
+//     the KV head fastest.
 //   * All G query heads of the KV group are computed together, so each K/V
-//     byte is read from HBM exactly once per step.
-//   * Per page, a warp computes the G x 16 scores with codes converted to
-//     fp32 in registers, folds the token's K scale into the score, keeps a
-//     base-2 online softmax (running max m and sum l per head), folds the
-//     token's V scale into the probability and accumulates o += p * vc.
-//   * At the end of its chunk the warp writes the result from registers: the
-//     normalised output for a sequence that fits one chunk, else the chunk's
-//     (m, l, o) partial; the last chunk of each (sequence, KV group) to
-//     finish (a ticket, never a wait) merges the partials by log-sum-exp.
+//     byte is read from HBM once per step (the INT4 cache's groups of 8 run
+//     as two sub-groups of 4 whose second read of a page comes from L2).
+//   * Per page, the page math (kv8_page_math.cuh) scores the G heads against
+//     the 16 tokens, folds the token's K scale into the score, keeps a base-2
+//     online softmax (running max m and sum l per head), folds the token's V
+//     scale into the probability and accumulates o += p * v_code; the
+//     automatic form does both products on int8 tensor-core mma.
+//   * At the end of its chunk the warp writes the result: the normalised
+//     output for a sequence that fits one chunk, else the chunk's (m, l, o)
+//     partial; the last chunk of each (sequence, KV group) to finish (a
+//     ticket, never a wait) merges the partials by log-sum-exp.
+//   * Fused append (kv8_paged_decode_attention_append): the warp that takes a
+//     sequence's last chunk first quantises the step's new token into the
+//     cache, then copies the page that holds it.
 #include "../../include/kv8.h"
 #include "kv8_common.cuh"
 #include "kv8_internal.h"

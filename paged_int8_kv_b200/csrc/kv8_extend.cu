@@ -20,7 +20,9 @@
 //                                           V16: the V codes, exact in fp16
 // The K scale is applied to S and the V scale folded into P, per key.
 //
-// CTA (8 warps, one per SM, persistent over items):
+// CTA (12 warps, one per SM, persistent over items; the producer, issuer
+// and converter roles and the key-tile softmax live in kv8_tc.cuh, shared
+// with the shared-prefix kernel):
 //   warp 0      TMA producer: each key tile's 8 K pages, 8 V pages and their
 //               scales into a 2-stage ring;
 //   warp 1      MMA issuer (one thread): S of tile j+1 is issued before O of
@@ -28,11 +30,14 @@
 //               the softmax warps work;
 //   warps 2-3   converters: int8 codes -> fp16 operand tiles (128-byte
 //               swizzle) in shared memory, scales copied aside;
-//   warps 4-7   softmax, one thread per row (its tensor-memory lane): loads
-//               the item's q rows, reads S, masks causally, keeps a base-2
-//               online softmax with lazy moves of the reference max m and of
-//               the V-scale exponent E (rescaling O in tensor memory only
-//               then), writes P16, and at the end normalises and stores O.
+//   warps 4-11  softmax, two warps per tensor-memory lane quarter, one row
+//               per thread, each of the pair taking 64 key columns and 64
+//               output dims of its rows: loads the item's q rows, reads S,
+//               masks causally, meets its partner once per tile for the
+//               row's maxima, keeps a base-2 online softmax with lazy moves
+//               of the reference max m and of the V-scale exponent E
+//               (rescaling O in tensor memory only then), writes P16, and at
+//               the end normalises and stores O.
 // Roles hand over through mbarriers only; every wait is bounded in time and
 // records a status bit on timeout.
 #include <cuda_fp16.h>

@@ -10,17 +10,19 @@
 // share a prefix so the shared part is handled once [garden.houmin.site
 // infra/kv-cache-optimize, §4.3.1 Prefix-aware Scheduling (BatchLLM)].
 //
-// For one shared chunk of the prefix and one KV head, the new tokens of the
-// group's members form a block of query rows -- member m, head h -- all
+// For whole chunks of the shared prefix and one KV head, the new tokens of
+// the group's members form a block of query rows -- member m, head h -- all
 // attending to the same keys: a dense contraction of up to 128 rows, which
-// is the extend kernel's tile.  A work item is (prefix chunk, KV head,
-// group, round of 128 / G members); the CTA runs the extend kernel's roles
-// (TMA producer, tcgen05 issuer, int8 -> fp16 converters, four softmax
-// warps, one row per thread) with no causal mask, and each row ends as the
-// member's chunk partial (m, l, o) in the split workspace.  It then takes
-// the member's merge ticket: chunks computed here and the member's own
-// chunks computed by the decode kernel merge into one output row by
-// log-sum-exp, in either order.
+// is the extend kernel's tile.  A work item is (a run of whole prefix
+// chunks of about 512 keys, KV head, group, round of 128 / G members); the
+// CTA runs the extend kernel's roles from kv8_tc.cuh (TMA producer, tcgen05
+// issuer, int8 -> fp16 converters, eight softmax warps, each row split over
+// two of them) with no causal mask, and each row ends as the member's
+// partial (m, l, o) in the split workspace, in the slot of the run's first
+// chunk (the run's other slots hold empty partials).  It then advances the
+// member's merge ticket by the run's chunk count: chunks computed here and
+// the member's own chunks computed by the decode kernel merge into one
+// output row by log-sum-exp, in either order.
 #include "../../include/kv8.h"
 #include "kv8_common.cuh"
 #include "kv8_internal.h"
