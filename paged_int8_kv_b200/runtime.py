@@ -75,6 +75,24 @@ class PagedKV8Cache:
             chunk_tokens=chunk_tokens, workspace=ws,
             softmax_scale=softmax_scale, form=form, stream=stream)
 
+    def step(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+             block_tables: torch.Tensor, context_lens: torch.Tensor,
+             max_context_len: int, chunk_tokens: int = 512,
+             out: torch.Tensor | None = None,
+             out_dtype: torch.dtype = torch.bfloat16,
+             softmax_scale: float = 0.0, stream=None) -> torch.Tensor:
+        """One decode step in one launch: sequence b's new K/V (bf16
+        [B, H_kv, D]) join the cache at position context_lens[b] - 1, then
+        every query head attends over the whole context."""
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        ws = self.workspace(q.shape[0], q.shape[1], max_context_len, chunk_tokens)
+        return B.kv8_paged_decode_attention_append(
+            q, k_new, v_new, self.k_cache, self.v_cache, self.k_scales,
+            self.v_scales, block_tables, context_lens, out, max_context_len,
+            chunk_tokens=chunk_tokens, workspace=ws,
+            softmax_scale=softmax_scale, stream=stream)
+
 
 def fill_from_host(cache: PagedKV8Cache, segments, stream=None) -> int:
     """Copy host (k, v, slot_mapping) segments to the GPU and append them.

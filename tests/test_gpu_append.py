@@ -90,3 +90,22 @@ def test_append_matches_two_calls_and_oracle(pk, oracle_mod, name, chunk):
     ref = oracle_mod.decode_attention(w.q(), kc, vc, ks, vs, w.block_tables,
                                       w.context_lens)
     U.assert_close(out_b.cpu().numpy(), ref, bf16=False)
+
+
+def test_runtime_step_is_the_fused_call(pk, oracle_mod):
+    # PagedKV8Cache.step wraps kv8_paged_decode_attention_append
+    w = W.tiny()
+    kn, vn, _ = w.step_tokens()
+    c = _cache_without_step(w)
+    q = torch.from_numpy(w.q()).view(torch.bfloat16).cuda()
+    out = c.step(q, torch.from_numpy(kn).view(torch.bfloat16).cuda(),
+                 torch.from_numpy(vn).view(torch.bfloat16).cuda(),
+                 torch.from_numpy(w.block_tables).cuda(),
+                 torch.from_numpy(w.context_lens).cuda(), w.max_context_len,
+                 chunk_tokens=64, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    kc, vc, ks, vs = U.oracle_full_cache(oracle_mod, w)
+    assert np.array_equal(c.k_cache.cpu().numpy(), kc)
+    ref = oracle_mod.decode_attention(w.q(), kc, vc, ks, vs, w.block_tables,
+                                      w.context_lens)
+    U.assert_close(out.cpu().numpy(), ref, bf16=False)
