@@ -88,14 +88,40 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# the translation units a decode launch is built from: the kernel and the
+# host code that sizes and launches it (plus the files they include)
+DECODE_ROOTS = ("kv8_decode.cu", "kv8_api.cu")
+
+
+def decode_sources() -> list:
+    """csrc files the decode launch is compiled from: DECODE_ROOTS and,
+    recursively, the csrc files they #include."""
+    csrc = os.path.join(ROOT, "paged_int8_kv_b200", "csrc")
+    seen, todo = set(), list(DECODE_ROOTS)
+    while todo:
+        fn = todo.pop()
+        if fn in seen or not os.path.exists(os.path.join(csrc, fn)):
+            continue
+        seen.add(fn)
+        with open(os.path.join(csrc, fn)) as f:
+            for line in f:
+                line = line.strip()
+                if line.startswith("#include \""):
+                    name = line.split('"')[1]
+                    if "/" not in name:  # the public header is not csrc
+                        todo.append(name)
+    return sorted(seen)
+
+
 def kernel_source_hash() -> str:
+    """Hash of the decode launch's sources: a committed DRAM-traffic record
+    counts only while it matches (other kernels' files do not enter)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_int8_kv_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode())
-                h.update(f.read())
+    for fn in decode_sources():
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
