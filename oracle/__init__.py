@@ -63,6 +63,12 @@ def _load():
     lib.oracle_decode_attention_int4.restype = ctypes.c_int
     lib.oracle_decode_attention_int4.argtypes = [
         P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, f64, P]
+    lib.oracle_kivi_append.restype = ctypes.c_int
+    lib.oracle_kivi_append.argtypes = [
+        P, P, P, P, P, i32, i32, i32, i32, i32, i64, P, P, P, P, P, P, P]
+    lib.oracle_kivi_decode_attention.restype = ctypes.c_int
+    lib.oracle_kivi_decode_attention.argtypes = [
+        P, P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, f64, P]
     lib.oracle_kv_cache_bytes.restype = f64
     lib.oracle_kv_cache_bytes.argtypes = [i64] * 7
     lib.oracle_kv8_scale_bytes.restype = f64
@@ -207,6 +213,76 @@ def decode_attention_int4(q_bf16: np.ndarray, k_cache: np.ndarray,
         _ptr(bt), _ptr(cl), B, hq, hkv, d, bs, bt.shape[1], nb,
         float(softmax_scale), _ptr(out))
     _check(rc, "oracle_decode_attention_int4")
+    return out
+
+
+class KiviCache:
+    """The oracle's KIVI cache in plain layouts (one code per byte):
+
+    k_codes, v_codes uint8 [NB, H_kv, BS, D]; k_scale, k_zero float32
+    [NB, H_kv, D] (per channel); v_scale, v_zero float32 [NB, H_kv, BS]
+    (per token); tail uint16 bf16 bits [B, H_kv, 2, BS, D] (the K and V rows
+    of each sequence's page that is not yet full).  Fields start as
+    `fill_code` / NaN / 0xFFFF so that a slot the oracle never writes shows.
+    """
+
+    def __init__(self, num_blocks, num_kv_heads, batch, block_size=16,
+                 head_dim=128, fill_code=0xFF):
+        nb, h, bs, d = num_blocks, num_kv_heads, block_size, head_dim
+        self.k_codes = np.full((nb, h, bs, d), fill_code, np.uint8)
+        self.v_codes = np.full((nb, h, bs, d), fill_code, np.uint8)
+        self.k_scale = np.full((nb, h, d), np.nan, np.float32)
+        self.k_zero = np.full((nb, h, d), np.nan, np.float32)
+        self.v_scale = np.full((nb, h, bs), np.nan, np.float32)
+        self.v_zero = np.full((nb, h, bs), np.nan, np.float32)
+        self.tail = np.full((batch, h, 2, bs, d), 0xFFFF, np.uint16)
+
+    def fields(self):
+        return (self.k_codes, self.k_scale, self.k_zero, self.v_codes,
+                self.v_scale, self.v_zero)
+
+
+def kivi_append(cache: KiviCache, k_new: np.ndarray, v_new: np.ndarray,
+                cu_new: np.ndarray, context_lens: np.ndarray,
+                block_tables: np.ndarray) -> None:
+    """Append sequence b's rows k_new/v_new[cu_new[b]:cu_new[b+1]] (uint16
+    bf16 bits, [N, H_kv, D]) at its last positions (context_lens counts
+    them), quantising every page they complete; in place."""
+    lib = _load()
+    kn = np.ascontiguousarray(k_new, dtype=np.uint16)
+    vn = np.ascontiguousarray(v_new, dtype=np.uint16)
+    cu = np.ascontiguousarray(cu_new, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    nb, hkv, bs, d = cache.k_codes.shape
+    B = cl.shape[0]
+    assert cu.shape == (B + 1,) and kn.shape == vn.shape
+    assert kn.shape[0] == int(cu[-1]) and kn.shape[1:] == (hkv, d)
+    assert bt.shape[0] == B and cache.tail.shape == (B, hkv, 2, bs, d)
+    rc = lib.oracle_kivi_append(
+        _ptr(kn), _ptr(vn), _ptr(cu), _ptr(cl), _ptr(bt), B, hkv, d, bs,
+        bt.shape[1], nb, *[_ptr(a) for a in cache.fields()], _ptr(cache.tail))
+    _check(rc, "oracle_kivi_append")
+
+
+def kivi_decode_attention(q_bf16: np.ndarray, cache: KiviCache,
+                          block_tables: np.ndarray, context_lens: np.ndarray,
+                          softmax_scale: float = 0.0) -> np.ndarray:
+    """fp64 decode attention over the KIVI cache (full pages dequantised,
+    the partial page's rows from the tail); [B, H_q, D]."""
+    lib = _load()
+    q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    B, hq, d = q.shape
+    nb, hkv, bs, d2 = cache.k_codes.shape
+    assert d2 == d and bt.shape[0] == B and cl.shape == (B,)
+    out = np.zeros((B, hq, d), dtype=np.float64)
+    rc = lib.oracle_kivi_decode_attention(
+        _ptr(q), *[_ptr(a) for a in cache.fields()], _ptr(cache.tail),
+        _ptr(bt), _ptr(cl), B, hq, hkv, d, bs, bt.shape[1], nb,
+        float(softmax_scale), _ptr(out))
+    _check(rc, "oracle_kivi_decode_attention")
     return out
 
 

@@ -19,6 +19,11 @@
  *       block table; several sequences may map to the same physical block.
  *   [same page, §2.3 KV Cache 内存计算公式]
  *       memory = 2 * L * B * T * H_kv * d_h * bytes_per_element.
+ *   [same page, §7.1 and §7.2 KIVI]   the KIVI variant: 2-bit asymmetric
+ *       codes, keys per channel, values per token (its readings are stated
+ *       where it is defined, below).
+ *   [nano-KvLLM, §2.2 量化感知缓存]   the INT4 variant of historical tokens,
+ *       and recent tokens kept at their original precision.
  *
  * Readings where the pages are silent (all listed in the design notes):
  *   - one scale per (token, KV head), s = fl32(max|x| / 127), stored as fp32;
@@ -428,6 +433,289 @@ int oracle_decode_attention_int4(const uint16_t *q, const uint8_t *k_cache,
             if (rc != ORACLE_OK)
                 return rc;
         }
+    return ORACLE_OK;
+}
+
+/*
+ * The KIVI variant of the cache: 2-bit asymmetric codes, keys grouped per
+ * channel and values per token [KV Cache 优化全景解析——从基础原理到工程实践,
+ * §7.1 量化的核心挑战 (keys differ strongly between channels, values are even
+ * within a token) and §7.2 KIVI：2bit 无损非对称量化 (2-bit asymmetric codes,
+ * K per channel, V per token)].  The page fixes the axes, the width and the
+ * asymmetry and nothing else; these readings fill the rest:
+ *   - a group is quantised by its minimum z and its range:
+ *       s = fl32(fl32(max - z) / 3)
+ *       c = clamp(rint(fl32(fl32(x - z) / s)), 0, 3)  (ties to even)
+ *     with s = 0 and every c = 0 when the group is constant, and
+ *     dequantised as x_hat = c * s + z (exact in double);
+ *   - a key group is one channel of one page (16 tokens of one KV head):
+ *     the block the block table maps, so a group never spans pages;
+ *   - a page is quantised when its 16th token arrives; until then its
+ *     tokens' K and V rows stay in bf16 in the sequence's tail ("recent
+ *     tokens keep their original precision", [nano-KvLLM, §2.2 量化感知缓存]),
+ *     and attention reads them there exactly;
+ *   - values are quantised per token at the same moment as the page's keys.
+ *
+ * Plain layouts (one code per byte; the library packs its own):
+ *   k_codes, v_codes  uint8 [num_blocks][H_kv][BS][D]
+ *   k_scale, k_zero   fp32  [num_blocks][H_kv][D]    (per channel)
+ *   v_scale, v_zero   fp32  [num_blocks][H_kv][BS]   (per token)
+ *   tail (bf16 bits)  [batch][H_kv][2][BS][D]        (K rows, then V rows)
+ */
+
+/* Asymmetric 2-bit quantisation of one group of n values x[i * stride]. */
+static int kivi_quantise_group(const float *x, int32_t n, int64_t stride,
+                               uint8_t *codes, int64_t code_stride,
+                               float *scale, float *zero)
+{
+    float lo = x[0], hi = x[0];
+    for (int32_t i = 1; i < n; ++i) {
+        float v = x[i * stride];
+        if (v < lo)
+            lo = v;
+        if (v > hi)
+            hi = v;
+    }
+    float s = (hi - lo) / 3.0f;
+    if (!isfinite(s))
+        return ORACLE_NONFINITE;
+    for (int32_t i = 0; i < n; ++i) {
+        int code = 0;
+        if (s != 0.0f) {
+            float y = (x[i * stride] - lo) / s;
+            float r = nearbyintf(y);
+            if (r > 3.0f)
+                r = 3.0f;
+            if (r < 0.0f)
+                r = 0.0f;
+            code = (int)r;
+        }
+        codes[i * code_stride] = (uint8_t)code;
+    }
+    *scale = s;
+    *zero = lo;
+    return ORACLE_OK;
+}
+
+/*
+ * Quantise the full page that sequence b's tail holds (all heads) into
+ * physical block blk: keys per channel over the 16 tokens, values per token
+ * over the D channels.
+ */
+static int kivi_quantise_page(const uint16_t *tail_b, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t block_size,
+                              int64_t blk, uint8_t *k_codes, float *k_scale,
+                              float *k_zero, uint8_t *v_codes, float *v_scale,
+                              float *v_zero)
+{
+    const int64_t row_elems = (int64_t)block_size * head_dim;
+    float *x = (float *)malloc(sizeof(float) * (size_t)row_elems);
+    if (!x)
+        return ORACLE_NOMEM;
+    int rc = ORACLE_OK;
+    for (int32_t h = 0; h < num_kv_heads && rc == ORACLE_OK; ++h) {
+        const int64_t page = blk * num_kv_heads + h;
+        for (int kv = 0; kv < 2 && rc == ORACLE_OK; ++kv) {
+            const uint16_t *rows = tail_b + ((int64_t)h * 2 + kv) * row_elems;
+            for (int64_t i = 0; i < row_elems; ++i) {
+                x[i] = bf16_bits_to_float(rows[i]);
+                if (!isfinite(x[i]))
+                    rc = ORACLE_NONFINITE;
+            }
+            if (rc != ORACLE_OK)
+                break;
+            if (kv == 0) {
+                /* keys: one group per channel j, tokens t = 0..BS-1 */
+                for (int32_t j = 0; j < head_dim && rc == ORACLE_OK; ++j)
+                    rc = kivi_quantise_group(
+                        x + j, block_size, head_dim,
+                        k_codes + page * row_elems + j, head_dim,
+                        &k_scale[page * head_dim + j],
+                        &k_zero[page * head_dim + j]);
+            } else {
+                /* values: one group per token t, channels j = 0..D-1 */
+                for (int32_t t = 0; t < block_size && rc == ORACLE_OK; ++t)
+                    rc = kivi_quantise_group(
+                        x + (int64_t)t * head_dim, head_dim, 1,
+                        v_codes + page * row_elems + (int64_t)t * head_dim, 1,
+                        &v_scale[page * block_size + t],
+                        &v_zero[page * block_size + t]);
+            }
+        }
+    }
+    free(x);
+    return rc;
+}
+
+/*
+ * Append new tokens to the KIVI cache, one token at a time in position
+ * order.  Sequence b gets the n_b = cu_new[b+1] - cu_new[b] rows
+ * k_new/v_new[cu_new[b] .. cu_new[b+1]) (bf16 bits, [*][H_kv][D]) at
+ * positions context_lens[b] - n_b .. context_lens[b] - 1 (context_lens
+ * counts them).  Each row goes to tail row (position % BS); when a position
+ * completes a page (position % BS == BS - 1) the tail's page is quantised
+ * into block block_tables[b][position / BS].  Returns ORACLE_BAD_ARG for
+ * n_b < 0, n_b > context_lens[b], a context longer than the table or a
+ * block out of range; ORACLE_NONFINITE for a non-finite input or scale.
+ */
+int oracle_kivi_append(const uint16_t *k_new, const uint16_t *v_new,
+                       const int32_t *cu_new, const int32_t *context_lens,
+                       const int32_t *block_tables, int32_t batch,
+                       int32_t num_kv_heads, int32_t head_dim,
+                       int32_t block_size, int32_t max_blocks_per_seq,
+                       int64_t num_blocks, uint8_t *k_codes, float *k_scale,
+                       float *k_zero, uint8_t *v_codes, float *v_scale,
+                       float *v_zero, uint16_t *tail)
+{
+    if (batch < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        cu_new[0] != 0)
+        return ORACLE_BAD_ARG;
+    const int64_t row_elems = (int64_t)block_size * head_dim;
+    for (int32_t b = 0; b < batch; ++b) {
+        const int32_t n_new = cu_new[b + 1] - cu_new[b];
+        const int32_t len = context_lens[b];
+        if (n_new < 0 || n_new > len ||
+            len > (int64_t)max_blocks_per_seq * block_size)
+            return ORACLE_BAD_ARG;
+        uint16_t *tail_b = tail + (int64_t)b * num_kv_heads * 2 * row_elems;
+        for (int32_t i = 0; i < n_new; ++i) {
+            const int32_t pos = len - n_new + i;
+            const int64_t tok = (int64_t)cu_new[b] + i;
+            for (int32_t h = 0; h < num_kv_heads; ++h)
+                for (int kv = 0; kv < 2; ++kv) {
+                    const uint16_t *src = (kv ? v_new : k_new) +
+                                          (tok * num_kv_heads + h) * head_dim;
+                    uint16_t *dst = tail_b + ((int64_t)h * 2 + kv) * row_elems +
+                                    (int64_t)(pos % block_size) * head_dim;
+                    memcpy(dst, src, sizeof(uint16_t) * (size_t)head_dim);
+                }
+            if (pos % block_size == block_size - 1) {
+                const int64_t blk = block_tables[(int64_t)b * max_blocks_per_seq +
+                                                 pos / block_size];
+                if (blk < 0 || blk >= num_blocks)
+                    return ORACLE_BAD_ARG;
+                int rc = kivi_quantise_page(tail_b, num_kv_heads, head_dim,
+                                            block_size, blk, k_codes, k_scale,
+                                            k_zero, v_codes, v_scale, v_zero);
+                if (rc != ORACLE_OK)
+                    return rc;
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Decode attention over the KIVI cache, fp64: as oracle_decode_attention,
+ * with, for sequence b's n cached tokens and F = BS * floor(n / BS):
+ *   t <  F: k_hat_t[j] = kc * k_scale[j] + k_zero[j]   (page of token t)
+ *           v_hat_t[j] = vc * v_scale[t] + v_zero[t]
+ *   t >= F: k_hat_t, v_hat_t = the bf16 rows in tail row t % BS.
+ * out (fp64) [B][H_q][D].
+ */
+int oracle_kivi_decode_attention(const uint16_t *q, const uint8_t *k_codes,
+                                 const float *k_scale, const float *k_zero,
+                                 const uint8_t *v_codes, const float *v_scale,
+                                 const float *v_zero, const uint16_t *tail,
+                                 const int32_t *block_tables,
+                                 const int32_t *context_lens, int32_t batch,
+                                 int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t block_size,
+                                 int32_t max_blocks_per_seq, int64_t num_blocks,
+                                 double softmax_scale, double *out)
+{
+    if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_q_heads % num_kv_heads != 0)
+        return ORACLE_BAD_ARG;
+    if (softmax_scale <= 0.0)
+        softmax_scale = 1.0 / sqrt((double)head_dim);
+    const int32_t group = num_q_heads / num_kv_heads;
+    const int64_t row_elems = (int64_t)block_size * head_dim;
+    for (int32_t b = 0; b < batch; ++b) {
+        const int32_t n = context_lens[b];
+        if (n < 0 || n > (int64_t)max_blocks_per_seq * block_size)
+            return ORACLE_BAD_ARG;
+        const int32_t full = n / block_size * block_size;
+        double *khat = (double *)malloc(sizeof(double) * (size_t)(n + 1) * head_dim);
+        double *vhat = (double *)malloc(sizeof(double) * (size_t)(n + 1) * head_dim);
+        double *score = (double *)malloc(sizeof(double) * (size_t)(n + 1));
+        if (!khat || !vhat || !score) {
+            free(khat);
+            free(vhat);
+            free(score);
+            return ORACLE_NOMEM;
+        }
+        for (int32_t kvh = 0; kvh < num_kv_heads; ++kvh) {
+            /* the dequantised rows of this KV head */
+            for (int32_t t = 0; t < n; ++t) {
+                const int32_t r = t % block_size;
+                for (int32_t j = 0; j < head_dim; ++j) {
+                    double kx, vx;
+                    if (t < full) {
+                        const int64_t blk =
+                            block_tables[(int64_t)b * max_blocks_per_seq + t / block_size];
+                        if (blk < 0 || blk >= num_blocks) {
+                            free(khat);
+                            free(vhat);
+                            free(score);
+                            return ORACLE_BAD_ARG;
+                        }
+                        const int64_t page = blk * num_kv_heads + kvh;
+                        const int64_t at = page * row_elems + (int64_t)r * head_dim + j;
+                        kx = (double)k_codes[at] * (double)k_scale[page * head_dim + j] +
+                             (double)k_zero[page * head_dim + j];
+                        vx = (double)v_codes[at] * (double)v_scale[page * block_size + r] +
+                             (double)v_zero[page * block_size + r];
+                    } else {
+                        const uint16_t *tb =
+                            tail + ((int64_t)b * num_kv_heads + kvh) * 2 * row_elems;
+                        kx = (double)bf16_bits_to_float(tb[(int64_t)r * head_dim + j]);
+                        vx = (double)bf16_bits_to_float(
+                            tb[row_elems + (int64_t)r * head_dim + j]);
+                    }
+                    khat[(int64_t)t * head_dim + j] = kx;
+                    vhat[(int64_t)t * head_dim + j] = vx;
+                }
+            }
+            for (int32_t g = 0; g < group; ++g) {
+                const int32_t h = kvh * group + g;
+                const uint16_t *qrow = q + ((int64_t)b * num_q_heads + h) * head_dim;
+                double *orow = out + ((int64_t)b * num_q_heads + h) * head_dim;
+                for (int32_t j = 0; j < head_dim; ++j)
+                    orow[j] = 0.0;
+                if (n == 0)
+                    continue;
+                double smax = -INFINITY;
+                for (int32_t t = 0; t < n; ++t) {
+                    double dot = 0.0;
+                    for (int32_t j = 0; j < head_dim; ++j)
+                        dot += (double)bf16_bits_to_float(qrow[j]) *
+                               khat[(int64_t)t * head_dim + j];
+                    score[t] = softmax_scale * dot;
+                    if (score[t] > smax)
+                        smax = score[t];
+                }
+                double denom = 0.0;
+                for (int32_t t = 0; t < n; ++t) {
+                    score[t] = exp(score[t] - smax);
+                    denom += score[t];
+                }
+                for (int32_t t = 0; t < n; ++t)
+                    for (int32_t j = 0; j < head_dim; ++j)
+                        orow[j] += score[t] / denom * vhat[(int64_t)t * head_dim + j];
+                for (int32_t j = 0; j < head_dim; ++j)
+                    if (!isfinite(orow[j])) {
+                        free(khat);
+                        free(vhat);
+                        free(score);
+                        return ORACLE_NONFINITE;
+                    }
+            }
+        }
+        free(khat);
+        free(vhat);
+        free(score);
+    }
     return ORACLE_OK;
 }
 
