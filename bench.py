@@ -925,6 +925,108 @@ def run_int4(args, w: W.Workload, rank: int, world: int, dist):
     return 0
 
 
+KIVI_PAGE_BYTES = 2176  # one (block, KV head) page record of the KIVI cache
+
+
+def kivi_algorithmic_bytes(w: W.Workload) -> dict:
+    """Bytes one KIVI decode launch must move: the page record of every full
+    page attended, the bf16 K and V rows of each partial page (read from the
+    tail), q, out and the block-table entries used."""
+    full = sum(int(t) // w.block_size for t in w.context_lens)
+    rows = sum(int(t) % w.block_size for t in w.context_lens)
+    kv = (full * KIVI_PAGE_BYTES + rows * 2 * w.head_dim * 2) * w.num_kv_heads
+    ab = algorithmic_bytes(w)
+    return {"kv": kv, "total": kv + ab["total"] - ab["kv"]}
+
+
+def run_kivi(args, w: W.Workload, rank: int, world: int, dist):
+    """The KIVI cache variant on the timed workload: one step = the step's
+    kv8_kivi_append (one token per sequence; a token that completes its page
+    quantises it) plus one kv8_kivi_paged_decode_attention call, inputs
+    resident (the 32K workload's page records, 2.3 GB, are larger than L2)."""
+    import torch
+    import paged_int8_kv_b200 as pk
+    dev = torch.device("cuda", _env_int("LOCAL_RANK", 0))
+    torch.cuda.set_device(dev)
+    cache = torch.zeros((w.num_blocks, w.num_kv_heads, KIVI_PAGE_BYTES),
+                        dtype=torch.uint8, device=dev)
+    tail = torch.zeros((w.batch, w.num_kv_heads, 2, w.block_size, w.head_dim),
+                       dtype=torch.bfloat16, device=dev)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+
+    def to_dev(a, bf16=False):
+        t = torch.from_numpy(np.ascontiguousarray(a)).pin_memory().to(dev, non_blocking=True)
+        return t.view(torch.bfloat16) if bf16 else t
+
+    def call_args(c):
+        k, v, cu, cl = c
+        return (to_dev(k, True), to_dev(v, True), to_dev(cu), to_dev(cl), bt,
+                cache, tail, max(int(np.diff(cu).max(initial=0)), 1))
+    for c in w.kivi_fill_calls():
+        pk.kv8_kivi_append(*call_args(c))
+        torch.cuda.synchronize()  # the pinned host rows are reused
+    step_args = call_args(w.kivi_step_call())
+    q = to_dev(w.q(), True)
+    cl = torch.from_numpy(w.context_lens).to(dev)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    chunk = pick_chunk(w, args.chunk)
+    nbytes = pk.kv8_decode_workspace_bytes(w.batch, w.num_q_heads, w.head_dim,
+                                           w.max_context_len, chunk)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def decode():
+        pk.kv8_kivi_paged_decode_attention(q, cache, tail, bt, cl, out,
+                                           w.max_context_len,
+                                           chunk_tokens=chunk, workspace=ws)
+
+    def step():
+        pk.kv8_kivi_append(*step_args)
+        decode()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks([t0.elapsed_time(t1) / args.steps], dist, dev)[0]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b in ev:
+        a.record(stream)
+        decode()
+        b.record(stream)
+    torch.cuda.synchronize()
+    dec_ms = statistics.median([a.elapsed_time(b) for a, b in ev])
+    status = pk.kv8_read_device_status(clear=True)
+    total = kivi_algorithmic_bytes(w)["total"]
+    peak, src = measured_peaks()
+    gbs = total / (dec_ms * 1e-3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "paged KIVI-KV decode attention tokens/s and achieved HBM GB/s",
+            "value": whole_job_rate(w.batch, world, ms), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u2 codes, f32 CUDA-core arithmetic",
+            "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": w.name + "_kivi", "batch": w.batch,
+                       "context_tokens": int(w.context_lens.sum()),
+                       "chunk_tokens": chunk, "l2": "inputs larger than L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak,
+                         "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "peak_source": src,
+                         "algorithmic_bytes": total,
+                         "decode_us": dec_ms * 1e3},
+            "device_status": status}), flush=True)
+    return 0
+
+
 def run_dry_cpu(args, rank: int, world: int, dist):
     """The launch and rank logic alone, on CPU ranks over gloo: every rank
     times a trivial host step, the max over ranks is taken, rank 0 prints a
@@ -987,6 +1089,8 @@ def main():
                     help="time extend (chunked-prefill) attention instead")
     ap.add_argument("--int4", action="store_true",
                     help="time the INT4 cache variant on --workload instead")
+    ap.add_argument("--kivi", action="store_true",
+                    help="time the KIVI cache variant on --workload instead")
     ap.add_argument("--dry-run-cpu", action="store_true",
                     help="rank/launch logic only, on CPU over gloo (no GPU work, "
                          "no measurement)")
@@ -1020,6 +1124,8 @@ def main():
             return run_extend(args, rank, world, dist)
         if args.int4:
             return run_int4(args, W.NAMED[args.workload](), rank, world, dist)
+        if args.kivi:
+            return run_kivi(args, W.NAMED[args.workload](), rank, world, dist)
         return run_kv8(args, W.NAMED[args.workload](), rank, world, dist)
     finally:
         if dist is not None:

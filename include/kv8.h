@@ -505,6 +505,93 @@ KV8_API int32_t kv8_int4_paged_decode_attention(
     float softmax_scale, int32_t chunk_tokens, void *workspace,
     size_t workspace_bytes, void *out, int32_t out_dtype, void *stream);
 
+/*
+ * The KIVI variant of the cache [KV Cache 优化全景解析——从基础原理到工程实践,
+ * §7.1 量化的核心挑战 and §7.2 KIVI：2bit 无损非对称量化]: 2-bit asymmetric
+ * codes, keys grouped per channel (channels differ widely) and values per
+ * token (a token's channels are even).  The page gives the axes, the width
+ * and the asymmetry; the library's readings:
+ *   - a group x is stored as its minimum z, a scale
+ *     s = fl32(fl32(max - z) / 3) (IEEE subtraction and division) and codes
+ *     c = clamp(rint(fl32(fl32(x - z) / s)), 0, 3), ties to even; s = 0 and
+ *     c = 0 for a constant group; x_hat = c * s + z;
+ *   - a key group is one channel of one 16-token page (one block of one KV
+ *     head); a value group is one token of one KV head (128 channels);
+ *   - a page is quantised when its 16th token is appended.  Until then the
+ *     page's K and V rows stay in bf16 in the sequence's tail and attention
+ *     reads them as they are (recent tokens keep their precision
+ *     [nano-KvLLM, §2.2 量化感知缓存]).
+ *
+ * Layout
+ *   kivi_cache  uint8 [num_blocks][num_kv_heads][KV8_KIVI_PAGE_BYTES], one
+ *               page record per (block, KV head):
+ *       [   0,  512)  K codes: 128 little-endian 32-bit words, word j =
+ *                     channel j, token t in bits 2t and 2t+1
+ *       [ 512, 1024)  V codes, the same layout
+ *       [1024, 1536)  K scales, fp32 [128] (per channel)
+ *       [1536, 2048)  K zero points, fp32 [128]
+ *       [2048, 2112)  V scales, fp32 [16] (per token)
+ *       [2112, 2176)  V zero points, fp32 [16]
+ *   kivi_tail   bf16 [batch][num_kv_heads][2][block_size][head_dim]: the K
+ *               rows (index 0) and V rows (index 1) of each sequence's last
+ *               page while it holds fewer than 16 tokens; row r = position
+ *               % 16.  Row b of the tail belongs to the sequence in batch
+ *               row b, in every append and decode call.
+ * 136 bytes a token per KV head, against 264 for the INT8 cache.
+ */
+#define KV8_KIVI_PAGE_BYTES 2176
+
+/*
+ * kv8_kivi_append -- append new tokens to the KIVI cache.
+ *
+ *   k_new, v_new   bf16 [cu_new[batch]][num_kv_heads][head_dim]: sequence
+ *                  b's new rows are rows cu_new[b] .. cu_new[b+1]-1, for
+ *                  positions context_lens[b] - n_b .. context_lens[b] - 1
+ *                  (n_b = cu_new[b+1] - cu_new[b]; context_lens counts them)
+ *   cu_new         int32 [batch + 1], cu_new[0] = 0, non-decreasing
+ *   context_lens   int32 [batch], n_b <= context_lens[b] <= max_blocks_per_seq
+ *                  * block_size
+ *   block_tables   int32 [batch][max_blocks_per_seq]; the blocks of the
+ *                  pages this call completes are written
+ *   max_new_tokens host-side bound on every n_b (sizes the grid); 0 = no-op
+ * Every page that one of the new positions completes (positions 16j .. 16j+15
+ * all present after the call) is quantised from the tail's earlier rows and
+ * the new rows into its record; then the new rows of the last, partial page
+ * are copied into the tail.  The tail rows of positions before this call
+ * must hold what earlier calls appended.  The caller must not point a new
+ * position at a block other sequences share.  Two kernels on `stream`.
+ */
+KV8_API int32_t kv8_kivi_append(const void *k_new, const void *v_new,
+                                const int32_t *cu_new,
+                                const int32_t *context_lens,
+                                const int32_t *block_tables, int32_t batch,
+                                int32_t num_kv_heads, int32_t head_dim,
+                                int32_t block_size, int32_t max_blocks_per_seq,
+                                int64_t num_blocks, int32_t max_new_tokens,
+                                uint8_t *kivi_cache, void *kivi_tail,
+                                void *stream);
+
+/*
+ * kv8_kivi_paged_decode_attention -- kv8_paged_decode_attention over the
+ * KIVI cache: for sequence b with n = context_lens[b] and F = 16 * floor(n /
+ * 16), tokens t < F are dequantised from their page record,
+ *     k_hat_t[j] = c * k_scale[j] + k_zero[j],  v_hat_t[j] = c * v_scale[t]
+ *                  + v_zero[t],
+ * and tokens F <= t < n are the bf16 rows of the tail.  Same arguments,
+ * workspace (kv8_decode_workspace_bytes), split, output types and status
+ * codes as kv8_paged_decode_attention; groups of 1, 2, 4 or 8 query heads per
+ * KV head (8: two sub-groups of 4).  fp32 arithmetic on the CUDA cores; one
+ * kernel (and a memset of the merge tickets when split).
+ */
+KV8_API int32_t kv8_kivi_paged_decode_attention(
+    const void *q, const uint8_t *kivi_cache, const void *kivi_tail,
+    const int32_t *block_tables, const int32_t *context_lens, int32_t batch,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, float softmax_scale, int32_t chunk_tokens,
+    void *workspace, size_t workspace_bytes, void *out, int32_t out_dtype,
+    void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -48,7 +48,11 @@ EXPORTED = (
     "kv8_paged_decode_attention_append",
     "kv8_int4_quantize_append",
     "kv8_int4_paged_decode_attention",
+    "kv8_kivi_append",
+    "kv8_kivi_paged_decode_attention",
 )
+
+KV8_KIVI_PAGE_BYTES = 2176
 
 
 class Kv8Error(RuntimeError):
@@ -114,6 +118,13 @@ def _load() -> ctypes.CDLL:
     lib.kv8_int4_paged_decode_attention.argtypes = [
         P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
         P, sz, P, i32, P]
+    lib.kv8_kivi_append.restype = i32
+    lib.kv8_kivi_append.argtypes = [
+        P, P, P, P, P, i32, i32, i32, i32, i32, i64, i32, P, P, P]
+    lib.kv8_kivi_paged_decode_attention.restype = i32
+    lib.kv8_kivi_paged_decode_attention.argtypes = [
+        P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32, P, sz,
+        P, i32, P]
     lib.kv8_read_device_status.restype = i32
     lib.kv8_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
     return lib
@@ -252,6 +263,49 @@ def kv8_int4_paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor,
                              block_tables, context_lens, out, max_context_len,
                              chunk_tokens, workspace, softmax_scale),
                _stream(stream)))
+    return out
+
+
+def kv8_kivi_append(k_new: torch.Tensor, v_new: torch.Tensor,
+                    cu_new: torch.Tensor, context_lens: torch.Tensor,
+                    block_tables: torch.Tensor, kivi_cache: torch.Tensor,
+                    kivi_tail: torch.Tensor, max_new_tokens: int,
+                    stream=None) -> None:
+    """Append rows to the KIVI cache: k_new/v_new bf16 [N, H_kv, D], cu_new
+    int32 [B + 1], context_lens int32 [B] (after the append); kivi_cache
+    uint8 [NB, H_kv, KV8_KIVI_PAGE_BYTES]; kivi_tail bf16
+    [B, H_kv, 2, 16, D]."""
+    nb, hkv, _ = kivi_cache.shape
+    B = context_lens.shape[0]
+    _check("kv8_kivi_append", lib.kv8_kivi_append(
+        _p(k_new), _p(v_new), _p(cu_new), _p(context_lens), _p(block_tables),
+        B, hkv, kivi_tail.shape[-1], kivi_tail.shape[-2], block_tables.shape[1],
+        nb, int(max_new_tokens), _p(kivi_cache), _p(kivi_tail),
+        _stream(stream)))
+
+
+def kv8_kivi_paged_decode_attention(q: torch.Tensor, kivi_cache: torch.Tensor,
+                                    kivi_tail: torch.Tensor,
+                                    block_tables: torch.Tensor,
+                                    context_lens: torch.Tensor,
+                                    out: torch.Tensor, max_context_len: int,
+                                    chunk_tokens: int = 512,
+                                    workspace: torch.Tensor | None = None,
+                                    softmax_scale: float = 0.0,
+                                    stream=None) -> torch.Tensor:
+    """Decode attention over the KIVI cache; q bf16 [B, H_q, D], out bf16
+    or fp32 [B, H_q, D] (written in place)."""
+    B, hq, d = q.shape
+    nb, hkv, _ = kivi_cache.shape
+    out_dtype = KV8_OUT_F32 if out.dtype == torch.float32 else KV8_OUT_BF16
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("kv8_kivi_paged_decode_attention",
+           lib.kv8_kivi_paged_decode_attention(
+               _p(q), _p(kivi_cache), _p(kivi_tail), _p(block_tables),
+               _p(context_lens), B, hq, hkv, d, kivi_tail.shape[-2],
+               block_tables.shape[1], nb, int(max_context_len),
+               float(softmax_scale), int(chunk_tokens), _p(workspace),
+               ws_bytes, _p(out), out_dtype, _stream(stream)))
     return out
 
 

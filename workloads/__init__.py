@@ -205,6 +205,41 @@ class Workload:
             slots[b] = self.slots(b, [t - 1])[0]
         return k, v, slots
 
+    # ----------------------------------------------------------- KIVI fill
+    def kivi_fill_calls(self):
+        """Append calls that put every token but each sequence's last into a
+        KIVI cache, one call per sequence so that host memory stays at one
+        sequence's rows: yields (k, v, cu_new [B+1], context_lens [B]) with
+        only sequence b's rows.  A shared prefix is appended by its group's
+        first member only (its blocks are shared; the prefix is a whole
+        number of pages), the other members start after it."""
+        B = self.batch
+        seen = set()
+        for b in range(B):
+            n = max(int(self.context_lens[b]) - 1, 0)
+            lo = 0
+            if self.prefix_group is not None and self.prefix_group[b] >= 0:
+                grp = int(self.prefix_group[b])
+                lo = self.prefix_len if grp in seen else 0
+                seen.add(grp)
+            lo = min(lo, n)
+            if n == lo:
+                continue
+            k, v = self.sequence_kv(b)
+            cu = np.zeros(B + 1, np.int32)
+            cu[b + 1:] = n - lo
+            cl = np.zeros(B, np.int32)
+            cl[b] = n
+            yield k[lo:n], v[lo:n], cu, cl
+
+    def kivi_step_call(self):
+        """The decode step's append call: each sequence's last token
+        (sequences with an empty context append nothing)."""
+        k, v, slots = self.step_tokens()
+        has = slots >= 0
+        cu = np.concatenate([[0], np.cumsum(has)]).astype(np.int32)
+        return k[has], v[has], cu, self.context_lens.astype(np.int32)
+
     # ----------------------------------------------------------- accounting
     def token_heads(self) -> int:
         return int(self.context_lens.astype(np.int64).sum()) * self.num_kv_heads
