@@ -93,11 +93,15 @@ def measured_peaks():
 DECODE_ROOTS = ("kv8_decode.cu", "kv8_api.cu")
 
 
-def decode_sources() -> list:
-    """csrc files the decode launch is compiled from: DECODE_ROOTS and,
-    recursively, the csrc files they #include."""
+# the KIVI decode's translation unit (its kernels and their entry points)
+KIVI_ROOTS = ("kv8_kivi.cu",)
+
+
+def decode_sources(roots=DECODE_ROOTS) -> list:
+    """csrc files a launch is compiled from: `roots` and, recursively, the
+    csrc files they #include."""
     csrc = os.path.join(ROOT, "paged_int8_kv_b200", "csrc")
-    seen, todo = set(), list(DECODE_ROOTS)
+    seen, todo = set(), list(roots)
     while todo:
         fn = todo.pop()
         if fn in seen or not os.path.exists(os.path.join(csrc, fn)):
@@ -113,21 +117,21 @@ def decode_sources() -> list:
     return sorted(seen)
 
 
-def kernel_source_hash() -> str:
-    """Hash of the decode launch's sources: a committed DRAM-traffic record
-    counts only while it matches (other kernels' files do not enter)."""
+def kernel_source_hash(roots=DECODE_ROOTS) -> str:
+    """Hash of a launch's sources: a committed DRAM-traffic record counts
+    only while it matches (other kernels' files do not enter)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_int8_kv_b200", "csrc")
-    for fn in decode_sources():
+    for fn in decode_sources(roots):
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per decode launch from a committed ncu capture, if it was
-    taken on the current kernel source (else None)."""
+def recorded_traffic(workload: str, roots=DECODE_ROOTS):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken
+    on the current source of the launch built from `roots` (else None)."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
@@ -135,7 +139,7 @@ def recorded_traffic(workload: str):
     except Exception:
         return None
     rec = d.get(workload)
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(roots):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -1020,7 +1024,8 @@ def run_kivi(args, w: W.Workload, rank: int, world: int, dist):
                        "chunk_tokens": chunk, "l2": "inputs larger than L2"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak,
                          "unit": "GB/s", "frac": gbs / peak,
-                         "traffic": None, "peak_source": src,
+                         "traffic": recorded_traffic(w.name + "_kivi", KIVI_ROOTS),
+                         "peak_source": src,
                          "algorithmic_bytes": total,
                          "decode_us": dec_ms * 1e3},
             "device_status": status}), flush=True)
