@@ -111,6 +111,45 @@ def test_host_validation_rejects_before_launch(lib):
              0, 0, 16, 0, 2, 0) == 2                # head_dim unsupported
 
 
+def test_kivi_host_validation(lib):
+    # Every call below fails (or finishes) in its host checks: no pointer is
+    # dereferenced and no kernel is launched.
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    a = lib.kv8_kivi_append
+    a.restype = i32
+    a.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i64, i32, P, P, P]
+
+    def app(k=16, batch=2, hkv=2, d=128, bs=16, mbs=4, nb=8, max_new=4, cache=16):
+        return a(k, 16, 16, 16, 16, batch, hkv, d, bs, mbs, nb, max_new, cache, 16, 0)
+    assert app(d=64) == 2            # head_dim unsupported
+    assert app(bs=32) == 2           # block size unsupported
+    assert app(max_new=-1) == 1      # negative bound
+    assert app(batch=-1) == 1
+    assert app(k=0) == 1             # null rows
+    assert app(cache=8) == 1         # misaligned cache
+    assert app(max_new=0) == 0       # nothing to append
+    assert app(batch=0) == 0
+    f = lib.kv8_kivi_paged_decode_attention
+    f.restype = i32
+    f.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32,
+                  ctypes.c_float, i32, P, ctypes.c_size_t, P, i32, P]
+
+    def dec(q=16, batch=1, hq=8, hkv=2, d=128, bs=16, mbs=4, maxlen=64,
+            chunk=0, ws=0, odt=1):
+        return f(q, 16, 16, 16, 16, batch, hq, hkv, d, bs, mbs, 8, maxlen, 0.0,
+                 chunk, ws, 0, 16, odt, 0)
+    assert dec(d=64) == 2            # head_dim unsupported
+    assert dec(hq=6, hkv=2) == 2     # group of 3 not built
+    assert dec(hq=8, hkv=3) == 1     # not a multiple
+    assert dec(maxlen=65) == 1       # > mbs * block_size
+    assert dec(chunk=24) == 1        # not a block multiple
+    assert dec(odt=7) == 1           # bad output dtype
+    assert dec(q=0) == 1             # null pointer
+    assert dec(q=8) == 1             # misaligned q
+    assert dec(chunk=16) == 3        # a split needs a workspace
+    assert dec(batch=0) == 0         # nothing to do
+
+
 def test_chunk_suggestion(lib):
     # no GPU here: the suggestion assumes 148 SMs x 12 resident warps and
     # cuts the longest context into equal block-aligned chunks of 64..512

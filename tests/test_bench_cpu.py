@@ -49,3 +49,29 @@ def test_prefix_shared_workload_unique_share():
     suffix = sum(int(t) - 4096 for t in w.context_lens) * w.num_kv_heads * BYTES
     assert u == prefix + suffix
     assert math.isclose(kv / u, (8 * prefix + suffix) / (prefix + suffix))
+
+
+def test_kivi_algorithmic_bytes_closed_form():
+    # full pages move their 2176-byte record per KV head; the partial page's
+    # rows are read from the bf16 tail (K and V, 256 B each)
+    assert bench.KIVI_PAGE_BYTES == 2 * 512 + 2 * 512 + 2 * 64 == 2176
+    w = W.make_workload("kacct", 4244, [17, 300, 1, 32], 8, 2)
+    kb = bench.kivi_algorithmic_bytes(w)
+    full = 1 + 18 + 0 + 2
+    rows = 1 + 12 + 1 + 0
+    assert kb["kv"] == (full * 2176 + rows * 2 * 256) * 2
+    ab = bench.algorithmic_bytes(w)
+    assert kb["total"] == kb["kv"] + ab["q"] + ab["out"] + ab["tables"]
+    # the bench workload: 136 B per (token, KV head), every page full
+    big = W.llama8b_b64_32k()
+    assert bench.kivi_algorithmic_bytes(big)["kv"] == 64 * 32768 * 8 * 136
+
+
+def test_traffic_records_follow_their_own_sources():
+    # each launch's record is keyed to the sources it is built from
+    dec = bench.decode_sources()
+    kivi = bench.decode_sources(bench.KIVI_ROOTS)
+    assert "kv8_decode.cu" in dec and "kv8_api.cu" in dec
+    assert "kv8_kivi.cu" not in dec and "kv8_decode.cu" not in kivi
+    assert "kv8_kivi.cu" in kivi and "kv8_merge.cuh" in kivi
+    assert bench.kernel_source_hash() != bench.kernel_source_hash(bench.KIVI_ROOTS)

@@ -96,3 +96,44 @@ def test_bf16_rounding():
     assert back[1] == 1.0
     assert back[2] == np.float32(1.015625)
     assert back[0] == 1.0 and back[3] == -2.5
+
+
+def _replay_kivi_calls(w):
+    """Per sequence, the rows the KIVI fill and step calls append, keyed by
+    position (every call's context_lens counts its rows: the new rows of
+    sequence b sit at positions cl[b] - n_b .. cl[b] - 1)."""
+    got = {b: {} for b in range(w.batch)}
+    for k, v, cu, cl in list(w.kivi_fill_calls()) + [w.kivi_step_call()]:
+        assert cu[0] == 0 and np.all(np.diff(cu) >= 0) and cu[-1] == k.shape[0]
+        assert k.shape == v.shape and k.shape[1:] == (w.num_kv_heads, w.head_dim)
+        for b in range(w.batch):
+            n = int(cu[b + 1] - cu[b])
+            assert 0 <= n <= int(cl[b])
+            for i in range(n):
+                pos = int(cl[b]) - n + i
+                assert pos not in got[b], (b, pos)  # each position once
+                got[b][pos] = (k[cu[b] + i], v[cu[b] + i])
+    return got
+
+
+def test_kivi_calls_append_every_position_once():
+    w = W.make_workload("kv", 7, [33, 0, 16, 47, 1], 4, 2)
+    got = _replay_kivi_calls(w)
+    for b, t in enumerate(w.context_lens):
+        assert sorted(got[b]) == list(range(int(t)))
+        k, v = w.sequence_kv(b)
+        for pos, (kr, vr) in got[b].items():
+            assert np.array_equal(kr, k[pos]) and np.array_equal(vr, v[pos])
+
+
+def test_kivi_calls_write_a_shared_prefix_once():
+    w = W.make_workload("kp", 8, [48 + 5, 48 + 20, 48 + 1, 9], 8, 1,
+                        prefix_group=[0, 0, 0, -1], prefix_len=48)
+    got = _replay_kivi_calls(w)
+    assert sorted(got[0]) == list(range(53))          # the first member: all
+    assert sorted(got[1]) == list(range(48, 68))      # later members: suffix
+    assert sorted(got[2]) == [48]
+    assert sorted(got[3]) == list(range(9))
+    # the step call appends exactly the last token of each sequence
+    k, v, cu, cl = w.kivi_step_call()
+    assert list(np.diff(cu)) == [1, 1, 1, 1] and list(cl) == [53, 68, 49, 9]
