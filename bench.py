@@ -270,6 +270,87 @@ def oracle_sample_seconds(w: W.Workload, seqs, threads: int = 1) -> tuple[float,
     return total, desc
 
 
+def oracle_kivi_sample_seconds(w: W.Workload, seqs, threads: int = 1) -> tuple[float, str]:
+    """Time the oracle's KIVI decode step (append of the new token + attention
+    for every query head) on sequences ``seqs``, each in a private cache
+    holding its other tokens (cache build excluded); with ``threads`` > 1 the
+    sequences run on a pool of that many threads (the C oracle releases the
+    interpreter lock).  Returns (seconds, description)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    prep = []
+    for b in seqs:
+        k, v = w.sequence_kv(b)
+        n = k.shape[0]
+        nblk = max(1, math.ceil(n / w.block_size))
+        table = np.arange(nblk, dtype=np.int32)[None, :]
+        c = oracle.KiviCache(nblk, w.num_kv_heads, 1)
+        if n > 1:
+            oracle.kivi_append(c, k[:-1], v[:-1], np.array([0, n - 1]),
+                               np.array([n - 1]), table)
+        prep.append((b, k, v, n, table, c))
+
+    def one(item):
+        b, k, v, n, table, c = item
+        if n:
+            oracle.kivi_append(c, k[-1:], v[-1:], np.array([0, 1]), np.array([n]), table)
+        oracle.kivi_decode_attention(w.q()[b:b + 1], c, table, np.array([n]))
+
+    used = max(1, min(threads, len(prep)))
+    t0 = time.perf_counter()
+    if used > 1:
+        with ThreadPoolExecutor(max_workers=used) as ex:
+            list(ex.map(one, prep))
+    else:
+        for item in prep:
+            one(item)
+    total = time.perf_counter() - t0
+    desc = (f"{len(prep)} sequences of {w.name} (KIVI), one decode step each "
+            f"(append of the new token + all {w.num_q_heads} heads' attention), "
+            f"{used} thread{'s' if used > 1 else ''}")
+    return total, desc
+
+
+def oracle_int4_sample_seconds(w: W.Workload, seqs, threads: int = 1) -> tuple[float, str]:
+    """oracle_kivi_sample_seconds for the INT4 cache: per sequence, the
+    quantise-append of its new token and the attention of all its heads."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    prep = []
+    for b in seqs:
+        k, v = w.sequence_kv(b)
+        n = k.shape[0]
+        nblk = max(1, math.ceil(n / w.block_size))
+        shape = (nblk, w.num_kv_heads, w.block_size, w.head_dim // 2)
+        kc, vc = np.zeros(shape, np.uint8), np.zeros(shape, np.uint8)
+        ks, vs = np.zeros(shape[:3], np.float32), np.zeros(shape[:3], np.float32)
+        slots = np.arange(n, dtype=np.int64)
+        oracle.quantize_append_int4(k[:-1], slots[:-1], kc, ks)
+        oracle.quantize_append_int4(v[:-1], slots[:-1], vc, vs)
+        prep.append((b, k, v, n, slots, kc, vc, ks, vs))
+
+    def one(item):
+        b, k, v, n, slots, kc, vc, ks, vs = item
+        oracle.quantize_append_int4(k[-1:], slots[-1:], kc, ks)
+        oracle.quantize_append_int4(v[-1:], slots[-1:], vc, vs)
+        table = np.arange(kc.shape[0], dtype=np.int32)[None, :]
+        oracle.decode_attention_int4(w.q()[b:b + 1], kc, vc, ks, vs, table, np.array([n]))
+
+    used = max(1, min(threads, len(prep)))
+    t0 = time.perf_counter()
+    if used > 1:
+        with ThreadPoolExecutor(max_workers=used) as ex:
+            list(ex.map(one, prep))
+    else:
+        for item in prep:
+            one(item)
+    total = time.perf_counter() - t0
+    desc = (f"{len(prep)} sequences of {w.name} (INT4), one decode step each "
+            f"(quantise-append of the new token + all {w.num_q_heads} heads' "
+            f"attention), {used} thread{'s' if used > 1 else ''}")
+    return total, desc
+
+
 def host_cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -909,6 +990,14 @@ def run_int4(args, w: W.Workload, rank: int, world: int, dist):
     total = kv + ab["total"] - ab["kv"]
     peak, src = measured_peaks()
     gbs = total / (dec_ms * 1e-3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        seqs = list(range(min(args.cpu_seqs, w.batch)))
+        cores = host_cores()
+        sec, desc = oracle_int4_sample_seconds(w, seqs, cores)
+        cpu = {"value": len(seqs) / sec, "unit": "tokens/s",
+               "cores": max(1, min(cores, len(seqs))), "kind": "oracle",
+               "sample": desc}
     if rank == 0:
         print(json.dumps({
             "metric": "paged INT4-KV decode attention tokens/s and achieved HBM GB/s",
@@ -925,6 +1014,7 @@ def run_int4(args, w: W.Workload, rank: int, world: int, dist):
                          "traffic": None, "peak_source": src,
                          "algorithmic_bytes": total,
                          "decode_us": dec_ms * 1e3},
+            "cpu_baseline": cpu,
             "device_status": status}), flush=True)
     return 0
 
@@ -1011,6 +1101,14 @@ def run_kivi(args, w: W.Workload, rank: int, world: int, dist):
     total = kivi_algorithmic_bytes(w)["total"]
     peak, src = measured_peaks()
     gbs = total / (dec_ms * 1e-3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        seqs = list(range(min(args.cpu_seqs, w.batch)))
+        cores = host_cores()
+        sec, desc = oracle_kivi_sample_seconds(w, seqs, cores)
+        cpu = {"value": len(seqs) / sec, "unit": "tokens/s",
+               "cores": max(1, min(cores, len(seqs))), "kind": "oracle",
+               "sample": desc}
     if rank == 0:
         print(json.dumps({
             "metric": "paged KIVI-KV decode attention tokens/s and achieved HBM GB/s",
@@ -1028,6 +1126,7 @@ def run_kivi(args, w: W.Workload, rank: int, world: int, dist):
                          "peak_source": src,
                          "algorithmic_bytes": total,
                          "decode_us": dec_ms * 1e3},
+            "cpu_baseline": cpu,
             "device_status": status}), flush=True)
     return 0
 

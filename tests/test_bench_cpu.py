@@ -75,3 +75,17 @@ def test_traffic_records_follow_their_own_sources():
     assert "kv8_kivi.cu" not in dec and "kv8_decode.cu" not in kivi
     assert "kv8_kivi.cu" in kivi and "kv8_merge.cuh" in kivi
     assert bench.kernel_source_hash() != bench.kernel_source_hash(bench.KIVI_ROOTS)
+
+
+def test_kivi_cpu_baseline_runs_the_oracle():
+    w = W.make_workload("kcpu", 4245, [40, 17, 1, 0], 8, 2)
+    sec, desc = bench.oracle_kivi_sample_seconds(w, [0, 1, 2, 3], threads=2)
+    assert sec > 0 and "4 sequences" in desc and "2 threads" in desc
+    sec1, desc1 = bench.oracle_kivi_sample_seconds(w, [1], threads=8)
+    assert sec1 > 0 and "1 thread" in desc1
+
+
+def test_int4_cpu_baseline_runs_the_oracle():
+    w = W.make_workload("i4cpu", 4246, [40, 17, 1], 8, 2)
+    sec, desc = bench.oracle_int4_sample_seconds(w, [0, 1, 2], threads=3)
+    assert sec > 0 and "3 sequences" in desc and "3 threads" in desc
