@@ -506,6 +506,30 @@ KV8_API int32_t kv8_int4_paged_decode_attention(
     size_t workspace_bytes, void *out, int32_t out_dtype, void *stream);
 
 /*
+ * kv8_check_indices -- debug check of the device-resident indices the other
+ * calls trust (they are the caller's contract and are not checked there).
+ * Counts, into counts[0..2] (device uint32, zeroed by the call first):
+ *   counts[0]  sequences with context_lens[b] < 0 or > max_context_len
+ *   counts[1]  block-table entries a decode would read (the first
+ *              ceil(len / block_size) of row b, len clamped to [0,
+ *              min(max_context_len, max_blocks_per_seq * 16)]) outside
+ *              [0, num_blocks)
+ *   counts[2]  slot_mapping entries >= num_blocks * 16 (negative entries are
+ *              padding)
+ * batch may be 0 (no table check) and n_tokens may be 0 (no slot check;
+ * slot_mapping may be NULL).  The kernels read only those arrays, within the
+ * bounds given here, so the check is safe on inputs a decode must not see.
+ * Asynchronous on `stream`: read counts after synchronising.  Status codes
+ * as elsewhere.
+ */
+KV8_API int32_t kv8_check_indices(const int32_t *block_tables,
+                                  const int32_t *context_lens, int32_t batch,
+                                  int32_t max_blocks_per_seq,
+                                  int64_t num_blocks, int32_t max_context_len,
+                                  const int64_t *slot_mapping, int64_t n_tokens,
+                                  uint32_t *counts, void *stream);
+
+/*
  * The KIVI variant of the cache [KV Cache 优化全景解析——从基础原理到工程实践,
  * §7.1 量化的核心挑战 and §7.2 KIVI：2bit 无损非对称量化]: 2-bit asymmetric
  * codes, keys grouped per channel (channels differ widely) and values per

@@ -27,6 +27,7 @@ _BINDING_NAMES = {
     "kv8_quantize_append", "kv8_int4_quantize_append",
     "kv8_int4_paged_decode_attention", "kv8_kivi_append",
     "kv8_kivi_paged_decode_attention", "KV8_KIVI_PAGE_BYTES",
+    "kv8_check_indices",
     "kv8_read_device_status", "kv8_split_reduce",
     "kv8_status_string",
 }

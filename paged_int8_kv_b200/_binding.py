@@ -50,6 +50,7 @@ EXPORTED = (
     "kv8_int4_paged_decode_attention",
     "kv8_kivi_append",
     "kv8_kivi_paged_decode_attention",
+    "kv8_check_indices",
 )
 
 KV8_KIVI_PAGE_BYTES = 2176
@@ -125,6 +126,8 @@ def _load() -> ctypes.CDLL:
     lib.kv8_kivi_paged_decode_attention.argtypes = [
         P, P, P, P, P, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32, P, sz,
         P, i32, P]
+    lib.kv8_check_indices.restype = i32
+    lib.kv8_check_indices.argtypes = [P, P, i32, i32, i64, i32, P, i64, P, P]
     lib.kv8_read_device_status.restype = i32
     lib.kv8_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
     return lib
@@ -264,6 +267,31 @@ def kv8_int4_paged_decode_attention(q: torch.Tensor, k_cache: torch.Tensor,
                              chunk_tokens, workspace, softmax_scale),
                _stream(stream)))
     return out
+
+
+def kv8_check_indices(block_tables: torch.Tensor | None,
+                      context_lens: torch.Tensor | None, max_context_len: int,
+                      num_blocks: int, slot_mapping: torch.Tensor | None = None,
+                      stream=None) -> tuple[int, int, int]:
+    """Debug check of the trusted indices: returns (context lengths out of
+    [0, max_context_len], block-table entries a decode would read outside
+    [0, num_blocks), slots at or past num_blocks * 16), after synchronising
+    the stream."""
+    dev = next(t.device for t in (block_tables, context_lens, slot_mapping)
+               if t is not None)
+    counts = torch.zeros(3, dtype=torch.int32, device=dev)
+    batch = 0 if context_lens is None else context_lens.shape[0]
+    mbs = 1 if block_tables is None else block_tables.shape[1]
+    n = 0 if slot_mapping is None else slot_mapping.shape[0]
+    st = _stream(stream)
+    _check("kv8_check_indices", lib.kv8_check_indices(
+        _p(block_tables), _p(context_lens), batch, mbs, int(num_blocks),
+        int(max_context_len), _p(slot_mapping), n, _p(counts), st))
+    if stream is None:
+        torch.cuda.current_stream(dev).synchronize()
+    else:
+        stream.synchronize()
+    return tuple(int(x) for x in counts.cpu().tolist())
 
 
 def kv8_kivi_append(k_new: torch.Tensor, v_new: torch.Tensor,

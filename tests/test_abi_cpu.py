@@ -150,6 +150,21 @@ def test_kivi_host_validation(lib):
     assert dec(batch=0) == 0         # nothing to do
 
 
+def test_check_indices_host_validation(lib):
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    f = lib.kv8_check_indices
+    f.restype = i32
+    f.argtypes = [P, P, i32, i32, i64, i32, P, i64, P, P]
+    assert f(16, 16, 2, 4, 8, 64, 0, 0, 0, 0) == 1      # no counts buffer
+    assert f(16, 16, 2, 4, 8, 64, 0, 0, 18, 0) == 1     # misaligned counts
+    assert f(16, 16, -1, 4, 8, 64, 0, 0, 16, 0) == 1    # negative batch
+    assert f(0, 16, 2, 4, 8, 64, 0, 0, 16, 0) == 1      # tables missing
+    assert f(16, 16, 2, 0, 8, 64, 0, 0, 16, 0) == 1     # empty rows
+    assert f(16, 16, 0, 4, 8, 64, 0, 3, 16, 0) == 1     # slots missing
+    assert f(16, 16, 0, 4, 8, 64, 12, 3, 16, 0) == 1    # misaligned slots
+    assert f(16, 16, 2, 4, 0, 64, 0, 0, 16, 0) == 1     # no blocks
+
+
 def test_chunk_suggestion(lib):
     # no GPU here: the suggestion assumes 148 SMs x 12 resident warps and
     # cuts the longest context into equal block-aligned chunks of 64..512
