@@ -4,12 +4,36 @@
 and V, layout as in include/kv8.h) and a reusable split-K workspace with
 PyTorch, and forwards to the C entry points.  It is plumbing only: every
 number it produces comes from the CUDA kernels.
+
+Debug mode: with the environment variable ``KV8_DEBUG`` set (to anything but
+``0``), every append, decode and step first runs ``kv8_check_indices`` on
+the indices it is given (slots; block tables and context lengths) and raises
+``ValueError`` instead of launching when any is out of range.  The calls
+themselves trust those indices.
 """
 from __future__ import annotations
+
+import os
 
 import torch
 
 from . import _binding as B
+
+
+def debug_checks_enabled() -> bool:
+    return os.environ.get("KV8_DEBUG", "") not in ("", "0")
+
+
+def check_indices(num_blocks: int, block_tables=None, context_lens=None,
+                  max_context_len: int = 0, slot_mapping=None, stream=None) -> None:
+    """Raise ValueError if kv8_check_indices finds an index out of range."""
+    bad = B.kv8_check_indices(block_tables, context_lens, max_context_len,
+                              num_blocks, slot_mapping=slot_mapping, stream=stream)
+    if any(bad):
+        raise ValueError(
+            f"KV8_DEBUG: {bad[0]} context lengths outside [0, {max_context_len}], "
+            f"{bad[1]} block-table entries outside [0, {num_blocks}), "
+            f"{bad[2]} slots past the cache's {num_blocks * 16}")
 
 
 class PagedKV8Cache:
@@ -44,6 +68,8 @@ class PagedKV8Cache:
 
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor,
                slot_mapping: torch.Tensor, stream=None) -> None:
+        if debug_checks_enabled():
+            check_indices(self.num_blocks, slot_mapping=slot_mapping, stream=stream)
         B.kv8_quantize_append(k_new, v_new, slot_mapping, self.k_cache,
                               self.v_cache, self.k_scales, self.v_scales,
                               stream=stream)
@@ -66,6 +92,9 @@ class PagedKV8Cache:
                stream=None) -> torch.Tensor:
         """One decode step over this cache; ``form`` picks the decode form
         for this call (KV8_FORM_AUTO: the library's default)."""
+        if debug_checks_enabled():
+            check_indices(self.num_blocks, block_tables, context_lens,
+                          max_context_len, stream=stream)
         if out is None:
             out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
         ws = self.workspace(q.shape[0], q.shape[1], max_context_len, chunk_tokens)
@@ -84,6 +113,9 @@ class PagedKV8Cache:
         """One decode step in one launch: sequence b's new K/V (bf16
         [B, H_kv, D]) join the cache at position context_lens[b] - 1, then
         every query head attends over the whole context."""
+        if debug_checks_enabled():
+            check_indices(self.num_blocks, block_tables, context_lens,
+                          max_context_len, stream=stream)
         if out is None:
             out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
         ws = self.workspace(q.shape[0], q.shape[1], max_context_len, chunk_tokens)
