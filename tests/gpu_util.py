@@ -77,3 +77,38 @@ def assert_close(gpu: np.ndarray, ref: np.ndarray, bf16: bool, tol=2e-3):
     assert not bad.any(), (
         f"{int(bad.sum())} elements outside tolerance; max err {err.max():.3e}")
     return float(err.max())
+
+
+def oracle_kivi_sequence(oracle, w: W.Workload, b: int):
+    """The oracle's private KIVI cache for sequence b (contiguously numbered
+    blocks), built as the fill and step calls build a device cache: every
+    token but the last, then the last.  Returns (cache, table)."""
+    k, v = w.sequence_kv(b)
+    n = k.shape[0]
+    nblk = max(1, math.ceil(n / w.block_size))
+    table = np.arange(nblk, dtype=np.int32)[None, :]
+    c = oracle.KiviCache(nblk, w.num_kv_heads, 1)
+    if n > 1:
+        oracle.kivi_append(c, k[:-1], v[:-1], np.array([0, n - 1]),
+                           np.array([n - 1]), table)
+    if n > 0:
+        oracle.kivi_append(c, k[-1:], v[-1:], np.array([0, 1]), np.array([n]),
+                           table)
+    return c, table
+
+
+def oracle_int4_sequence(oracle, w: W.Workload, b: int):
+    """The oracle's private INT4 cache for sequence b (contiguously numbered
+    blocks): (k codes, v codes, k scales, v scales, table)."""
+    k, v = w.sequence_kv(b)
+    n = k.shape[0]
+    nblk = max(1, math.ceil(n / w.block_size))
+    shape = (nblk, w.num_kv_heads, w.block_size, w.head_dim // 2)
+    kc = np.zeros(shape, dtype=np.uint8)
+    vc = np.zeros(shape, dtype=np.uint8)
+    ks = np.zeros(shape[:3], dtype=np.float32)
+    vs = np.zeros(shape[:3], dtype=np.float32)
+    slots = np.arange(n, dtype=np.int64)
+    oracle.quantize_append_int4(k, slots, kc, ks)
+    oracle.quantize_append_int4(v, slots, vc, vs)
+    return kc, vc, ks, vs, np.arange(nblk, dtype=np.int32)[None, :]

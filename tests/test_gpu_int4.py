@@ -10,6 +10,8 @@
   * groups of 8 (two sub-groups of 4 heads per KV head): the prefix-shared
     70B batch and ragged contexts.
 """
+import itertools
+
 import numpy as np
 import pytest
 
@@ -60,13 +62,13 @@ def _segments(w):
     return list(w.fill_segments()) + [w.step_tokens()]
 
 
-def _device_int4(pk, w):
+def _device_int4(pk, w, segments=None):
     shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim // 2)
     kc = torch.full(shape, POISON_BYTE, dtype=torch.uint8, device="cuda")
     vc = torch.full(shape, POISON_BYTE, dtype=torch.uint8, device="cuda")
     ks = torch.full(shape[:3], float("nan"), dtype=torch.float32, device="cuda")
     vs = torch.full(shape[:3], float("nan"), dtype=torch.float32, device="cuda")
-    for k, v, s in _segments(w):
+    for k, v, s in (_segments(w) if segments is None else segments):
         if s.shape[0] == 0:
             continue
         kt = torch.from_numpy(k).view(torch.bfloat16).cuda()
@@ -139,3 +141,41 @@ def test_int4_decode_all_pairs(built, oracle_mod, name, chunk_tokens, out_dtype)
     U.assert_close(gpu, ref, bf16=(out_dtype == "bf16"))
     if out_dtype == "f32":
         assert np.abs(gpu - ref).max() < 1e-4
+
+
+@pytest.fixture(scope="module")
+def big_int4(built):
+    _cache.clear()
+    torch.cuda.empty_cache()
+    w = W.llama8b_b64_32k()
+    dev = _device_int4(built, w, itertools.chain(w.fill_segments(), [w.step_tokens()]))
+    yield w, dev
+    del dev
+    torch.cuda.empty_cache()
+
+
+BIG_SEQS = [0, 37, 63]
+
+
+def test_big_int4_sampled_sequences(built, oracle_mod, big_int4):
+    """The batch-64 x 32K workload in the bench's launch (chunk 512): the
+    sampled sequences' packed codes and scales bit-exact against a private
+    oracle cache of each, and their output rows within the decode
+    tolerance."""
+    w, dev = big_int4
+    kc, vc, ks, vs = dev
+    outs = {dt: _decode(built, w, dev, 512, dt) for dt in (torch.float32, torch.bfloat16)}
+    for b in BIG_SEQS:
+        t = int(w.context_lens[b])
+        assert t % 16 == 0  # every page of the workload is full
+        pkc, pvc, pks, pvs, table = U.oracle_int4_sequence(oracle_mod, w, b)
+        blocks = torch.from_numpy(w.block_tables[b, :t // 16].astype(np.int64)).cuda()
+        assert np.array_equal(kc[blocks].cpu().numpy(), pkc)
+        assert np.array_equal(vc[blocks].cpu().numpy(), pvc)
+        assert np.array_equal(_u32(ks[blocks].cpu().numpy()), _u32(pks))
+        assert np.array_equal(_u32(vs[blocks].cpu().numpy()), _u32(pvs))
+        ref = oracle_mod.decode_attention_int4(w.q()[b:b + 1], pkc, pvc, pks, pvs, table,
+                                               w.context_lens[b:b + 1])[0]
+        U.assert_close(outs[torch.float32][b], ref, bf16=False)
+        U.assert_close(outs[torch.bfloat16][b], ref, bf16=True)
+    assert all(np.all(np.isfinite(o)) for o in outs.values())

@@ -13,6 +13,8 @@
     heads, split (64, 512) and unsplit, ragged and empty contexts, shared
     prefixes, permuted block tables.
 """
+import itertools
+
 import numpy as np
 import pytest
 
@@ -117,11 +119,9 @@ def full_page_blocks(w):
         + [np.zeros(0, np.int32)])).astype(np.int64)
 
 
-def assert_same_cache(w, dev, oc):
-    cache, tail = dev
-    blocks = full_page_blocks(w)
-    got = unpack_records(cache.cpu().numpy()[blocks])
-    ref = [a[blocks] for a in oc.fields()]
+def assert_same_fields(got, ref):
+    """Unpacked records against the oracle's fields: codes and scales bit
+    for bit, zero points by value."""
     names = ("k codes", "k scales", "k zeros", "v codes", "v scales", "v zeros")
     for name, g, r in zip(names, got, ref):
         if name.endswith("zeros"):
@@ -130,6 +130,13 @@ def assert_same_cache(w, dev, oc):
             assert np.array_equal(g.view(np.uint32), r.view(np.uint32)), name
         else:
             assert np.array_equal(g, r), name
+
+
+def assert_same_cache(w, dev, oc):
+    cache, tail = dev
+    blocks = full_page_blocks(w)
+    got = unpack_records(cache.cpu().numpy()[blocks])
+    assert_same_fields(got, [a[blocks] for a in oc.fields()])
     t = tail.view(torch.int16).cpu().numpy().view(np.uint16)
     for b, n in enumerate(w.context_lens):
         f = int(n) % 16
@@ -196,6 +203,41 @@ def test_kivi_decode_all_pairs(pk, oracle_mod, name, chunk, out_dtype):
     U.assert_close(gpu, ref, bf16=(out_dtype == "bf16"))
     if out_dtype == "f32":
         assert np.abs(gpu - ref).max() < 1e-4
+
+
+@pytest.fixture(scope="module")
+def big_kivi(pk):
+    _cache.clear()
+    torch.cuda.empty_cache()
+    w = W.llama8b_b64_32k()
+    dev = device_kivi(pk, w, itertools.chain(w.kivi_fill_calls(), [w.kivi_step_call()]))
+    yield w, dev
+    del dev
+    torch.cuda.empty_cache()
+
+
+BIG_SEQS = [0, 37, 63]
+
+
+def test_big_kivi_sampled_sequences(pk, oracle_mod, big_kivi):
+    """The batch-64 x 32K workload, filled and decoded as the bench does
+    (one append call per sequence, the step's token, chunk 512): the sampled
+    sequences' page records bit-exact against a private oracle cache of each,
+    and their output rows within the decode tolerance."""
+    w, dev = big_kivi
+    cache, tail = dev
+    outs = {dt: _decode(pk, w, dev, 512, dt) for dt in (torch.float32, torch.bfloat16)}
+    for b in BIG_SEQS:
+        t = int(w.context_lens[b])
+        oc, table = U.oracle_kivi_sequence(oracle_mod, w, b)
+        blocks = torch.from_numpy(w.block_tables[b, :t // 16].astype(np.int64)).cuda()
+        assert_same_fields(unpack_records(cache[blocks].cpu().numpy()),
+                           [a[:t // 16] for a in oc.fields()])
+        ref = oracle_mod.kivi_decode_attention(w.q()[b:b + 1], oc, table,
+                                               w.context_lens[b:b + 1])[0]
+        U.assert_close(outs[torch.float32][b], ref, bf16=False)
+        U.assert_close(outs[torch.bfloat16][b], ref, bf16=True)
+    assert all(np.all(np.isfinite(o)) for o in outs.values())
 
 
 def test_kivi_rejects_bad_shapes(pk):

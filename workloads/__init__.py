@@ -30,6 +30,7 @@ groups of 8 sequences share a 4096-token prefix.
 from __future__ import annotations
 
 import math
+from collections import deque
 from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
@@ -206,15 +207,17 @@ class Workload:
         return k, v, slots
 
     # ----------------------------------------------------------- KIVI fill
-    def kivi_fill_calls(self):
+    def kivi_fill_calls(self, threads: int = 8):
         """Append calls that put every token but each sequence's last into a
-        KIVI cache, one call per sequence so that host memory stays at one
-        sequence's rows: yields (k, v, cu_new [B+1], context_lens [B]) with
-        only sequence b's rows.  A shared prefix is appended by its group's
-        first member only (its blocks are shared; the prefix is a whole
-        number of pages), the other members start after it."""
+        KIVI cache, one call per sequence: yields (k, v, cu_new [B+1],
+        context_lens [B]) with only sequence b's rows, in sequence order.  A
+        shared prefix is appended by its group's first member only (its
+        blocks are shared; the prefix is a whole number of pages), the other
+        members start after it.  Up to ``threads`` sequences are drawn ahead
+        on a thread pool, so host memory holds that many sequences' rows."""
         B = self.batch
         seen = set()
+        jobs = []
         for b in range(B):
             n = max(int(self.context_lens[b]) - 1, 0)
             lo = 0
@@ -223,14 +226,28 @@ class Workload:
                 lo = self.prefix_len if grp in seen else 0
                 seen.add(grp)
             lo = min(lo, n)
-            if n == lo:
-                continue
+            if n > lo:
+                jobs.append((b, lo, n))
+
+        def work(job):
+            b, lo, n = job
             k, v = self.sequence_kv(b)
             cu = np.zeros(B + 1, np.int32)
             cu[b + 1:] = n - lo
             cl = np.zeros(B, np.int32)
             cl[b] = n
-            yield k[lo:n], v[lo:n], cu, cl
+            return k[lo:n], v[lo:n], cu, cl
+
+        ahead = max(1, threads)
+        with ThreadPoolExecutor(max_workers=ahead) as ex:
+            pending = deque(ex.submit(work, j) for j in jobs[:ahead])
+            nxt = ahead
+            while pending:
+                res = pending.popleft().result()
+                if nxt < len(jobs):
+                    pending.append(ex.submit(work, jobs[nxt]))
+                    nxt += 1
+                yield res
 
     def kivi_step_call(self):
         """The decode step's append call: each sequence's last token
