@@ -7,7 +7,8 @@ extend attention, through the C ABI.
     lengths that end inside a page and inside a key tile; every GQA group
     size; fp32 and bf16 output, |gpu - oracle| <= 2e-3 (+ half a bf16 ulp);
   * one new row per sequence agrees with the decode entry point;
-  * a 4096-token cache extended by 1000 rows (many key and query tiles).
+  * a 4096-token cache extended by 1000 rows (many key and query tiles);
+  * the extend bench's own workload at full size, sampled rows.
 """
 import numpy as np
 import pytest
@@ -87,3 +88,22 @@ def test_extend_long(pk, oracle_mod):
             qh[i:i + 1], kc, vc, ks, vs, w.block_tables,
             np.array([4096 - 1000 + i + 1], dtype=np.int32), np.array([0, 1]))
         U.assert_close(got[i:i + 1], sub, bf16=False)
+
+
+def test_extend_bench_size_sampled_rows(pk, oracle_mod):
+    """The extend bench's workload at full size (batch 4, 32768 cached
+    tokens each, the last 2048 new; q drawn as the bench draws it): sampled
+    rows of two sequences, all heads, against the oracle one row at a time
+    (row i of sequence b sees the first 32768 - 2048 + i + 1 tokens)."""
+    T, NEW = 32768, 2048
+    w = W.make_workload("llama8b_extend_b4_ctx32k_new2k", 1006, [T] * 4, 32, 8)
+    got, qh, qs, _ = _extend(pk, w, [NEW] * 4, 1006)
+    kc, vc, ks, vs = U.oracle_full_cache(oracle_mod, w)
+    for b in (0, 3):
+        for i in (0, 1023, NEW - 1):
+            r = int(qs[b]) + i
+            sub = oracle_mod.extend_attention(
+                qh[r:r + 1], kc, vc, ks, vs, w.block_tables[b:b + 1],
+                np.array([T - NEW + i + 1], dtype=np.int32), np.array([0, 1]))
+            U.assert_close(got[r:r + 1], sub, bf16=False)
+    assert np.all(np.isfinite(got))
