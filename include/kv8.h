@@ -508,6 +508,7 @@ KV8_API int32_t kv8_int4_paged_decode_attention(
 /*
  * kv8_check_indices -- debug check of the device-resident indices the other
  * calls trust (they are the caller's contract and are not checked there).
+ * A debug aid with no counterpart on the pages.
  * Counts, into counts[0..2] (device uint32, zeroed by the call first):
  *   counts[0]  sequences with context_lens[b] < 0 or > max_context_len
  *   counts[1]  block-table entries a decode would read (the first
