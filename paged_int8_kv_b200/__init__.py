@@ -32,8 +32,9 @@ _BINDING_NAMES = {
     "kv8_status_string",
 }
 _RUNTIME_NAMES = {"PagedKV8Cache", "fill_from_host"}
+_BLOCK_NAMES = {"BlockAllocator", "OutOfBlocks"}
 
-__all__ = sorted(_BINDING_NAMES | _RUNTIME_NAMES)
+__all__ = sorted(_BINDING_NAMES | _RUNTIME_NAMES | _BLOCK_NAMES)
 
 
 def __getattr__(name):
@@ -41,4 +42,6 @@ def __getattr__(name):
         return getattr(importlib.import_module("._binding", __name__), name)
     if name in _RUNTIME_NAMES:
         return getattr(importlib.import_module(".runtime", __name__), name)
+    if name in _BLOCK_NAMES:
+        return getattr(importlib.import_module(".blocks", __name__), name)
     raise AttributeError(f"module {__name__!r} has no attribute {name!r}")
