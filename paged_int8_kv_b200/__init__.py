@@ -31,7 +31,7 @@ _BINDING_NAMES = {
     "kv8_read_device_status", "kv8_split_reduce",
     "kv8_status_string",
 }
-_RUNTIME_NAMES = {"PagedKV8Cache", "fill_from_host"}
+_RUNTIME_NAMES = {"PagedKV8Cache", "PagedKiviCache", "fill_from_host"}
 _BLOCK_NAMES = {"BlockAllocator", "OutOfBlocks"}
 
 __all__ = sorted(_BINDING_NAMES | _RUNTIME_NAMES | _BLOCK_NAMES)

@@ -126,6 +126,68 @@ class PagedKV8Cache:
             softmax_scale=softmax_scale, stream=stream)
 
 
+class PagedKiviCache:
+    """Device memory of one layer's KIVI cache: the page records
+    (uint8 [num_blocks, H_kv, KV8_KIVI_PAGE_BYTES]) and the bf16 tail of each
+    batch row's partial page ([batch, H_kv, 2, 16, 128]); forwards to
+    kv8_kivi_append and kv8_kivi_paged_decode_attention."""
+
+    def __init__(self, num_blocks: int, num_kv_heads: int, batch: int,
+                 head_dim: int = 128, block_size: int = 16,
+                 device: str | torch.device = "cuda"):
+        self.num_blocks = int(num_blocks)
+        self.num_kv_heads = int(num_kv_heads)
+        self.batch = int(batch)
+        self.head_dim = int(head_dim)
+        self.block_size = int(block_size)
+        self.device = torch.device(device)
+        self.records = torch.zeros((self.num_blocks, self.num_kv_heads,
+                                    B.KV8_KIVI_PAGE_BYTES), dtype=torch.uint8,
+                                   device=self.device)
+        self.tail = torch.zeros((self.batch, self.num_kv_heads, 2,
+                                 self.block_size, self.head_dim),
+                                dtype=torch.bfloat16, device=self.device)
+        self._ws = None
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor,
+               cu_new: torch.Tensor, context_lens: torch.Tensor,
+               block_tables: torch.Tensor, max_new_tokens: int,
+               stream=None) -> None:
+        """Batch row b's new rows are k_new/v_new[cu_new[b] : cu_new[b+1]],
+        at its last positions (context_lens counts them)."""
+        if debug_checks_enabled():
+            check_indices(self.num_blocks, block_tables, context_lens,
+                          block_tables.shape[1] * self.block_size, stream=stream)
+        B.kv8_kivi_append(k_new, v_new, cu_new, context_lens, block_tables,
+                          self.records, self.tail, max_new_tokens, stream=stream)
+
+    def workspace(self, batch: int, num_q_heads: int, max_context_len: int,
+                  chunk_tokens: int) -> torch.Tensor | None:
+        need = B.kv8_decode_workspace_bytes(batch, num_q_heads, self.head_dim,
+                                            max_context_len, chunk_tokens)
+        if need == 0:
+            return None
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def decode(self, q: torch.Tensor, block_tables: torch.Tensor,
+               context_lens: torch.Tensor, max_context_len: int,
+               chunk_tokens: int = 512, out: torch.Tensor | None = None,
+               out_dtype: torch.dtype = torch.bfloat16,
+               softmax_scale: float = 0.0, stream=None) -> torch.Tensor:
+        if debug_checks_enabled():
+            check_indices(self.num_blocks, block_tables, context_lens,
+                          max_context_len, stream=stream)
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        ws = self.workspace(q.shape[0], q.shape[1], max_context_len, chunk_tokens)
+        return B.kv8_kivi_paged_decode_attention(
+            q, self.records, self.tail, block_tables, context_lens, out,
+            max_context_len, chunk_tokens=chunk_tokens, workspace=ws,
+            softmax_scale=softmax_scale, stream=stream)
+
+
 def fill_from_host(cache: PagedKV8Cache, segments, stream=None) -> int:
     """Copy host (k, v, slot_mapping) segments to the GPU and append them.
 

@@ -84,3 +84,33 @@ def test_bad_indices_raise_before_launch(rt, monkeypatch):
     with pytest.raises(ValueError, match="3 slots"):
         cache.append(kv, kv, torch.zeros(2, dtype=torch.int64))
     assert all(c[0] == "check" for c in calls)
+
+
+def test_kivi_runtime_forwards_and_checks(rt, monkeypatch):
+    runtime, _, calls, verdict = rt
+    seen = []
+
+    def rec(name):
+        def f(*a, **k):
+            seen.append((name, a, k))
+            return a[5] if name == "decode" else None
+        return f
+    monkeypatch.setattr(runtime.B, "kv8_kivi_append", rec("append"))
+    monkeypatch.setattr(runtime.B, "kv8_kivi_paged_decode_attention", rec("decode"))
+    c = runtime.PagedKiviCache(8, 2, 2, device="cpu")
+    assert c.records.shape == (8, 2, 2176) and c.tail.shape == (2, 2, 2, 16, 128)
+    q, bt, cl, kv = _args()
+    cu = torch.tensor([0, 1, 2], dtype=torch.int32)
+    monkeypatch.delenv("KV8_DEBUG", raising=False)
+    c.append(kv, kv, cu, cl, bt, 1)
+    out = c.decode(q, bt, cl, 64, chunk_tokens=0, out_dtype=torch.float32)
+    assert [s[0] for s in seen] == ["append", "decode"] and not calls
+    assert seen[0][1][5] is c.records and seen[0][1][6] is c.tail
+    assert seen[1][1][1] is c.records and out.dtype == torch.float32
+    monkeypatch.setenv("KV8_DEBUG", "1")
+    verdict["bad"] = (0, 1, 0)
+    with pytest.raises(ValueError):
+        c.decode(q, bt, cl, 64, chunk_tokens=0)
+    with pytest.raises(ValueError):
+        c.append(kv, kv, cu, cl, bt, 1)
+    assert len(seen) == 2
