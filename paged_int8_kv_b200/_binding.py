@@ -277,8 +277,10 @@ def kv8_check_indices(block_tables: torch.Tensor | None,
     [0, max_context_len], block-table entries a decode would read outside
     [0, num_blocks), slots at or past num_blocks * 16), after synchronising
     the stream."""
-    dev = next(t.device for t in (block_tables, context_lens, slot_mapping)
-               if t is not None)
+    given = [t for t in (block_tables, context_lens, slot_mapping) if t is not None]
+    if not given:
+        raise ValueError("kv8_check_indices: nothing to check")
+    dev = given[0].device
     counts = torch.zeros(3, dtype=torch.int32, device=dev)
     batch = 0 if context_lens is None else context_lens.shape[0]
     mbs = 1 if block_tables is None else block_tables.shape[1]

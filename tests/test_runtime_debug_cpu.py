@@ -114,3 +114,11 @@ def test_kivi_runtime_forwards_and_checks(rt, monkeypatch):
     with pytest.raises(ValueError):
         c.append(kv, kv, cu, cl, bt, 1)
     assert len(seen) == 2
+
+
+def test_check_indices_needs_something_to_check():
+    from paged_int8_kv_b200 import build
+    build.build()
+    from paged_int8_kv_b200 import _binding
+    with pytest.raises(ValueError):
+        _binding.kv8_check_indices(None, None, 0, 8)
