@@ -16,7 +16,8 @@ precision].  Pins:
     evenly spaced levels of their own are reconstructed exactly -- which
     fails if an axis is swapped, since the spacings differ along the other
     axis;
-  * constant groups (s = 0);
+  * constant groups (s = 0); a context whose tokens all carry one key
+    gives the plain mean of its values (pages and tail alike);
   * attention over pages built that way, plus bf16 tail rows, equals torch
     SDPA in float64 on the original K/V, for g in {1, 2, 4, 8}, ragged
     contexts and permuted block tables;
@@ -288,3 +289,27 @@ def test_kivi_bad_args(oracle_mod):
     with pytest.raises(ValueError):
         oracle_mod.kivi_append(c2, y16, y16, np.array([0, 16]), np.array([16]), bt)
     assert math.isnan(float(c2.k_scale[0, 0, 0]))
+
+
+def test_kivi_uniform_weights_give_the_mean(oracle_mod):
+    # every token carries the same key (a constant channel quantises to its
+    # zero point exactly, and the tail keeps bf16), so every weight is 1/n
+    # and the output is the plain mean of the values, pages and tail alike
+    rng = np.random.default_rng(78)
+    hkv, hq, n = 2, 4, 40
+    key = bf16_bits_to_f32(f32_to_bf16_bits(rng.standard_normal((hkv, D)).astype(np.float32)))
+    k = np.broadcast_to(key, (n, hkv, D)).copy()
+    v = np.empty((n, hkv, D), np.float32)
+    for p in range(n // BS):
+        ev = rng.integers(-9, -3, size=(BS, hkv)).astype(np.float64)
+        v[p * BS:(p + 1) * BS] = _levels(rng, (BS, hkv, D), ev, 2)[0]
+    f = n // BS * BS
+    v[f:] = bf16_bits_to_f32(f32_to_bf16_bits(rng.standard_normal((n - f, hkv, D)).astype(np.float32)))
+    c = oracle_mod.KiviCache(4, hkv, 1)
+    table = np.array([[2, 0, 3]], np.int32)
+    oracle_mod.kivi_append(c, _bits(k), _bits(v), np.array([0, n]), np.array([n]), table)
+    q = f32_to_bf16_bits(rng.standard_normal((1, hq, D)).astype(np.float32))
+    out = oracle_mod.kivi_decode_attention(q, c, table, np.array([n]))
+    mean = v.astype(np.float64).mean(axis=0)            # [hkv, D]
+    for h in range(hq):
+        np.testing.assert_allclose(out[0, h], mean[h // (hq // hkv)], rtol=1e-12, atol=1e-14)
